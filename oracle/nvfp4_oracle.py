@@ -1,0 +1,458 @@
+"""CPU oracle for the NVFP4 quantised linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, calls or links
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may use it.  It
+shares no code, table or constant generator with the CUDA library; the two
+meet only through the seeded synthetic inputs and the stored-layout definitions
+(packed E2M1 nibbles, UE4M3 bytes) that both must honour.
+
+What it computes, and where it comes from
+-----------------------------------------
+Source pages (all cited by title and passage):
+
+* [NVFP4-12B] "Preentrenamiento de 4 bits con NVFP4 en un híbrido
+  Mamba-Transformer de 12B (10T tokens)" (q2bstudio blog, NVIDIA 4-bit
+  pretraining summary).  Its format passage: NVFP4 stores 4-bit elements in
+  blocks of 16 with one E4M3 scale per block and one extra FP32 scale per
+  tensor, so that at least one value in sixteen (the block maximum, 6.25 %) is
+  held with near-FP8 precision.  Its recipe passage: 16x16 random Hadamard
+  transforms on the weight-gradient operands, two-dimensional block scaling
+  for weights, stochastic rounding on gradients only; NVFP4 only inside the
+  GEMMs of linear layers.  Its performance passage: FP4 GEMMs, half the operand
+  memory of FP8.
+* [Full-Stack FP4] "Full-Stack FP4: Preentrenamiento Estable de LLM": error
+  accumulates fast in low-precision matrix products (so the oracle and the
+  kernels accumulate in FP32 or wider).
+
+The pages give no equations.  The readings below are this library's, each
+stated where it is used:
+
+1. E2M1 element magnitudes are {0, 0.5, 1, 1.5, 2, 3, 4, 6} (3-bit index, plus
+   a sign bit: code = sign<<3 | index).  Round-to-nearest with ties to the even
+   index, saturating at 6; the sign of a value that rounds to zero is kept.
+2. The per-tensor FP32 decode scale is S = amax / (6 * 448): the tensor maximum
+   lands on the largest element magnitude (6) times the largest E4M3 scale
+   (448).  amax == 0 gives S = 1.
+3. Block scale s = E4M3(round-to-nearest-even, saturating at 448) of
+   (b / 6) / S, b the block's absolute maximum; every FP32 step is one IEEE
+   round-to-nearest operation, in exactly the order written here.
+4. Encode: d = s * S, r = 1 / d, y = x * r, code = E2M1(y).  A block with s == 0,
+   d == 0 or a non-finite r stores all-zero codes.
+5. Stochastic rounding (gradients): with lo <= |y| < hi adjacent grid points,
+   round up iff u < (|y| - lo) / (hi - lo), u = (w >> 8) * 2**-24 and w a 32-bit
+   Philox4x32-10 word; |y| >= 6 gives 6.
+6. Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy
+   as 1, 2, 3", SC'11): key = (seed lo32, seed hi32); counter =
+   (i/4 lo32, i/4 hi32, layout tag (0 row, 1 col), offset lo32); w = word i%4,
+   i the element's linear index in the layout it is stored in.
+7. The 16-point random Hadamard transform of a group g: v = D g (D = diag of
+   +-1 from a 16-bit sign mask, bit j set -> element j negated), then the
+   Walsh-Hadamard butterfly in stages h = 1, 2, 4, 8 ((a, b) -> (a+b, a-b) for
+   the pair (i, i+h) with bit h of i clear), then v * 0.25, which makes the
+   16x16 transform orthonormal.  Its tensor scale uses the amax of the
+   transformed values.
+8. Layouts: "row" = blocks of 16 along the contiguous (last) axis of an
+   [R x C] tensor, codes [R][C/2], scales [R][C/16]; "col" = blocks of 16 along
+   the first axis, stored transposed: codes [C][R/2], scales [C][R/16].  Two
+   codes per byte, low nibble = even element index.
+9. 2D weight blocks: one scale per 16x16 tile from the tile maximum; the row
+   and col layouts hold the same codes and scales, transposed.
+10. GEMM reference: C = A_hat . B_hat^T in FP64 from the dequantised FP32
+    operands x_hat = (code * s) * S.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+F32 = np.float32
+U32 = np.uint32
+U64 = np.uint64
+
+# E2M1 magnitude of each 3-bit index (reading 1).
+E2M1_MAGNITUDES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
+E2M1_MAX = 6.0
+E4M3_MAX = 448.0
+TENSOR_SCALE_DIVISOR = F32(E2M1_MAX * E4M3_MAX)  # 2688
+
+# ---------------------------------------------------------------------------
+# bfloat16 <-> float32 (host representation of the BF16 inputs)
+# ---------------------------------------------------------------------------
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """BF16 bit patterns (uint16) -> float32, exact (BF16 is the top half of FP32)."""
+    return (np.asarray(bits, dtype=np.uint16).astype(U32) << U32(16)).view(F32)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> BF16 bit patterns, round to nearest even (finite inputs)."""
+    b = np.asarray(x, dtype=F32).view(U32).astype(np.uint64)
+    rounded = (b + U64(0x7FFF) + ((b >> U64(16)) & U64(1))) >> U64(16)
+    return rounded.astype(np.uint16)
+
+
+# ---------------------------------------------------------------------------
+# E4M3 block scales (reading 3)
+# ---------------------------------------------------------------------------
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """Non-negative float -> E4M3 byte, round to nearest even, saturating at 448.
+
+    E4M3 (no infinities): bias 7, 3 mantissa bits.  Normal numbers are
+    (1 + m/8) * 2**(e-7) for exponent field e in 1..15 (e = 15, m = 7 is NaN and
+    never produced); subnormals are m * 2**-9.  Written from that definition:
+    the byte of a normal number is (e + 6) * 8 + q with q = v * 2**(3 - E) in
+    [8, 16) rounded half-to-even (q = 16 carries into the next binade, which the
+    formula absorbs); a subnormal's byte is round(v * 2**9).
+    """
+    v = np.asarray(v, dtype=np.float64)
+    if np.any(v < 0) or not np.all(np.isfinite(v)):
+        raise ValueError("block scales are non-negative and finite")
+    out = np.zeros(v.shape, dtype=np.int64)
+    sat = v >= E4M3_MAX
+    sub = v < 2.0 ** -6
+    nrm = ~sat & ~sub
+    out[sub] = np.rint(v[sub] * 2.0 ** 9).astype(np.int64)          # 0..8
+    if np.any(nrm):
+        mant, exp = np.frexp(v[nrm])                                  # v = mant * 2**exp, mant in [0.5, 1)
+        e_unb = exp - 1                                               # v = (2*mant) * 2**e_unb
+        q = np.rint(v[nrm] * np.exp2(3.0 - e_unb)).astype(np.int64)    # in [8, 16]
+        out[nrm] = (e_unb + 6) * 8 + q
+    out[sat] = 0x7E
+    out = np.minimum(out, 0x7E)
+    return out.astype(np.uint8)
+
+
+def e4m3_decode(b: np.ndarray) -> np.ndarray:
+    """E4M3 byte (sign bit clear, not NaN) -> float32 (exact)."""
+    b = np.asarray(b, dtype=np.int64)
+    e = b >> 3
+    m = b & 7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    return val.astype(F32)
+
+
+# ---------------------------------------------------------------------------
+# E2M1 elements (readings 1 and 5)
+# ---------------------------------------------------------------------------
+
+
+def e2m1_encode_rne(y: np.ndarray) -> np.ndarray:
+    """float32 -> 4-bit E2M1 code: nearest magnitude, ties to the even index, sign kept."""
+    y = np.asarray(y, dtype=F32)
+    # anything above 6 is nearest to 6; clamping first keeps the distances distinct
+    a = np.minimum(np.abs(y).astype(np.float64), E2M1_MAX)[..., None]
+    dist = np.abs(a - E2M1_MAGNITUDES)                    # [..., 8]
+    best = dist.min(axis=-1, keepdims=True)
+    cand = dist == best                                   # one or two adjacent candidates
+    # among tied candidates prefer the even index
+    even_pref = cand & ((np.arange(8) % 2) == 0)
+    has_even = even_pref.any(axis=-1)
+    idx = np.where(has_even, even_pref.argmax(axis=-1), cand.argmax(axis=-1))
+    sign = np.signbit(y).astype(np.uint8) << 3
+    return (idx.astype(np.uint8) | sign).astype(np.uint8)
+
+
+def e2m1_encode_sr(y: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """float32 -> E2M1 code with stochastic rounding driven by 32-bit words w."""
+    y = np.asarray(y, dtype=F32)
+    a = np.abs(y).astype(F32)
+    w = np.asarray(w, dtype=U32)
+    a64 = a.astype(np.float64)
+    lo_idx = np.searchsorted(E2M1_MAGNITUDES, a64, side="right") - 1   # largest grid point <= a
+    lo_idx = np.clip(lo_idx, 0, 7)
+    top = lo_idx >= 7
+    hi_idx = np.minimum(lo_idx + 1, 7)
+    lo = E2M1_MAGNITUDES[lo_idx].astype(F32)
+    step = (E2M1_MAGNITUDES[hi_idx] - E2M1_MAGNITUDES[lo_idx]).astype(F32)
+    step = np.where(top, F32(1.0), step).astype(F32)
+    frac = ((a - lo).astype(F32) / step).astype(F32)      # exact: Sterbenz, power-of-two step
+    u = ((w >> U32(8)).astype(F32) * F32(2.0 ** -24)).astype(F32)
+    up = (u < frac) & ~top
+    idx = np.where(top, 7, lo_idx + up.astype(np.int64))
+    sign = np.signbit(y).astype(np.uint8) << 3
+    return (idx.astype(np.uint8) | sign).astype(np.uint8)
+
+
+def e2m1_decode(code: np.ndarray) -> np.ndarray:
+    code = np.asarray(code, dtype=np.uint8)
+    mag = E2M1_MAGNITUDES[code & 7]
+    return np.where(code & 8, -mag, mag).astype(F32)
+
+
+# ---------------------------------------------------------------------------
+# Philox4x32-10 (reading 6)
+# ---------------------------------------------------------------------------
+
+PHILOX_M0 = 0xD2511F53
+PHILOX_M1 = 0xCD9E8D57
+PHILOX_W0 = 0x9E3779B9
+PHILOX_W1 = 0xBB67AE85
+
+
+def philox4x32_10(c0, c1, c2, c3, k0, k1):
+    """Philox4x32 with 10 rounds, vectorised over the counter words.
+
+    One round: (hi0, lo0) = M0 * c0, (hi1, lo1) = M1 * c2 (64-bit products);
+    new counter = (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0).  The key is bumped by
+    the Weyl constants (W0, W1) before every round after the first.
+    """
+    mask = U64(0xFFFFFFFF)
+    c = [np.asarray(v, dtype=U64) & mask for v in (c0, c1, c2, c3)]
+    c = list(np.broadcast_arrays(*c))
+    c = [v.copy() for v in c]
+    ka = np.asarray(k0, dtype=U64) & mask
+    kb = np.asarray(k1, dtype=U64) & mask
+    for rnd in range(10):
+        if rnd > 0:
+            ka = (ka + U64(PHILOX_W0)) & mask
+            kb = (kb + U64(PHILOX_W1)) & mask
+        p0 = U64(PHILOX_M0) * c[0]
+        p1 = U64(PHILOX_M1) * c[2]
+        hi0, lo0 = p0 >> U64(32), p0 & mask
+        hi1, lo1 = p1 >> U64(32), p1 & mask
+        c = [(hi1 ^ c[1] ^ ka) & mask, lo1, (hi0 ^ c[3] ^ kb) & mask, lo0]
+    return tuple(v.astype(U32) for v in c)
+
+
+def philox_words(first_index: int, count: int, seed: int, offset: int, tag: int) -> np.ndarray:
+    """Random word for each linear element index first_index .. first_index+count-1."""
+    if first_index % 4 or count % 4:
+        raise ValueError("element ranges are whole counters (multiples of 4)")
+    ctr = np.arange(first_index // 4, (first_index + count) // 4, dtype=U64)
+    w = philox4x32_10(ctr & U64(0xFFFFFFFF), ctr >> U64(32), np.full_like(ctr, tag),
+                      np.full_like(ctr, offset & 0xFFFFFFFF), seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
+    return np.stack(w, axis=-1).reshape(-1)
+
+
+# ---------------------------------------------------------------------------
+# 16-point random Hadamard transform (reading 7)
+# ---------------------------------------------------------------------------
+
+
+def rht16(g: np.ndarray, signs: int) -> np.ndarray:
+    """Apply the signed, normalised 16-point Walsh-Hadamard transform to the last axis."""
+    v = np.array(g, dtype=F32, copy=True)
+    if v.shape[-1] != 16:
+        raise ValueError("RHT groups have 16 elements")
+    flip = np.array([(signs >> j) & 1 for j in range(16)], dtype=bool)
+    v[..., flip] = -v[..., flip]
+    for h in (1, 2, 4, 8):
+        for i in range(16):
+            if i & h:
+                continue
+            a = v[..., i].copy()
+            b = v[..., i + h].copy()
+            v[..., i] = (a + b).astype(F32)
+            v[..., i + h] = (a - b).astype(F32)
+    return (v * F32(0.25)).astype(F32)
+
+
+# ---------------------------------------------------------------------------
+# Scales and block encoding (readings 2-5)
+# ---------------------------------------------------------------------------
+
+
+def tensor_scale(amax) -> np.float32:
+    amax = F32(amax)
+    if amax == 0:
+        return F32(1.0)
+    return F32(amax / TENSOR_SCALE_DIVISOR)
+
+
+def encode_blocks(vals: np.ndarray, bmax: np.ndarray, S: np.float32, words=None):
+    """Encode groups of 16 values that share one block scale.
+
+    vals : [..., 16] float32 values to encode (already transformed, if RHT);
+    bmax : [...] float32 absolute maximum that sets each group's scale (the
+           group's own maximum for 1D blocks, the 16x16 tile maximum for 2D);
+    words: None for round-to-nearest-even, else [..., 16] uint32 Philox words.
+    Returns (codes [..., 16] uint8 4-bit, scales [...] uint8 E4M3).
+    """
+    vals = np.asarray(vals, dtype=F32)
+    bmax = np.asarray(bmax, dtype=F32)
+    S = F32(S)
+    s_f = ((bmax / F32(6.0)).astype(F32) / S).astype(F32)
+    s = e4m3_encode(s_f)
+    d = (e4m3_decode(s) * S).astype(F32)
+    with np.errstate(divide="ignore", over="ignore"):
+        r = (F32(1.0) / d).astype(F32)
+    dead = (s == 0) | (d == 0) | ~np.isfinite(r)
+    r_safe = np.where(dead, F32(0.0), r).astype(F32)
+    y = (vals * r_safe[..., None]).astype(F32)
+    if words is None:
+        codes = e2m1_encode_rne(y)
+    else:
+        codes = e2m1_encode_sr(y, words)
+    codes = np.where(dead[..., None], np.uint8(0), codes).astype(np.uint8)
+    return codes, s
+
+
+def pack_codes(codes: np.ndarray) -> np.ndarray:
+    """[..., n] 4-bit codes -> [..., n/2] bytes, low nibble = even index."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_codes(packed: np.ndarray) -> np.ndarray:
+    packed = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = packed & 0xF
+    out[..., 1::2] = packed >> 4
+    return out
+
+
+def transformed_amax(v: np.ndarray, rht: bool, signs: int) -> np.float32:
+    """amax of a layout's values, [n_rows, n_cols] with blocks along the last axis."""
+    v = np.asarray(v, dtype=F32)
+    if rht:
+        g = rht16(v.reshape(v.shape[0], -1, 16), signs)
+        return F32(np.abs(g).max()) if g.size else F32(0.0)
+    return F32(np.abs(v).max()) if v.size else F32(0.0)
+
+
+def quantize_layout_rows(v: np.ndarray, row_ids, n_layout_cols: int, S, *, rht: bool, signs: int,
+                         stochastic: bool, seed: int, offset: int, tag: int):
+    """1D-quantise selected rows of one stored layout.
+
+    v       : [len(row_ids), n_layout_cols] float32, the layout's rows (rows of x for
+              the row layout, rows of x^T for the col layout);
+    row_ids : their row numbers in the layout (for the Philox element index).
+    Returns (codes [n, n_cols] 4-bit, scales [n, n_cols/16]).
+    """
+    v = np.asarray(v, dtype=F32)
+    n = v.shape[0]
+    g = v.reshape(n, n_layout_cols // 16, 16)
+    if rht:
+        g = rht16(g, signs)
+    bmax = np.abs(g).max(axis=-1).astype(F32)
+    words = None
+    if stochastic:
+        words = np.stack([philox_words(int(r) * n_layout_cols, n_layout_cols, seed, offset, tag)
+                          for r in np.asarray(row_ids).reshape(-1)])
+        words = words.reshape(n, n_layout_cols // 16, 16)
+    codes, s = encode_blocks(g, bmax, S, words)
+    return codes.reshape(n, n_layout_cols), s.reshape(n, n_layout_cols // 16)
+
+
+def quantize(x: np.ndarray, *, emit_row=True, emit_col=False, stochastic=False, rht_row=False,
+             rht_col=False, block_2d=False, seed=0, offset=0, rht_signs=0, amax_in=None):
+    """Quantise an [R x C] tensor (float32 values of BF16 inputs) to NVFP4.
+
+    Returns a dict with, per emitted layout ("row", "col"), a tuple
+    (packed codes uint8, scales uint8 canonical [rows][cols/16], S float32), plus
+    "amax": (raw amax, amax of the RHT-transformed col layout or None,
+    amax of the RHT-transformed row layout or None).
+    amax_in, when given, is (raw, rht) and replaces the computed maxima.
+    """
+    x = np.asarray(x, dtype=F32)
+    R, C = x.shape
+    if C % 16 or ((emit_col or block_2d) and R % 16):
+        raise ValueError("the blocked axis of every emitted layout is a multiple of 16")
+    if block_2d and (stochastic or rht_row or rht_col):
+        raise ValueError("2D weight blocks are round-to-nearest, untransformed")
+    out = {}
+    raw_amax = F32(np.abs(x).max()) if x.size else F32(0.0)
+    amax_row = raw_amax
+    amax_col = raw_amax
+    if rht_row:
+        amax_row = transformed_amax(x, True, rht_signs)
+    if rht_col:
+        amax_col = transformed_amax(x.T, True, rht_signs)
+    if amax_in is not None:
+        raw_amax = F32(amax_in[0])
+        amax_row = F32(amax_in[1]) if rht_row else raw_amax
+        amax_col = F32(amax_in[1]) if rht_col else raw_amax
+    out["amax"] = (raw_amax, amax_col if rht_col else None, amax_row if rht_row else None)
+
+    if block_2d:
+        S = tensor_scale(raw_amax)
+        tiles = x.reshape(R // 16, 16, C // 16, 16)
+        tmax = np.abs(tiles).max(axis=(1, 3)).astype(F32)                    # [R/16, C/16]
+        g = x.reshape(R, C // 16, 16)
+        bmax = np.repeat(tmax, 16, axis=0)                                   # [R, C/16]
+        codes, s = encode_blocks(g, bmax, S)
+        codes = codes.reshape(R, C)
+        if emit_row:
+            out["row"] = (pack_codes(codes), s.astype(np.uint8), S)
+        if emit_col:
+            # the same tiles read along the other axis: codes and tile scales transposed
+            s_tile = s[::16, :]                                              # [R/16, C/16]
+            out["col"] = (pack_codes(codes.T.copy()), np.repeat(s_tile.T, 16, axis=0).copy(), S)
+        return out
+
+    if emit_row:
+        S_r = tensor_scale(amax_row)
+        codes, s = quantize_layout_rows(x, np.arange(R), C, S_r, rht=rht_row, signs=rht_signs,
+                                        stochastic=stochastic, seed=seed, offset=offset, tag=0)
+        out["row"] = (pack_codes(codes), s, S_r)
+    if emit_col:
+        S_c = tensor_scale(amax_col)
+        codes, s = quantize_layout_rows(x.T.copy(), np.arange(C), R, S_c, rht=rht_col, signs=rht_signs,
+                                        stochastic=stochastic, seed=seed, offset=offset, tag=1)
+        out["col"] = (pack_codes(codes), s, S_c)
+    return out
+
+
+def dequantize(packed: np.ndarray, scales: np.ndarray, S) -> np.ndarray:
+    """x_hat = (code * s) * S in float32; code * s is exact."""
+    codes = unpack_codes(packed)
+    n, c = codes.shape
+    val = e2m1_decode(codes).reshape(n, c // 16, 16)
+    s = e4m3_decode(scales).reshape(n, c // 16, 1)
+    return ((val * s).astype(F32) * F32(S)).astype(F32).reshape(n, c)
+
+
+# ---------------------------------------------------------------------------
+# GEMM and the linear layer (reading 10)
+# ---------------------------------------------------------------------------
+
+
+def gemm_ref(a_hat: np.ndarray, b_hat: np.ndarray, alpha: float = 1.0) -> np.ndarray:
+    """C[m, n] = alpha * sum_k a_hat[m, k] * b_hat[n, k], in FP64."""
+    return float(alpha) * (np.asarray(a_hat, dtype=np.float64) @ np.asarray(b_hat, dtype=np.float64).T)
+
+
+def gemm_abs_ref(a_hat: np.ndarray, b_hat: np.ndarray, alpha: float = 1.0) -> np.ndarray:
+    """sum_k |a_k b_k| (times |alpha|): the scale of the GEMM tolerance bound."""
+    return abs(float(alpha)) * (np.abs(np.asarray(a_hat, dtype=np.float64)) @ np.abs(np.asarray(b_hat, dtype=np.float64)).T)
+
+
+def gemm_tolerance(a_hat, b_hat, alpha: float = 1.0) -> np.ndarray:
+    """|C - C_ref| <= 1e-5 * sum_k |a_k b_k| + 1e-6 (FP32 output)."""
+    return 1e-5 * gemm_abs_ref(a_hat, b_hat, alpha) + 1e-6
+
+
+def quantize_weight(w: np.ndarray):
+    """W [N x K] with 16x16 blocks: row layout for fprop, col layout (W^T, [K x N]) for dgrad."""
+    return quantize(w, emit_row=True, emit_col=True, block_2d=True)
+
+
+def linear_fwd_ref(x: np.ndarray, wq: dict, rht_signs: int = 0):
+    """Y = Q(X) Q(W)^T.  X [M x K] row-quantised with round-to-nearest; also returns
+    the col layout of X (RHT, round-to-nearest) that wgrad consumes."""
+    xq = quantize(x, emit_row=True, emit_col=True, rht_col=True, rht_signs=rht_signs)
+    a_hat = dequantize(*xq["row"])
+    b_hat = dequantize(*wq["row"])
+    return gemm_ref(a_hat, b_hat), (a_hat, b_hat), xq
+
+
+def linear_dgrad_ref(dy: np.ndarray, wq: dict, seed: int, offset: int, rht_signs: int = 0):
+    """dX = Q_sr(dY) Q(W): dY [M x N] row-quantised with stochastic rounding, W from
+    the col layout of its 2D quantisation ([K x N]); also returns dY's col layout
+    (RHT + stochastic rounding) for wgrad."""
+    dyq = quantize(dy, emit_row=True, emit_col=True, stochastic=True, rht_col=True,
+                   seed=seed, offset=offset, rht_signs=rht_signs)
+    a_hat = dequantize(*dyq["row"])
+    b_hat = dequantize(*wq["col"])
+    return gemm_ref(a_hat, b_hat), (a_hat, b_hat), dyq
+
+
+def linear_wgrad_ref(dyq: dict, xq: dict):
+    """dW = Q(H dY)^T Q(H X): both col layouts, contraction over tokens."""
+    a_hat = dequantize(*dyq["col"])
+    b_hat = dequantize(*xq["col"])
+    return gemm_ref(a_hat, b_hat), (a_hat, b_hat)
