@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 linear-layer training step on B200.
+
+One step = the whole hot path for both linears of the 12B-class hybrid
+Mamba-Transformer MLP shapes (tokens 16384, hidden 5120, FFN 20480: the
+up-projection W[20480 x 5120] and the down-projection W[5120 x 20480]):
+  quantise W (16x16 blocks, row + col layouts)
+  fprop:  quantise X (row, RNE; col with 16x16 RHT, RNE)   + GEMM  Y  = X W^T
+  dgrad:  quantise dY (row, SR; col with RHT + SR)          + GEMM  dX = dY W
+  wgrad:                                                      GEMM  dW = dY^T X
+Inputs are seeded synthetic BF16 tensors resident in HBM (each larger than the
+126 MB L2, so no flush is needed between steps).
+
+Prints one JSON line (rank 0).  `value` is the step's NVFP4 GEMM work (6 GEMMs,
+2MNK each) divided by the device time of the whole step, quantisers included.
+`e2e` is the same metric through the public C-ABI linear calls with the step's
+activations and gradients copied from pinned host memory and the weight
+gradients read back, inside the timed region.  `roofline` covers the dominant
+kernel (the GEMM) against the FP4 tensor peak; `quantizer` the HBM side.
+`--impl reference` times the CPU oracle on a bounded sample of the same step.
+Multi-GPU (torchrun): data parallel, each rank runs the full per-GPU step on its
+own tokens and the weight gradients are all-reduced with NCCL (weak scaling).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "NVFP4 GEMM TFLOPS & % FP4 peak; quantizer GB/s & % HBM (1×B200)"
+UNIT = "TFLOP/s"
+WORKLOAD = "hybrid12b-mlp-linear-step"
+FP4_OVER_BF16 = 4.0          # nominal dense ratio (9 / 2.25 PFLOP/s)
+RHT_SIGNS = 0x5A3C
+SR_SEED = 1234
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms (read-only query)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-i", uuid, "-lms", "200"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        self.t_start = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+
+class Linear:
+    """Buffers of one NVFP4 linear layer step (all device-resident, preallocated)."""
+
+    def __init__(self, name, x, w, dy):
+        from nvfp4_pretraining_linear_b200.api import QTensor, SCALE_MMA
+        self.name = name
+        self.x, self.w, self.dy = x, w, dy
+        M, K = x.shape
+        N = w.shape[0]
+        self.M, self.K, self.N = M, K, N
+        dev = x.device
+        self.wq_row = QTensor.empty(N, K, SCALE_MMA, dev)
+        self.wq_col = QTensor.empty(K, N, SCALE_MMA, dev)
+        self.xq_row = QTensor.empty(M, K, SCALE_MMA, dev)
+        self.xq_col = QTensor.empty(K, M, SCALE_MMA, dev)
+        self.dyq_row = QTensor.empty(M, N, SCALE_MMA, dev)
+        self.dyq_col = QTensor.empty(N, M, SCALE_MMA, dev)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        self.dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+
+    def gemm_flops(self):
+        return 3 * 2.0 * self.M * self.N * self.K
+
+    def quant_bytes(self):
+        # two-pass quantiser: 2 B/elem amax read + 2 B/elem quantise read + 0.5625 B/elem per layout
+        elems = self.M * self.K + self.N * self.K + self.M * self.N
+        return elems * (4.0 + 2 * 0.5625)
+
+
+def build_workload(device, rank):
+    from nvfp4_pretraining_linear_b200 import synthetic as syn
+    T, H, F = syn.HYBRID12B["tokens"], syn.HYBRID12B["hidden"], syn.HYBRID12B["ffn"]
+    s = 1000 * rank  # each data-parallel rank draws its own tokens
+    up = Linear("up", syn.normal((T, H), 1.0, seed=12 + s, device=device, outlier_frac=0.001, outlier_mult=100.0),
+                syn.normal((F, H), 0.014, seed=10, device=device),
+                syn.normal((T, F), 1e-3, seed=14 + s, device=device))
+    down = Linear("down", syn.normal((T, F), 1.0, seed=13 + s, device=device, outlier_frac=0.001, outlier_mult=100.0),
+                  syn.normal((H, F), 0.014, seed=11, device=device),
+                  syn.normal((T, H), 1e-3, seed=15 + s, device=device))
+    return [up, down]
+
+
+def instrumented_step(linears, ev, offset):
+    """One step from the quantiser and GEMM entry points, with CUDA events
+    bracketing each GEMM and each quantiser call (same kernels, same order as
+    the linear_fwd / linear_dgrad / linear_wgrad entry points)."""
+    from nvfp4_pretraining_linear_b200 import api
+    for L in linears:
+        ev.mark("q")
+        api.quantize(L.w, emit_row=True, emit_col=True, block_2d=True, out_row=L.wq_row, out_col=L.wq_col)
+        api.quantize(L.x, emit_row=True, emit_col=True, rht_col=True, rht_signs=RHT_SIGNS, out_row=L.xq_row,
+                     out_col=L.xq_col)
+        ev.mark("g")
+        api.gemm(L.xq_row, L.wq_row, out=L.y)
+        ev.mark("q")
+        api.quantize(L.dy, emit_row=True, emit_col=True, stochastic=True, rht_col=True, seed=SR_SEED, offset=offset,
+                     rht_signs=RHT_SIGNS, out_row=L.dyq_row, out_col=L.dyq_col)
+        ev.mark("g")
+        api.gemm(L.dyq_row, L.wq_col, out=L.dx)
+        api.gemm(L.dyq_col, L.xq_col, out=L.dw)
+    ev.mark("end")
+
+
+class PhaseEvents:
+    """Records an event at each phase boundary; sums device time per phase."""
+
+    def __init__(self, enabled=True):
+        self.enabled = enabled
+        self.marks = []
+
+    def mark(self, phase):
+        if not self.enabled:
+            return
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        self.marks.append((phase, e))
+
+    def totals(self):
+        out = {}
+        for (ph, e0), (_, e1) in zip(self.marks, self.marks[1:]):
+            if ph == "end":
+                continue
+            out[ph] = out.get(ph, 0.0) + e0.elapsed_time(e1)
+        return out
+
+
+def public_step(linears, offset, ws):
+    """One step through the public linear entry points (as a user calls them)."""
+    from nvfp4_pretraining_linear_b200 import api
+    for L in linears:
+        api.quantize(L.w, emit_row=True, emit_col=True, block_2d=True, out_row=L.wq_row, out_col=L.wq_col)
+        api.linear_fwd(L.x, L.wq_row, rht_signs=RHT_SIGNS, out=L.y, xq_row=L.xq_row, xq_col=L.xq_col)
+        api.linear_dgrad(L.dy, L.wq_col, seed=SR_SEED, offset=offset, rht_signs=RHT_SIGNS, out=L.dx,
+                         dyq_row=L.dyq_row, dyq_col=L.dyq_col)
+        api.linear_wgrad(L.dyq_col, L.xq_col, out=L.dw)
+
+
+LAUNCHES_PER_LINEAR = 2 + 2 + 1 + 2 + 1 + 1   # W quant (amax+quant), X quant, fprop, dY quant, dgrad, wgrad
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+
+
+def oracle_sample_step(state):
+    """The oracle on a bounded sample of the step: the up-projection linear restricted
+    to 64 tokens and 256 output features (full hidden width 5120)."""
+    from oracle import nvfp4_oracle as O
+    x, w, dy = state
+    wq = O.quantize_weight(w)
+    y, _, xq = O.linear_fwd_ref(x, wq, rht_signs=RHT_SIGNS)
+    dx, _, dyq = O.linear_dgrad_ref(dy, wq, seed=SR_SEED, offset=0, rht_signs=RHT_SIGNS)
+    dw, _ = O.linear_wgrad_ref(dyq, xq)
+    return y, dx, dw
+
+
+def oracle_sample_inputs():
+    from nvfp4_pretraining_linear_b200 import synthetic as syn
+    T, N, K = 64, 256, syn.HYBRID12B["hidden"]
+    x = syn.normal((T, K), 1.0, seed=12, device="cpu", outlier_frac=0.001, outlier_mult=100.0).float().numpy()
+    w = syn.normal((N, K), 0.014, seed=10, device="cpu").float().numpy()
+    dy = syn.normal((T, N), 1e-3, seed=14, device="cpu").float().numpy()
+    flops = 3 * 2.0 * T * N * K
+    return (x, w, dy), flops, "up-projection linear step restricted to 64 tokens x 256 outputs x 5120 hidden"
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def time_oracle(min_seconds=10.0, min_steps=3):
+    state, flops, desc = oracle_sample_inputs()
+    times = []
+    t_all = time.perf_counter()
+    while len(times) < min_steps or time.perf_counter() - t_all < min_seconds:
+        t0 = time.perf_counter()
+        oracle_sample_step(state)
+        times.append(time.perf_counter() - t0)
+        if len(times) >= 50:
+            break
+    t = statistics.median(times)
+    return {"value": flops / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": desc + "; median of %d steps, %.2f s each" % (len(times), t)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    state, flops, desc = oracle_sample_inputs()
+    for _ in range(args.warmup):
+        oracle_sample_step(state)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(state)
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantise / f64 GEMM",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "sample": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+
+
+def run_ours(args):
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    group = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        group = dist.group.WORLD
+    from nvfp4_pretraining_linear_b200 import api, _lib
+    from nvfp4_pretraining_linear_b200.parallel import allreduce_grads, sr_offset
+
+    peaks, peak_src = load_peaks()
+    linears = build_workload(device, rank)
+    ws = api.workspace(device)
+    offset = sr_offset(0, rank)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if group is not None:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    def device_step(ev):
+        instrumented_step(linears, ev, offset)
+        if group is not None:
+            allreduce_grads([L.dw for L in linears], group)
+
+    for _ in range(args.warmup):
+        device_step(PhaseEvents(False))
+    api.get_status()
+
+    # ---- device-timed region
+    evs = [PhaseEvents(True) for _ in range(args.steps)]
+    barrier()
+    clocks = ClockSampler(local)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(args.steps):
+        device_step(evs[i])
+    t_end.record()
+    barrier()
+    clock_info = clocks.stop()
+    api.get_status()
+    ms_total = t_start.elapsed_time(t_end)
+    if group is not None:
+        t = torch.tensor([ms_total], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    gemm_ms = sum(e.totals().get("g", 0.0) for e in evs) / args.steps
+    quant_ms = sum(e.totals().get("q", 0.0) for e in evs) / args.steps
+    flops = sum(L.gemm_flops() for L in linears)
+    qbytes = sum(L.quant_bytes() for L in linears)
+    value = flops * world / (ms_step * 1e-3) / 1e12
+
+    fp4_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP4_OVER_BF16
+    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+    quant_gbs = qbytes / (quant_ms * 1e-3) / 1e9
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    gemm_launches = 3 * len(linears)
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if os.path.exists(prof):
+        try:
+            with open(prof) as f:
+                traffic = json.load(f).get("bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    # ---- end to end through the public API, host buffers, copies inside the timed region
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    host_in = []
+    for L in linears:
+        host_in.append((L.x, torch.empty(L.x.shape, dtype=L.x.dtype, pin_memory=True)))
+        host_in.append((L.dy, torch.empty(L.dy.shape, dtype=L.dy.dtype, pin_memory=True)))
+    for dev_t, host_t in host_in:
+        host_t.copy_(dev_t)
+    host_out = [(L.dw, torch.empty(L.dw.shape, dtype=L.dw.dtype, pin_memory=True)) for L in linears]
+    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in host_out)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        for dev_t, host_t in host_in:
+            dev_t.copy_(host_t, non_blocking=True)
+        public_step(linears, offset, ws)
+        if group is not None:
+            allreduce_grads([L.dw for L in linears], group)
+        for dev_t, host_t in host_out:
+            host_t.copy_(dev_t, non_blocking=True)
+    e1.record()
+    barrier()
+    api.get_status()
+    e2e_ms = e0.elapsed_time(e1)
+    if group is not None:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = flops * world / (e2e_ms / e2e_steps * 1e-3) / 1e12
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3 block scales, fp32 accumulate), bf16 in/out",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tokens_per_gpu": linears[0].M, "hidden": linears[0].K,
+                       "ffn": linears[0].N, "linears": ["up 5120->20480", "down 20480->5120"],
+                       "gemms_per_step": gemm_launches, "parallelism": "dp%d" % world,
+                       "l2": "every input larger than the 126 MB L2; no flush"},
+            "gpu_launches": LAUNCHES_PER_LINEAR * len(linears) * args.steps,
+            "quantizer": {"gbs": quant_gbs, "frac_hbm": quant_gbs / hbm, "hbm_peak_gbs": hbm,
+                          "peak_source": peak_src, "ms_per_step": quant_ms,
+                          "bytes_per_elem": "4.5625 / layout-pair 5.125 (two-pass)"},
+            "gemm": {"tflops": gemm_tflops, "frac_fp4_peak": gemm_tflops / fp4_peak, "ms_per_step": gemm_ms},
+            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": gemm_tflops / fp4_peak, "traffic": traffic,
+                         "kernel": "nvfp4::gemm::gemm_kernel",
+                         "peak_source": "%s bf16 sustained x %.0f (nominal FP4/BF16 ratio), of %s" % (
+                             peak_src, FP4_OVER_BF16, peak_src)},
+            "clocks": clock_info,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps, "path": "nvfp4_linear_fwd/dgrad/wgrad via the C ABI, pinned host buffers"},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = time_oracle(args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if group is not None:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

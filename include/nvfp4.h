@@ -1,0 +1,207 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 quantised linear-layer library.
+ *
+ * The operation: the NVFP4 linear layer of 4-bit LLM pretraining, as described
+ * on the page "Preentrenamiento de 4 bits con NVFP4 en un hibrido
+ * Mamba-Transformer de 12B (10T tokens)" (NVIDIA method summary):
+ *   - format passage: 4-bit E2M1 elements in blocks of 16, one E4M3 scale per
+ *     block and one extra FP32 scale per tensor;
+ *   - scope passage: NVFP4 is used only inside the GEMMs of linear layers;
+ *   - recipe passage: 16x16 random Hadamard transforms on the weight-gradient
+ *     operands, two-dimensional (16x16) block scaling for weights, stochastic
+ *     rounding on gradients only;
+ *   - performance passage: FP4 GEMMs run at twice FP8's rate and halve the
+ *     operand memory.
+ *
+ * Conventions for every call
+ *   - Pointers named "device" point to GPU global memory of the current device;
+ *     everything else (structs, option blocks) is host memory read during the call.
+ *   - The caller owns every buffer and the stream.  The library allocates no
+ *     memory; calls that need scratch take a caller-supplied workspace.
+ *   - Calls enqueue work on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream) and return without synchronising.
+ *   - Argument errors are reported synchronously by the return value, before
+ *     anything is launched.  Device-side errors (a bounded wait that gave up)
+ *     are reported by nvfp4_get_status().  No exception crosses the ABI.
+ *   - nvfp4_last_error_string() describes the last non-OK status of the calling
+ *     thread.
+ *
+ * Stored format (every nvfp4_tensor)
+ *   - A logical [rows x cols] tensor blocked along cols (the contiguous axis).
+ *   - codes: [rows][cols/2] bytes, two 4-bit E2M1 codes per byte, the element
+ *     with the even column index in the low nibble.  Code = sign << 3 | index,
+ *     index into the magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+ *   - scales: one unsigned E4M3 byte per 16-element block, in one of two layouts:
+ *       NVFP4_SCALE_ROWMAJOR: [rows][cols/16], byte (r, j) at r*(cols/16) + j;
+ *       NVFP4_SCALE_MMA: tiles of 128 rows x 4 block-columns (512 bytes); tile
+ *         (r/128, j/4) at ((r/128) * ceil(cols/64) + j/4) * 512, and inside the
+ *         tile byte (r%32)*16 + ((r%128)/32)*4 + j%4.  This is the order in
+ *         which the tensor cores read block scales; nvfp4_gemm requires it.
+ *   - tensor_scale: one FP32 decode scale S on the device.  The value of element
+ *     (r, c) is E2M1(code) * E4M3(scale) * S.
+ *   - A "col" layout of an [R x C] tensor is the [C x R] tensor of its transpose,
+ *     blocked along R.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,       /* NULL where a buffer is needed, bad enum, bad option mix */
+  NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside the documented multiples */
+  NVFP4_ERR_MISALIGNED = 3,        /* pointer or leading dimension breaks 16-byte alignment */
+  NVFP4_ERR_CUDA = 4,              /* a CUDA runtime call failed (launch, attribute, ...) */
+  NVFP4_ERR_TIMEOUT = 5,           /* a device-side bounded wait gave up (nvfp4_get_status) */
+  NVFP4_ERR_WORKSPACE = 6          /* workspace missing or smaller than nvfp4_workspace_size() */
+} nvfp4_status;
+
+enum { NVFP4_SCALE_ROWMAJOR = 0, NVFP4_SCALE_MMA = 1 };
+enum { NVFP4_OUT_BF16 = 0, NVFP4_OUT_F32 = 1 };
+
+/* One NVFP4 tensor: see "Stored format" above.  All three buffers are device
+ * memory owned by the caller; sizes: codes rows*cols/2 bytes, scales
+ * nvfp4_scales_bytes(rows, cols, scale_layout) bytes, tensor_scale 4 bytes.
+ * An empty tensor (rows or cols 0) may leave codes and scales NULL. */
+typedef struct {
+  uint8_t* codes;
+  uint8_t* scales;
+  float* tensor_scale;
+  int64_t rows;
+  int64_t cols;
+  int32_t scale_layout; /* NVFP4_SCALE_ROWMAJOR or NVFP4_SCALE_MMA */
+  int32_t reserved;     /* must be 0 */
+} nvfp4_tensor;
+
+/* Quantiser options (recipe passage of the 12B NVFP4 page).
+ *   stochastic : stochastic rounding of the elements of every emitted layout
+ *                (gradients); otherwise round-to-nearest-even.  The random word
+ *                of element i of a layout is word i%4 of Philox4x32-10 with key
+ *                (seed lo32, seed hi32) and counter (i/4 lo32, i/4 hi32, tag,
+ *                offset), tag 0 for the row layout and 1 for the col layout;
+ *                the element rounds up iff (word >> 8) * 2^-24 is below its
+ *                fractional position between the two neighbouring magnitudes.
+ *   rht_row    : 16x16 random Hadamard transform along the blocks of the row layout.
+ *   rht_col    : the same along the blocks of the col layout (the token axis of
+ *                the weight-gradient operands).
+ *   block_2d   : one scale per 16x16 tile (weights); the row and col layouts then
+ *                hold the same codes and scales, transposed.  Excludes stochastic
+ *                and both RHT flags.
+ *   seed       : Philox key.
+ *   offset     : Philox counter word 3; must be < 2^32.
+ *   rht_signs  : low 16 bits; bit j set negates element j of every 16-group
+ *                before the transform.  Use the same value for both wgrad operands.
+ *   amax_in    : NULL, or 3 device floats {raw amax, amax of the transformed col
+ *                layout, amax of the transformed row layout} that replace the
+ *                amax pass (delayed or externally fused scaling).
+ *   amax_out   : NULL, or 3 device floats receiving the maxima used.
+ * The tensor scale of a layout is S = amax / (6 * 448) (S = 1 when amax = 0),
+ * with amax taken over the values that layout encodes (after its transform). */
+typedef struct {
+  int32_t stochastic;
+  int32_t rht_row;
+  int32_t rht_col;
+  int32_t block_2d;
+  uint64_t seed;
+  uint64_t offset;
+  uint32_t rht_signs;
+  uint32_t reserved; /* must be 0 */
+  const float* amax_in;
+  float* amax_out;
+} nvfp4_quant_opts;
+
+/* Library version, major*10000 + minor*100 + patch. */
+int nvfp4_version(void);
+
+/* Bytes of caller workspace that nvfp4_quantize and the linear calls need
+ * (device memory, 256-byte aligned; its contents need not be initialised). */
+size_t nvfp4_workspace_size(void);
+
+/* Bytes of the scale buffer of an NVFP4 tensor of logical shape [rows x cols]
+ * in the given layout (the MMA layout pads rows to 128 and cols/16 to 4). */
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t scale_layout);
+
+/* Quantise a BF16 tensor x [rows x cols] (device, row stride ld elements) to
+ * NVFP4 (format and recipe passages of the 12B NVFP4 page).
+ *   out_row : NULL, or the row layout, rows x cols (blocks along cols).
+ *   out_col : NULL, or the col layout, cols x rows (blocks along rows).
+ * At least one output.  Requires cols % 16 == 0; rows % 16 == 0 when out_col is
+ * given or block_2d is set; x and ld*2 bytes 16-byte aligned; codes buffers
+ * 16-byte aligned.  Work: one amax pass over x (skipped when amax_in is given)
+ * and one quantise pass writing every requested layout and its tensor scale. */
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                            const nvfp4_quant_opts* opts, nvfp4_tensor* out_row,
+                            nvfp4_tensor* out_col, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Dequantise q into out [rows x cols] (device, row stride ldo elements):
+ * out = E2M1(code) * E4M3(scale) * S, rounded to BF16 (nearest even) or kept
+ * in FP32.  Requires cols % 16 == 0 and 16-byte aligned out rows. */
+nvfp4_status nvfp4_dequantize(const nvfp4_tensor* q, void* out, int64_t ldo, int32_t out_dtype,
+                              void* stream);
+
+/* Block-scaled NVFP4 GEMM on the sm_100a tensor cores (performance passage of
+ * the 12B NVFP4 page; FP32 accumulation per the error-accumulation remark of
+ * "Full-Stack FP4: Preentrenamiento Estable de LLM"):
+ *   C[m][n] = alpha * S_A * S_B * sum_k A[m][k] * B[n][k]   (+ C[m][n] if accumulate)
+ * with A [M x K] and B [N x K] NVFP4 tensors blocked along K (MMA scale layout),
+ * C [M x N] device memory with row stride ldc elements, BF16 (nearest even) or FP32.
+ * Requires M % 128 == 0, N % 128 == 0, K % 64 == 0, 16-byte aligned C rows. */
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc,
+                        int32_t out_dtype, float alpha, int32_t accumulate, void* stream);
+
+/* Linear forward (fprop): Y [M x N] = Q(X) . Q(W)^T.
+ *   X      : BF16 [M x K] activations (device, row stride ldx), quantised here
+ *            row-wise with round-to-nearest-even into Xq_row (caller buffers,
+ *            MMA scale layout).
+ *   Wq_row : the row layout of the 2D-quantised weight W [N x K].
+ *   Xq_col : NULL, or buffers for the col layout of X (K x M, 16x16 RHT along
+ *            tokens with rht_signs, round-to-nearest-even) saved for wgrad,
+ *            produced by the same pass over X.
+ * Requires M % 128, N % 128, K % 64 == 0. */
+nvfp4_status nvfp4_linear_fwd(const void* X, int64_t M, int64_t K, int64_t ldx,
+                              const nvfp4_tensor* Wq_row, void* Y, int64_t ldy, int32_t out_dtype,
+                              nvfp4_tensor* Xq_row, nvfp4_tensor* Xq_col, uint32_t rht_signs,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Linear data gradient (dgrad): dX [M x K] = Q_sr(dY) . Q(W).
+ *   dY     : BF16 [M x N] output gradient (device, row stride ldy), quantised
+ *            row-wise with stochastic rounding (seed, offset) into dYq_row.
+ *   Wq_col : the col layout of the 2D-quantised weight ([K x N], the exact
+ *            transpose of Wq_row: no re-quantisation).
+ *   dYq_col: NULL, or buffers for dY's col layout (N x M, RHT along tokens +
+ *            stochastic rounding) saved for wgrad, from the same pass over dY.
+ * Requires M % 128, K % 128, N % 64 == 0. */
+nvfp4_status nvfp4_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ldy,
+                                const nvfp4_tensor* Wq_col, void* dX, int64_t ldx, int32_t out_dtype,
+                                nvfp4_tensor* dYq_row, nvfp4_tensor* dYq_col, uint64_t seed,
+                                uint64_t offset, uint32_t rht_signs, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* Linear weight gradient (wgrad): dW [N x K] = Q(H dY)^T . Q(H X), contracting
+ * over the M tokens.  dYq_col [N x M] and Xq_col [K x M] are the col layouts
+ * saved by nvfp4_linear_dgrad and nvfp4_linear_fwd with the same rht_signs, so
+ * the transforms cancel in the product.  accumulate adds into dW (gradient
+ * accumulation).  Requires N % 128, K % 128, M % 64 == 0. */
+nvfp4_status nvfp4_linear_wgrad(const nvfp4_tensor* dYq_col, const nvfp4_tensor* Xq_col, void* dW,
+                                int64_t ldw, int32_t out_dtype, int32_t accumulate, void* stream);
+
+/* Synchronise `stream`, then report and clear any device-side error recorded
+ * by this library's kernels on the current device since the last call
+ * (NVFP4_ERR_TIMEOUT), or a pending CUDA error (NVFP4_ERR_CUDA). */
+nvfp4_status nvfp4_get_status(void* stream);
+
+/* Text of the last non-OK status returned on the calling thread. */
+const char* nvfp4_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

@@ -1,0 +1,176 @@
+"""PyTorch-facing binding of the C ABI: the same entry points, with torch tensors.
+
+Only marshalling happens here -- buffers are torch CUDA tensors, the stream is
+torch's current stream, and every step of the computation runs in the CUDA
+library.  There is no CPU path: calls fail when the library or a GPU is missing.
+"""
+
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import OUT_BF16, OUT_F32, SCALE_MMA, SCALE_ROWMAJOR, NVFP4Error  # noqa: F401
+
+_workspaces = {}
+
+
+def _stream_ptr(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes_void(s.cuda_stream)
+
+
+def ctypes_void(v):
+    import ctypes
+    return ctypes.c_void_p(v)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def workspace(device=None, stream=None):
+    """A cached workspace buffer per (device, stream) for the quantiser's amax pass."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    key = (dev.index, s.cuda_stream)
+    ws = _workspaces.get(key)
+    if ws is None:
+        n = _lib.load().nvfp4_workspace_size()
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        _workspaces[key] = ws
+    return ws
+
+
+@dataclass
+class QTensor:
+    """An NVFP4 tensor: packed codes [rows, cols/2], block scales, FP32 tensor scale."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    tensor_scale: torch.Tensor
+    rows: int
+    cols: int
+    scale_layout: int = SCALE_MMA
+
+    def struct(self):
+        return _lib.NVFP4Tensor(self.codes.data_ptr(), self.scales.data_ptr(), self.tensor_scale.data_ptr(),
+                                self.rows, self.cols, self.scale_layout, 0)
+
+    @staticmethod
+    def empty(rows, cols, scale_layout=SCALE_MMA, device="cuda"):
+        lib = _lib.load()
+        nsc = lib.nvfp4_scales_bytes(rows, cols, scale_layout)
+        return QTensor(torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
+                       torch.zeros(max(nsc, 1), dtype=torch.uint8, device=device),
+                       torch.empty(1, dtype=torch.float32, device=device), rows, cols, scale_layout)
+
+
+def quantize(x: torch.Tensor, *, emit_row=True, emit_col=False, stochastic=False, rht_row=False, rht_col=False,
+             block_2d=False, seed=0, offset=0, rht_signs=0, scale_layout=SCALE_MMA, amax_in=None, amax_out=None,
+             out_row: Optional[QTensor] = None, out_col: Optional[QTensor] = None, stream=None):
+    """nvfp4_quantize on a BF16 CUDA tensor [rows, cols] (last dim contiguous)."""
+    lib = _lib.load()
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D BF16 CUDA tensor with a contiguous last dimension")
+    rows, cols = x.shape
+    if emit_row and out_row is None:
+        out_row = QTensor.empty(rows, cols, scale_layout, x.device)
+    if emit_col and out_col is None:
+        out_col = QTensor.empty(cols, rows, scale_layout, x.device)
+    opts = _lib.QuantOpts(int(stochastic), int(rht_row), int(rht_col), int(block_2d), seed, offset, rht_signs, 0,
+                          _ptr(amax_in), _ptr(amax_out))
+    ws = workspace(x.device, stream)
+    rs = out_row.struct() if emit_row else None
+    cs = out_col.struct() if emit_col else None
+    _lib.check(lib.nvfp4_quantize(x.data_ptr(), rows, cols, x.stride(0), opts, rs, cs, ws.data_ptr(), ws.numel(),
+                                  _stream_ptr(stream)))
+    return (out_row if emit_row else None), (out_col if emit_col else None)
+
+
+def dequantize(q: QTensor, out_dtype=torch.float32, out: Optional[torch.Tensor] = None, stream=None):
+    lib = _lib.load()
+    if out is None:
+        out = torch.empty((q.rows, q.cols), dtype=out_dtype, device=q.codes.device)
+    code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    _lib.check(lib.nvfp4_dequantize(q.struct(), out.data_ptr(), out.stride(0), code, _stream_ptr(stream)))
+    return out
+
+
+def gemm(A: QTensor, B: QTensor, out_dtype=torch.bfloat16, alpha=1.0, accumulate=False,
+         out: Optional[torch.Tensor] = None, stream=None):
+    """nvfp4_gemm: C[M, N] = alpha * S_A * S_B * A . B^T (+ C)."""
+    lib = _lib.load()
+    if out is None:
+        out = (torch.zeros if accumulate else torch.empty)((A.rows, B.rows), dtype=out_dtype, device=A.codes.device)
+    code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    _lib.check(lib.nvfp4_gemm(A.struct(), B.struct(), out.data_ptr(), out.stride(0), code, alpha, int(accumulate),
+                              _stream_ptr(stream)))
+    return out
+
+
+def quantize_weight(w: torch.Tensor, stream=None):
+    """2D 16x16-block quantisation of a weight [N, K]: (row layout [N x K], col layout [K x N])."""
+    return quantize(w, emit_row=True, emit_col=True, block_2d=True, stream=stream)
+
+
+def linear_fwd(x: torch.Tensor, wq_row: QTensor, *, save_col=True, rht_signs=0, out_dtype=torch.bfloat16,
+               out=None, xq_row=None, xq_col=None, stream=None):
+    """nvfp4_linear_fwd: returns (Y, Xq_row, Xq_col or None)."""
+    lib = _lib.load()
+    M, K = x.shape
+    N = wq_row.rows
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    if xq_row is None:
+        xq_row = QTensor.empty(M, K, SCALE_MMA, x.device)
+    if save_col and xq_col is None:
+        xq_col = QTensor.empty(K, M, SCALE_MMA, x.device)
+    ws = workspace(x.device, stream)
+    code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    xr = xq_row.struct()
+    xc = xq_col.struct() if save_col else None
+    _lib.check(lib.nvfp4_linear_fwd(x.data_ptr(), M, K, x.stride(0), wq_row.struct(), out.data_ptr(), out.stride(0),
+                                    code, xr, xc, rht_signs, ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
+    return out, xq_row, (xq_col if save_col else None)
+
+
+def linear_dgrad(dy: torch.Tensor, wq_col: QTensor, *, seed, offset=0, save_col=True, rht_signs=0,
+                 out_dtype=torch.bfloat16, out=None, dyq_row=None, dyq_col=None, stream=None):
+    """nvfp4_linear_dgrad: returns (dX, dYq_row, dYq_col or None)."""
+    lib = _lib.load()
+    M, N = dy.shape
+    K = wq_col.rows
+    if out is None:
+        out = torch.empty((M, K), dtype=out_dtype, device=dy.device)
+    if dyq_row is None:
+        dyq_row = QTensor.empty(M, N, SCALE_MMA, dy.device)
+    if save_col and dyq_col is None:
+        dyq_col = QTensor.empty(N, M, SCALE_MMA, dy.device)
+    ws = workspace(dy.device, stream)
+    code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    dr = dyq_row.struct()
+    dc = dyq_col.struct() if save_col else None
+    _lib.check(lib.nvfp4_linear_dgrad(dy.data_ptr(), M, N, dy.stride(0), wq_col.struct(), out.data_ptr(),
+                                      out.stride(0), code, dr, dc, seed, offset, rht_signs, ws.data_ptr(), ws.numel(),
+                                      _stream_ptr(stream)))
+    return out, dyq_row, (dyq_col if save_col else None)
+
+
+def linear_wgrad(dyq_col: QTensor, xq_col: QTensor, *, out_dtype=torch.bfloat16, accumulate=False, out=None,
+                 stream=None):
+    """nvfp4_linear_wgrad: dW [N, K] = Q(H dY)^T Q(H X)."""
+    lib = _lib.load()
+    if out is None:
+        out = (torch.zeros if accumulate else torch.empty)((dyq_col.rows, xq_col.rows), dtype=out_dtype,
+                                                           device=dyq_col.codes.device)
+    code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    _lib.check(lib.nvfp4_linear_wgrad(dyq_col.struct(), xq_col.struct(), out.data_ptr(), out.stride(0), code,
+                                      int(accumulate), _stream_ptr(stream)))
+    return out
+
+
+def get_status(stream=None):
+    """nvfp4_get_status: synchronise the stream and raise on a recorded device-side error."""
+    lib = _lib.load()
+    _lib.check(lib.nvfp4_get_status(_stream_ptr(stream)))

@@ -1,0 +1,230 @@
+// Device helpers shared by the NVFP4 kernels: format conversions written from
+// the E2M1 / E4M3 definitions, the Philox4x32-10 generator (Salmon et al.,
+// "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11), the 16-point
+// Hadamard butterfly, the tensor-core scale-tile addressing, and bounded
+// mbarrier waits.
+//
+// Every floating-point step of the quantiser is one IEEE round-to-nearest
+// operation (__fdiv_rn / __fmul_rn / __fadd_rn): no contraction into FMA, no
+// flush-to-zero, so the encoded bytes do not depend on compiler choices.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nvfp4 {
+
+// ----------------------------------------------------------------- errors
+
+// Bits of the device error word (one per device, module scope).
+constexpr unsigned kErrTimeout = 1u;
+__device__ unsigned int g_error_word;
+
+// A bounded wait gives up after this long (ns of %globaltimer) and reports
+// kErrTimeout instead of hanging the GPU.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ----------------------------------------------------------------- BF16
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// float -> BF16 bits, round to nearest even (finite inputs).
+__device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
+  uint32_t b = __float_as_uint(f);
+  return (b + 0x7FFFu + ((b >> 16) & 1u)) >> 16;
+}
+
+// ----------------------------------------------------------------- E4M3 scales
+
+// Non-negative float -> E4M3 byte, round to nearest even, saturating at 448.
+// E4M3: bias 7, 3 mantissa bits; normals (1 + m/8) * 2^(e-7), subnormals m * 2^-9.
+__device__ __forceinline__ uint32_t e4m3_encode(float v) {
+  if (!(v < 448.0f)) return 0x7Eu;                 // saturate (also +inf)
+  if (v < 0.015625f) {                             // below 2^-6: subnormal grid 2^-9
+    return (uint32_t)__float2int_rn(__fmul_rn(v, 512.0f));   // 0..8, exact scaling
+  }
+  const uint32_t bits = __float_as_uint(v);
+  const int e = (int)((bits >> 23) & 0xFFu) - 127;  // -6 .. 8
+  const uint32_t mant = bits & 0x7FFFFFu;
+  const uint32_t keep = mant >> 20;                 // top 3 mantissa bits
+  const uint32_t rest = mant & 0xFFFFFu;
+  uint32_t q = 8u + keep;
+  if (rest > 0x80000u || (rest == 0x80000u && (keep & 1u))) q += 1u;   // ties to even
+  return (uint32_t)((e + 6) * 8) + q;              // q == 16 carries into the next binade
+}
+
+__device__ __forceinline__ float e4m3_decode(uint32_t b) {
+  const uint32_t e = b >> 3, m = b & 7u;
+  if (e == 0) return __fmul_rn((float)m, 0.001953125f);        // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));      // (1 + m/8) * 2^(e-7)
+}
+
+// ----------------------------------------------------------------- E2M1 elements
+
+// float -> 4-bit E2M1 code (sign << 3 | index), nearest magnitude of
+// {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to the even index, saturating at 6, sign kept.
+__device__ __forceinline__ uint32_t e2m1_rne(float y) {
+  const float a = fabsf(y);
+  const uint32_t idx = (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
+                       (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) +
+                       (uint32_t)(a > 5.0f);
+  return idx | ((__float_as_uint(y) >> 31) << 3);
+}
+
+// Stochastic rounding between the two neighbouring magnitudes lo <= |y| < hi:
+// up iff (w >> 8) * 2^-24 < (|y| - lo) / (hi - lo); |y| >= 6 gives 6.
+__device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t w) {
+  const float a = fabsf(y);
+  const uint32_t sign = (__float_as_uint(y) >> 31) << 3;
+  if (a >= 6.0f) return 7u | sign;
+  const uint32_t lo = (uint32_t)(a >= 0.5f) + (uint32_t)(a >= 1.0f) + (uint32_t)(a >= 1.5f) +
+                      (uint32_t)(a >= 2.0f) + (uint32_t)(a >= 3.0f) + (uint32_t)(a >= 4.0f);
+  const float lo_v = lo < 4u ? __fmul_rn((float)lo, 0.5f) : (float)lo - 2.0f;   // 0,.5,1,1.5 | 2,3,4
+  const float inv_step = lo < 4u ? 2.0f : (lo < 6u ? 1.0f : 0.5f);
+  const float frac = __fmul_rn(__fsub_rn(a, lo_v), inv_step);                  // exact
+  const float u = __fmul_rn((float)(w >> 8), 5.9604644775390625e-08f);         // * 2^-24, exact
+  return (lo + (u < frac ? 1u : 0u)) | sign;
+}
+
+// ----------------------------------------------------------------- Philox4x32-10
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// The four random words of elements 4*ctr .. 4*ctr+3 of a layout.
+__device__ __forceinline__ uint4 philox_block(uint64_t ctr, uint32_t tag, uint32_t offset,
+                                              uint32_t k0, uint32_t k1) {
+  return philox4x32_10(make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), tag, offset), k0, k1);
+}
+
+// ----------------------------------------------------------------- Hadamard
+
+__device__ __forceinline__ float flip_sign(float v, uint32_t bit) {
+  return __uint_as_float(__float_as_uint(v) ^ (bit << 31));
+}
+
+// Butterfly stage h over N values held in registers: (v[i], v[i+h]) <- (v[i]+v[i+h], v[i]-v[i+h]).
+template <int N>
+__device__ __forceinline__ void wht_stage(float* v, int h) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    if (!(i & h)) {
+      const float a = v[i], b = v[i + h];
+      v[i] = __fadd_rn(a, b);
+      v[i + h] = __fsub_rn(a, b);
+    }
+  }
+}
+
+// Signed, normalised 16-point Walsh-Hadamard transform of v[0..15] (natural order).
+__device__ __forceinline__ void rht16(float* v, uint32_t signs) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = flip_sign(v[j], (signs >> j) & 1u);
+  wht_stage<16>(v, 1);
+  wht_stage<16>(v, 2);
+  wht_stage<16>(v, 4);
+  wht_stage<16>(v, 8);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], 0.25f);
+}
+
+// ----------------------------------------------------------------- scales
+
+// Per-tensor decode scale S = amax / (6 * 448); 1 for an all-zero tensor.
+__device__ __forceinline__ float tensor_scale_from_amax(float amax) {
+  return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
+}
+
+struct BlockScale {
+  float r;        // encode multiplier 1 / (s * S), 0 for a dead block
+  uint32_t sbyte; // E4M3 block scale
+};
+
+// Block scale s = E4M3((b / 6) / S), d = s * S, r = 1 / d.  A block whose scale
+// or decode factor is zero, or whose multiplier overflows, encodes all-zero codes.
+__device__ __forceinline__ BlockScale block_scale(float bmax, float S) {
+  BlockScale out;
+  const float s_f = __fdiv_rn(__fdiv_rn(bmax, 6.0f), S);
+  out.sbyte = e4m3_encode(s_f);
+  const float d = __fmul_rn(e4m3_decode(out.sbyte), S);
+  const float r = __fdiv_rn(1.0f, d);
+  const bool dead = (out.sbyte == 0u) || (d == 0.0f) || !isfinite(r);
+  out.r = dead ? 0.0f : r;
+  return out;
+}
+
+// Byte offset of block scale (row r, block j) in the tensor-core scale layout:
+// tiles of 128 rows x 4 blocks, tile-major along the blocks.
+__device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t j, int64_t kgroups) {
+  return (((r >> 7) * kgroups + (j >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (j & 3);
+}
+
+// ----------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait until the phase with the given parity of mbarrier `bar` has completed.
+// Gives up after kWaitLimitNs, or as soon as *abort is set by another role of
+// the CTA: records kErrTimeout, raises *abort and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&g_error_word, kErrTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,378 @@
+// Block-scaled NVFP4 GEMM for sm_100a: C = alpha * S_A * S_B * A . B^T.
+//
+// The performance passage of "Preentrenamiento de 4 bits con NVFP4 en un hibrido
+// Mamba-Transformer de 12B" rests on the FP4 tensor-core GEMM; "Full-Stack FP4"
+// notes how fast error accumulates in low-precision products, so the
+// accumulator is FP32 in tensor memory and the global scales are applied once,
+// in the epilogue.
+//
+// Structure (one CTA per SM, persistent over output tiles of 128 x 256):
+//   warp 0      TMA producer: per K-stage of 256 elements, one tiled TMA load of
+//               A (128 rows x 128 bytes) and of B (256 x 128 bytes), 128-byte
+//               swizzled, plus bulk copies of the matching block-scale tiles
+//               (already in the tensor-core order, 512 bytes per 128 rows x 64 K).
+//   warp 1      MMA issuer (one thread): copies each stage's scales into tensor
+//               memory (tcgen05.cp) and issues four tcgen05.mma kind::mxf4nvf4
+//               block16 (M=128, N=256, K=64) into an FP32 accumulator in tensor
+//               memory; tcgen05.commit frees the stage and, after the last one,
+//               hands the accumulator to the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter of the
+//               accumulator, scale by alpha*S_A*S_B, round to BF16 (or keep FP32),
+//               store; then release the accumulator.
+// All waits are bounded (see mbar_wait): a stuck pipeline records an error
+// and the CTA winds down instead of hanging.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace gemm {
+
+constexpr int BM = 128;                 // rows of A per tile (MMA M)
+constexpr int BN = 256;                 // rows of B per tile (MMA N)
+constexpr int BK = 256;                 // K elements per pipeline stage
+constexpr int BK_BYTES = BK / 2;        // 128: one 128-byte swizzle row
+constexpr int MMA_K = 64;               // K per tcgen05.mma (kind::mxf4nvf4)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK_BYTES;                        // 16 KiB
+constexpr int B_BYTES = BN * BK_BYTES;                        // 32 KiB
+constexpr int SF_ATOM = 512;                                  // 128 rows x 4 scales
+constexpr int SFA_BYTES = (BM / 128) * (BK / MMA_K) * SF_ATOM;  // 2 KiB
+constexpr int SFB_BYTES = (BN / 128) * (BK / MMA_K) * SF_ATOM;  // 4 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_COL = 0;              // 256 FP32 columns
+constexpr int SFA_COL = 256;            // 4 columns per MMA k-step -> 16
+constexpr int SFB_COL = 256 + 16;       // 8 columns per MMA k-step -> 32
+constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARP0 = 2;
+constexpr int NUM_EPI_WARPS = 4;
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+
+struct Params {
+  int32_t M, N, K;
+  int32_t num_m, num_n, num_k_stages, tail_atoms;   // tail_atoms: MMA k-steps in the last stage
+  int32_t group_m;
+  const uint8_t* sfa;       // tensor-core scale layout of A
+  const uint8_t* sfb;
+  int64_t sf_kgroups;       // 64-element K groups per 128-row scale block (= K / 64)
+  const float* scale_a;
+  const float* scale_b;
+  float alpha;
+  void* C;
+  int64_t ldc;
+  int32_t out_f32;
+  int32_t accumulate;
+};
+
+// Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), UE4M3
+// scales, K-major operands, M = 128, N = n, dense K = 64.
+__host__ __device__ constexpr uint32_t make_idesc(int n) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (uint32_t)(BM >> 4) << 24;
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), sm_100 descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Descriptor of one 512-byte scale tile as tcgen05.cp 32x128b source: 32 rows
+// of 16 bytes, no swizzle, 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_copy_scales(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// 32 lanes x 32 columns of 32-bit accumulator: lane i of the warp gets row i.
+__device__ __forceinline__ void tc_load_32cols(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Wait with a time limit only (teardown after an abort).
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_error_word, kErrTimeout);
+      return;
+    }
+  }
+}
+
+struct TileCoord {
+  int32_t m_blk, n_blk;
+};
+
+// Grouped rasterisation: runs of group_m row-blocks sweep all column blocks, so
+// the CTAs in flight share their A and B tiles through L2.
+__device__ __forceinline__ TileCoord tile_coord(const Params& p, int32_t t) {
+  const int32_t per_group = p.group_m * p.num_n;
+  const int32_t g = t / per_group, w = t - g * per_group;
+  const int32_t m_first = g * p.group_m;
+  const int32_t gm = min(p.group_m, p.num_m - m_first);
+  TileCoord c;
+  c.m_blk = m_first + w % gm;
+  c.n_blk = w / gm;
+  return c;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  uint8_t* bar_area = smem + STAGES * STAGE_BYTES;
+  const uint32_t bar_base = smem_u32(bar_area);
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  const uint32_t acc_full = bar_base + 8u * (2 * STAGES);
+  const uint32_t acc_empty = bar_base + 8u * (2 * STAGES + 1);
+  const uint32_t mma_done = bar_base + 8u * (2 * STAGES + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (2 * STAGES + 3));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * STAGES + 3) + 4);
+
+  auto a_smem = [&](int s) { return smem_base + (uint32_t)(s * STAGE_BYTES); };
+  auto b_smem = [&](int s) { return smem_base + (uint32_t)(s * STAGE_BYTES + A_BYTES); };
+  auto sfa_smem = [&](int s) { return smem_base + (uint32_t)(s * STAGE_BYTES + A_BYTES + B_BYTES); };
+  auto sfb_smem = [&](int s) { return smem_base + (uint32_t)(s * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, NUM_EPI_WARPS);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int32_t num_tiles = p.num_m * p.num_n;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_phase[STAGES];
+      bool issued[STAGES];
+      for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_phase[s] = 0;
+      bool ok = true;
+      for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = tile_coord(p, t);
+        const int nb_valid = min(2, (p.N - tc.n_blk * BN) / 128);
+        for (int ks = 0; ks < p.num_k_stages; ++ks) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
+          const uint32_t sf_bytes = (uint32_t)atoms * SF_ATOM;
+          mbar_arrive_expect_tx(full_bar(stage), (uint32_t)(A_BYTES + B_BYTES) + sf_bytes * (1u + nb_valid));
+          tma_load_2d(a_smem(stage), &tma_a, ks * BK_BYTES, tc.m_blk * BM, full_bar(stage));
+          tma_load_2d(b_smem(stage), &tma_b, ks * BK_BYTES, tc.n_blk * BN, full_bar(stage));
+          const int64_t kg = (int64_t)ks * (BK / MMA_K);
+          bulk_load(sfa_smem(stage), p.sfa + ((int64_t)tc.m_blk * p.sf_kgroups + kg) * SF_ATOM, sf_bytes,
+                    full_bar(stage));
+          for (int nb = 0; nb < nb_valid; ++nb)
+            bulk_load(sfb_smem(stage) + nb * (BK / MMA_K) * SF_ATOM,
+                      p.sfb + ((int64_t)(tc.n_blk * 2 + nb) * p.sf_kgroups + kg) * SF_ATOM, sf_bytes,
+                      full_bar(stage));
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // wind down: let every load already issued land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued[s]) mbar_wait_drain(full_bar(s), issued_phase[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int32_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = tile_coord(p, t);
+        const int nb_valid = min(2, (p.N - tc.n_blk * BN) / 128);
+        const uint32_t idesc = make_idesc(nb_valid * 128);
+        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int ks = 0; ks < p.num_k_stages; ++ks) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
+          for (int kk = 0; kk < atoms; ++kk) {
+            tc_copy_scales(tmem + SFA_COL + 4 * kk, sf_desc(sfa_smem(stage) + kk * SF_ATOM));
+            for (int nb = 0; nb < nb_valid; ++nb)
+              tc_copy_scales(tmem + SFB_COL + 8 * kk + 4 * nb,
+                             sf_desc(sfb_smem(stage) + (nb * (BK / MMA_K) + kk) * SF_ATOM));
+            tc_mma(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * (MMA_K / 2)),
+                   sw128_desc(b_smem(stage) + kk * (MMA_K / 2)), idesc, (ks | kk) != 0 ? 1u : 0u,
+                   tmem + SFA_COL + 4 * kk, tmem + SFB_COL + 8 * kk);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        acc_phase ^= 1u;
+      }
+      // every MMA issued by this thread has finished once mma_done flips
+      tc_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;                  // tensor-memory lanes 32*quarter ..
+    const int row_in_tile = quarter * 32 + lane;
+    const float g = __fmul_rn(__fmul_rn(*p.scale_a, *p.scale_b), p.alpha);
+    uint32_t acc_phase = 0;
+    for (int32_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const TileCoord tc = tile_coord(p, t);
+      const int n_cols = min(BN, p.N - tc.n_blk * BN);
+      // every lane polls; the warp proceeds (converged) only if all saw the phase complete
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, acc_phase, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t m = (int64_t)tc.m_blk * BM + row_in_tile;
+      for (int chunk = 0; chunk < n_cols / 32; ++chunk) {
+        uint32_t r[32];
+        tc_load_32cols(tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + chunk * 32, r);
+        const int64_t n0 = (int64_t)tc.n_blk * BN + chunk * 32;
+        if (p.out_f32) {
+          float* crow = static_cast<float*>(p.C) + m * p.ldc + n0;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 v = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), g), __fmul_rn(__uint_as_float(r[4 * q + 1]), g),
+                                   __fmul_rn(__uint_as_float(r[4 * q + 2]), g),
+                                   __fmul_rn(__uint_as_float(r[4 * q + 3]), g));
+            if (p.accumulate) {
+              const float4 o = reinterpret_cast<const float4*>(crow)[q];
+              v.x = __fadd_rn(v.x, o.x);
+              v.y = __fadd_rn(v.y, o.y);
+              v.z = __fadd_rn(v.z, o.z);
+              v.w = __fadd_rn(v.w, o.w);
+            }
+            reinterpret_cast<float4*>(crow)[q] = v;
+          }
+        } else {
+          uint16_t* crow = static_cast<uint16_t*>(p.C) + m * p.ldc + n0;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[4];
+            uint4 old = make_uint4(0u, 0u, 0u, 0u);
+            if (p.accumulate) old = reinterpret_cast<const uint4*>(crow)[q];
+            const uint32_t oldw[4] = {old.x, old.y, old.z, old.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float v0 = __fmul_rn(__uint_as_float(r[8 * q + 2 * e]), g);
+              float v1 = __fmul_rn(__uint_as_float(r[8 * q + 2 * e + 1]), g);
+              if (p.accumulate) {
+                v0 = __fadd_rn(v0, bf16_lo(oldw[e]));
+                v1 = __fadd_rn(v1, bf16_hi(oldw[e]));
+              }
+              w[e] = f32_to_bf16_bits(v0) | (f32_to_bf16_bits(v1) << 16);
+            }
+            reinterpret_cast<uint4*>(crow)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+}  // namespace gemm
+}  // namespace nvfp4

@@ -1,0 +1,410 @@
+// C ABI of the NVFP4 linear-layer library (declared in include/nvfp4.h).
+//
+// Host side only: argument validation, tensor-map construction for the GEMM's
+// TMA loads, and kernel launches on the caller's stream.  One translation unit
+// holds every kernel (quantize.cuh, gemm.cuh) so that the module-scope device
+// error word is shared by all of them.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "nvfp4.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "quantize.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kWorkspaceBytes = 256;
+
+thread_local char g_last_error[512] = "";
+
+nvfp4_status fail(nvfp4_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+nvfp4_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(NVFP4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+struct DeviceInfo {
+  int sm_count = 0;
+  bool gemm_attr = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+nvfp4_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(NVFP4_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (d.sm_count == 0) {
+    e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  }
+  if (!d.gemm_attr) {
+    e = cudaFuncSetAttribute(nvfp4::gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             nvfp4::gemm::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
+    d.gemm_attr = true;
+  }
+  *out = &d;
+  return NVFP4_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+nvfp4_status get_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::call_once(g_encode_once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  if (!g_encode) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  *fn = g_encode;
+  return NVFP4_OK;
+}
+
+// Tensor map of packed E2M1 codes [rows][cols/2 bytes]: box of box_rows x 128
+// bytes, 128-byte swizzle (the tensor cores' K-major operand layout).
+nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  nvfp4_status st = get_encoder(&encode);
+  if (st != NVFP4_OK) return st;
+  const cuuint64_t dims[2] = {(cuuint64_t)(t->cols / 2), (cuuint64_t)t->rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(t->cols / 2)};
+  const cuuint32_t box[2] = {128u, box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, t->codes, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return NVFP4_OK;
+}
+
+nvfp4_status check_tensor(const nvfp4_tensor* t, const char* name) {
+  if (!t) return fail(NVFP4_ERR_INVALID_ARG, "%s is NULL", name);
+  if (t->rows < 0 || t->cols < 0) return fail(NVFP4_ERR_INVALID_ARG, "%s has a negative extent", name);
+  const bool empty = t->rows == 0 || t->cols == 0;   // an empty tensor needs only its tensor scale
+  if (!t->tensor_scale || (!empty && (!t->codes || !t->scales)))
+    return fail(NVFP4_ERR_INVALID_ARG, "%s has a NULL buffer", name);
+  if (t->scale_layout != NVFP4_SCALE_ROWMAJOR && t->scale_layout != NVFP4_SCALE_MMA)
+    return fail(NVFP4_ERR_INVALID_ARG, "%s.scale_layout is %d", name, t->scale_layout);
+  if (t->reserved != 0) return fail(NVFP4_ERR_INVALID_ARG, "%s.reserved must be 0", name);
+  if (t->cols % 16) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s.cols %lld is not a multiple of 16", name, (long long)t->cols);
+  if (!aligned16(t->codes)) return fail(NVFP4_ERR_MISALIGNED, "%s.codes is not 16-byte aligned", name);
+  return NVFP4_OK;
+}
+
+nvfp4::QuantLayout layout_of(const nvfp4_tensor* t) {
+  nvfp4::QuantLayout L{};
+  if (!t) return L;
+  L.codes = t->codes;
+  L.scales = t->scales;
+  L.tensor_scale = t->tensor_scale;
+  L.kgroups = ceil_div(t->cols / 16, 4);
+  L.mma_layout = t->scale_layout == NVFP4_SCALE_MMA;
+  return L;
+}
+
+template <bool ER, bool EC, bool SR, bool RR, bool RC, bool TD>
+void launch_quant(const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
+  nvfp4::quantize_kernel<ER, EC, SR, RR, RC, TD><<<grid, nvfp4::kQuantThreads, 0, s>>>(p);
+}
+
+template <bool ER, bool EC, bool SR, bool RR, bool RC>
+void dispatch_td(bool td, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
+  if constexpr (!SR && !RR && !RC) {
+    if (td) return launch_quant<ER, EC, false, false, false, true>(p, grid, s);
+  }
+  launch_quant<ER, EC, SR, RR, RC, false>(p, grid, s);
+}
+
+template <bool ER, bool EC, bool SR, bool RR>
+void dispatch_rc(bool rc, bool td, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
+  if (rc) return dispatch_td<ER, EC, SR, RR, true>(td, p, grid, s);
+  dispatch_td<ER, EC, SR, RR, false>(td, p, grid, s);
+}
+
+template <bool ER, bool EC, bool SR>
+void dispatch_rr(bool rr, bool rc, bool td, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
+  if (rr) return dispatch_rc<ER, EC, SR, true>(rc, td, p, grid, s);
+  dispatch_rc<ER, EC, SR, false>(rc, td, p, grid, s);
+}
+
+template <bool ER, bool EC>
+void dispatch_sr(bool sr, bool rr, bool rc, bool td, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
+  if (sr) return dispatch_rr<ER, EC, true>(rr, rc, td, p, grid, s);
+  dispatch_rr<ER, EC, false>(rr, rc, td, p, grid, s);
+}
+
+void dispatch_quant(bool er, bool ec, bool sr, bool rr, bool rc, bool td, const nvfp4::QuantParams& p, int grid,
+                    cudaStream_t s) {
+  if (er && ec) return dispatch_sr<true, true>(sr, rr, rc, td, p, grid, s);
+  if (er) return dispatch_sr<true, false>(sr, rr, rc, td, p, grid, s);
+  dispatch_sr<false, true>(sr, rr, rc, td, p, grid, s);
+}
+
+void launch_amax(bool rc, bool rr, const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t signs,
+                 unsigned* out, int grid, cudaStream_t s) {
+  if (rc && rr) nvfp4::amax_kernel<true, true><<<grid, nvfp4::kQuantThreads, 0, s>>>(x, rows, cols, ld, signs, out);
+  else if (rc) nvfp4::amax_kernel<true, false><<<grid, nvfp4::kQuantThreads, 0, s>>>(x, rows, cols, ld, signs, out);
+  else if (rr) nvfp4::amax_kernel<false, true><<<grid, nvfp4::kQuantThreads, 0, s>>>(x, rows, cols, ld, signs, out);
+  else nvfp4::amax_kernel<false, false><<<grid, nvfp4::kQuantThreads, 0, s>>>(x, rows, cols, ld, signs, out);
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvfp4_version(void) { return 100; }
+
+size_t nvfp4_workspace_size(void) { return kWorkspaceBytes; }
+
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t scale_layout) {
+  if (rows < 0 || cols < 0) return 0;
+  if (scale_layout == NVFP4_SCALE_MMA) return (size_t)(ceil_div(rows, 128) * 128) * (size_t)(ceil_div(cols / 16, 4) * 4);
+  return (size_t)rows * (size_t)(cols / 16);
+}
+
+const char* nvfp4_last_error_string(void) { return g_last_error; }
+
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, const nvfp4_quant_opts* opts,
+                            nvfp4_tensor* out_row, nvfp4_tensor* out_col, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (!opts) return fail(NVFP4_ERR_INVALID_ARG, "opts is NULL");
+  if (!out_row && !out_col) return fail(NVFP4_ERR_INVALID_ARG, "no output layout requested");
+  if (rows < 0 || cols < 0) return fail(NVFP4_ERR_INVALID_ARG, "negative extent");
+  if (cols % 16) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "cols %lld is not a multiple of 16", (long long)cols);
+  if ((out_col || opts->block_2d) && rows % 16)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rows %lld is not a multiple of 16 (col layout / 2D blocks)", (long long)rows);
+  if (rows > 0 && cols > 0) {
+    if (!x) return fail(NVFP4_ERR_INVALID_ARG, "x is NULL");
+    if (ld < cols) return fail(NVFP4_ERR_INVALID_ARG, "ld %lld < cols %lld", (long long)ld, (long long)cols);
+    if (!aligned16(x) || ld % 8) return fail(NVFP4_ERR_MISALIGNED, "x rows are not 16-byte aligned");
+  }
+  if (opts->reserved) return fail(NVFP4_ERR_INVALID_ARG, "opts.reserved must be 0");
+  if (opts->block_2d && (opts->stochastic || opts->rht_row || opts->rht_col))
+    return fail(NVFP4_ERR_INVALID_ARG, "2D weight blocks exclude stochastic rounding and the RHT");
+  if (opts->offset >> 32) return fail(NVFP4_ERR_INVALID_ARG, "opts.offset must be < 2^32");
+  if (opts->rht_signs >> 16) return fail(NVFP4_ERR_INVALID_ARG, "opts.rht_signs has bits above 15");
+  if (opts->rht_row && !out_row) return fail(NVFP4_ERR_INVALID_ARG, "rht_row without a row layout");
+  if (opts->rht_col && !out_col) return fail(NVFP4_ERR_INVALID_ARG, "rht_col without a col layout");
+  nvfp4_status st;
+  if (out_row) {
+    if ((st = check_tensor(out_row, "out_row")) != NVFP4_OK) return st;
+    if (out_row->rows != rows || out_row->cols != cols)
+      return fail(NVFP4_ERR_INVALID_ARG, "out_row is %lldx%lld, x is %lldx%lld", (long long)out_row->rows,
+                  (long long)out_row->cols, (long long)rows, (long long)cols);
+  }
+  if (out_col) {
+    if ((st = check_tensor(out_col, "out_col")) != NVFP4_OK) return st;
+    if (out_col->rows != cols || out_col->cols != rows)
+      return fail(NVFP4_ERR_INVALID_ARG, "out_col is %lldx%lld, expected %lldx%lld", (long long)out_col->rows,
+                  (long long)out_col->cols, (long long)cols, (long long)rows);
+  }
+  const float* amax = opts->amax_in;
+  if (!amax) {
+    if (!workspace || workspace_bytes < kWorkspaceBytes)
+      return fail(NVFP4_ERR_WORKSPACE, "workspace of %zu bytes needed", kWorkspaceBytes);
+    if (!aligned16(workspace)) return fail(NVFP4_ERR_MISALIGNED, "workspace is not 16-byte aligned");
+  }
+  DeviceInfo* dev;
+  if ((st = device_info(&dev)) != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  const int64_t items = ceil_div(rows, nvfp4::kSlabRows) * ceil_div(cols, nvfp4::kSlabCols);
+  if (!amax) {
+    unsigned* ws = static_cast<unsigned*>(workspace);
+    cudaError_t e = cudaMemsetAsync(ws, 0, 3 * sizeof(unsigned), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+    if (items > 0) {
+      const int64_t want = ceil_div(items, nvfp4::kQuantWarps);
+      const int grid = (int)std::min<int64_t>(want, (int64_t)dev->sm_count * 8);
+      launch_amax(opts->rht_col != 0, opts->rht_row != 0, static_cast<const uint16_t*>(x), rows, cols, ld,
+                  opts->rht_signs, ws, grid, s);
+    }
+    amax = reinterpret_cast<const float*>(ws);
+  }
+  nvfp4::QuantParams p{};
+  p.x = static_cast<const uint16_t*>(x);
+  p.rows = rows;
+  p.cols = cols;
+  p.ld = ld;
+  p.row = layout_of(out_row);
+  p.col = layout_of(out_col);
+  p.amax = amax;
+  p.amax_out = opts->amax_out;
+  p.key0 = (uint32_t)opts->seed;
+  p.key1 = (uint32_t)(opts->seed >> 32);
+  p.offset = (uint32_t)opts->offset;
+  p.signs = opts->rht_signs;
+  const int64_t tiles = ceil_div(ceil_div(rows, nvfp4::kSlabRows), nvfp4::kQuantWarps) * ceil_div(cols, nvfp4::kSlabCols);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)1 << 30));
+  dispatch_quant(out_row != nullptr, out_col != nullptr, opts->stochastic != 0, opts->rht_row != 0,
+                 opts->rht_col != 0, opts->block_2d != 0, p, grid, s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_dequantize(const nvfp4_tensor* q, void* out, int64_t ldo, int32_t out_dtype, void* stream) {
+  nvfp4_status st = check_tensor(q, "q");
+  if (st != NVFP4_OK) return st;
+  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return fail(NVFP4_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
+  const int64_t total = q->rows * (q->cols / 16);
+  if (total == 0) return NVFP4_OK;
+  if (!out) return fail(NVFP4_ERR_INVALID_ARG, "out is NULL");
+  if (ldo < q->cols) return fail(NVFP4_ERR_INVALID_ARG, "ldo < cols");
+  if (!aligned16(out) || (ldo * (out_dtype == NVFP4_OUT_F32 ? 4 : 2)) % 16)
+    return fail(NVFP4_ERR_MISALIGNED, "out rows are not 16-byte aligned");
+  DeviceInfo* dev;
+  if ((st = device_info(&dev)) != NVFP4_OK) return st;
+  const int grid = (int)std::min<int64_t>(ceil_div(total, 256), (int64_t)dev->sm_count * 16);
+  nvfp4::dequantize_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      q->codes, q->scales, q->tensor_scale, q->rows, q->cols, q->scale_layout == NVFP4_SCALE_MMA,
+      ceil_div(q->cols / 16, 4), out, ldo, out_dtype == NVFP4_OUT_F32);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc, int32_t out_dtype,
+                        float alpha, int32_t accumulate, void* stream) {
+  nvfp4_status st;
+  if ((st = check_tensor(A, "A")) != NVFP4_OK) return st;
+  if ((st = check_tensor(B, "B")) != NVFP4_OK) return st;
+  if (A->cols != B->cols) return fail(NVFP4_ERR_INVALID_ARG, "A.cols %lld != B.cols %lld", (long long)A->cols, (long long)B->cols);
+  if (A->scale_layout != NVFP4_SCALE_MMA || B->scale_layout != NVFP4_SCALE_MMA)
+    return fail(NVFP4_ERR_INVALID_ARG, "GEMM operands need the tensor-core scale layout");
+  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return fail(NVFP4_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
+  const int64_t M = A->rows, N = B->rows, K = A->cols;
+  if (M % 128 || N % 128 || K % 64)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "GEMM needs M %% 128, N %% 128, K %% 64 == 0 (got %lld, %lld, %lld)",
+                (long long)M, (long long)N, (long long)K);
+  if (M > (1ll << 31) - 128 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "GEMM extent above 2^31");
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (!C) return fail(NVFP4_ERR_INVALID_ARG, "C is NULL");
+  if (ldc < N) return fail(NVFP4_ERR_INVALID_ARG, "ldc < N");
+  if (!aligned16(C) || (ldc * (out_dtype == NVFP4_OUT_F32 ? 4 : 2)) % 16)
+    return fail(NVFP4_ERR_MISALIGNED, "C rows are not 16-byte aligned");
+  if (!aligned16(A->scales) || !aligned16(B->scales)) return fail(NVFP4_ERR_MISALIGNED, "scales not 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    // empty contraction: C = 0 (or unchanged when accumulating)
+    if (accumulate) return NVFP4_OK;
+    const size_t esz = out_dtype == NVFP4_OUT_F32 ? 4 : 2;
+    cudaError_t e = cudaMemset2DAsync(C, (size_t)ldc * esz, 0, (size_t)N * esz, (size_t)M, s);
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "cudaMemset2DAsync");
+  }
+  DeviceInfo* dev;
+  if ((st = device_info(&dev)) != NVFP4_OK) return st;
+  CUtensorMap map_a, map_b;
+  if ((st = make_code_map(&map_a, A, nvfp4::gemm::BM)) != NVFP4_OK) return st;
+  if ((st = make_code_map(&map_b, B, nvfp4::gemm::BN)) != NVFP4_OK) return st;
+  nvfp4::gemm::Params p{};
+  p.M = (int32_t)M;
+  p.N = (int32_t)N;
+  p.K = (int32_t)K;
+  p.num_m = (int32_t)(M / nvfp4::gemm::BM);
+  p.num_n = (int32_t)ceil_div(N, nvfp4::gemm::BN);
+  p.num_k_stages = (int32_t)ceil_div(K, nvfp4::gemm::BK);
+  const int64_t tail = K % nvfp4::gemm::BK;
+  p.tail_atoms = tail ? (int32_t)(tail / nvfp4::gemm::MMA_K) : nvfp4::gemm::BK / nvfp4::gemm::MMA_K;
+  p.group_m = 16;
+  p.sfa = A->scales;
+  p.sfb = B->scales;
+  p.sf_kgroups = K / 64;
+  p.scale_a = A->tensor_scale;
+  p.scale_b = B->tensor_scale;
+  p.alpha = alpha;
+  p.C = C;
+  p.ldc = ldc;
+  p.out_f32 = out_dtype == NVFP4_OUT_F32;
+  p.accumulate = accumulate != 0;
+  const int64_t tiles = (int64_t)p.num_m * p.num_n;
+  const int grid = (int)std::min<int64_t>(tiles, dev->sm_count);
+  nvfp4::gemm::gemm_kernel<<<grid, nvfp4::gemm::NUM_THREADS, nvfp4::gemm::SMEM_BYTES, s>>>(map_a, map_b, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_linear_fwd(const void* X, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* Wq_row, void* Y,
+                              int64_t ldy, int32_t out_dtype, nvfp4_tensor* Xq_row, nvfp4_tensor* Xq_col,
+                              uint32_t rht_signs, void* workspace, size_t workspace_bytes, void* stream) {
+  nvfp4_status st = check_tensor(Wq_row, "Wq_row");
+  if (st != NVFP4_OK) return st;
+  if (Wq_row->cols != K) return fail(NVFP4_ERR_INVALID_ARG, "Wq_row.cols %lld != K %lld", (long long)Wq_row->cols, (long long)K);
+  if (!Xq_row) return fail(NVFP4_ERR_INVALID_ARG, "Xq_row is NULL");
+  if (M % 128 || Wq_row->rows % 128 || K % 64) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "linear needs M %% 128, N %% 128, K %% 64 == 0");
+  nvfp4_quant_opts o{};
+  o.rht_col = Xq_col != nullptr;
+  o.rht_signs = rht_signs;
+  if ((st = nvfp4_quantize(X, M, K, ldx, &o, Xq_row, Xq_col, workspace, workspace_bytes, stream)) != NVFP4_OK) return st;
+  return nvfp4_gemm(Xq_row, Wq_row, Y, ldy, out_dtype, 1.0f, 0, stream);
+}
+
+nvfp4_status nvfp4_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ldy, const nvfp4_tensor* Wq_col,
+                                void* dX, int64_t ldx, int32_t out_dtype, nvfp4_tensor* dYq_row, nvfp4_tensor* dYq_col,
+                                uint64_t seed, uint64_t offset, uint32_t rht_signs, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  nvfp4_status st = check_tensor(Wq_col, "Wq_col");
+  if (st != NVFP4_OK) return st;
+  if (Wq_col->cols != N) return fail(NVFP4_ERR_INVALID_ARG, "Wq_col.cols %lld != N %lld", (long long)Wq_col->cols, (long long)N);
+  if (!dYq_row) return fail(NVFP4_ERR_INVALID_ARG, "dYq_row is NULL");
+  if (M % 128 || Wq_col->rows % 128 || N % 64) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "dgrad needs M %% 128, K %% 128, N %% 64 == 0");
+  nvfp4_quant_opts o{};
+  o.stochastic = 1;
+  o.rht_col = dYq_col != nullptr;
+  o.seed = seed;
+  o.offset = offset;
+  o.rht_signs = rht_signs;
+  if ((st = nvfp4_quantize(dY, M, N, ldy, &o, dYq_row, dYq_col, workspace, workspace_bytes, stream)) != NVFP4_OK) return st;
+  return nvfp4_gemm(dYq_row, Wq_col, dX, ldx, out_dtype, 1.0f, 0, stream);
+}
+
+nvfp4_status nvfp4_linear_wgrad(const nvfp4_tensor* dYq_col, const nvfp4_tensor* Xq_col, void* dW, int64_t ldw,
+                                int32_t out_dtype, int32_t accumulate, void* stream) {
+  return nvfp4_gemm(dYq_col, Xq_col, dW, ldw, out_dtype, 1.0f, accumulate, stream);
+}
+
+nvfp4_status nvfp4_get_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned word = 0;
+  e = cudaMemcpyFromSymbol(&word, nvfp4::g_error_word, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (word) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(nvfp4::g_error_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    if (word & nvfp4::kErrTimeout) return fail(NVFP4_ERR_TIMEOUT, "a device-side wait exceeded its time limit");
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pending CUDA error");
+  return NVFP4_OK;
+}
+
+}  // extern "C"

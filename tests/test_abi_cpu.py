@@ -1,0 +1,106 @@
+"""CPU-side checks of the C ABI: the library builds for sm_100a, loads without a
+GPU, exports every function include/nvfp4.h declares, and rejects bad arguments
+before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from nvfp4_pretraining_linear_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _lib.load()
+
+
+def test_library_exports_every_declared_function(lib):
+    declared = header_functions()
+    assert {"nvfp4_quantize", "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_linear_fwd", "nvfp4_linear_dgrad",
+            "nvfp4_linear_wgrad"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared <= set(_lib.SIGNATURES), declared - set(_lib.SIGNATURES)
+
+
+def test_struct_layouts_match_header():
+    # sizes follow from the header's field order (x86-64 / aarch64 ABI)
+    assert ctypes.sizeof(_lib.NVFP4Tensor) == 8 * 3 + 8 * 2 + 4 * 2
+    assert ctypes.sizeof(_lib.QuantOpts) == 4 * 4 + 8 * 2 + 4 * 2 + 8 * 2
+
+
+def test_sizes(lib):
+    assert lib.nvfp4_version() >= 100
+    assert lib.nvfp4_workspace_size() >= 12
+    assert lib.nvfp4_scales_bytes(256, 256, _lib.SCALE_ROWMAJOR) == 256 * 16
+    assert lib.nvfp4_scales_bytes(256, 256, _lib.SCALE_MMA) == 256 * 16
+    assert lib.nvfp4_scales_bytes(200, 80, _lib.SCALE_MMA) == 256 * 8   # rows padded to 128, blocks to 4
+    assert lib.nvfp4_scales_bytes(16, 32, _lib.SCALE_ROWMAJOR) == 32
+
+
+def _tensor(rows, cols, layout=_lib.SCALE_MMA, ptr=0x10000):
+    return _lib.NVFP4Tensor(ptr, ptr + 0x100000, ptr + 0x200000, rows, cols, layout, 0)
+
+
+def test_quantize_argument_errors(lib):
+    opts = _lib.QuantOpts()
+    t = _tensor(32, 48)
+    st = lib.nvfp4_quantize(0x1000, 32, 48, 48, None, ctypes.byref(t), None, 0x2000, 256, None)
+    assert st == 1  # opts NULL
+    st = lib.nvfp4_quantize(0x1000, 32, 40, 40, ctypes.byref(opts), ctypes.byref(_tensor(32, 40)), None, 0x2000, 256, None)
+    assert st == 2  # cols % 16
+    st = lib.nvfp4_quantize(0x1000, 32, 48, 48, ctypes.byref(opts), None, None, 0x2000, 256, None)
+    assert st == 1  # no output
+    st = lib.nvfp4_quantize(0x1008, 32, 48, 48, ctypes.byref(opts), ctypes.byref(t), None, 0x2000, 256, None)
+    assert st == 3  # misaligned x
+    bad = _lib.QuantOpts(1, 0, 0, 1, 0, 0, 0, 0, None, None)
+    st = lib.nvfp4_quantize(0x1000, 32, 48, 48, ctypes.byref(bad), ctypes.byref(t), None, 0x2000, 256, None)
+    assert st == 1  # 2D with SR
+    big = _lib.QuantOpts(1, 0, 0, 0, 0, 1 << 32, 0, 0, None, None)
+    st = lib.nvfp4_quantize(0x1000, 32, 48, 48, ctypes.byref(big), ctypes.byref(t), None, 0x2000, 256, None)
+    assert st == 1  # offset >= 2^32
+    col = _tensor(48, 24)
+    st = lib.nvfp4_quantize(0x1000, 24, 48, 48, ctypes.byref(opts), None, ctypes.byref(col), 0x2000, 256, None)
+    assert st == 2  # col layout needs rows % 16
+    st = lib.nvfp4_quantize(0x1000, 32, 48, 48, ctypes.byref(opts), ctypes.byref(_tensor(32, 64)), None, 0x2000, 256, None)
+    assert st == 1  # shape mismatch
+    st = lib.nvfp4_quantize(0x1000, 32, 48, 48, ctypes.byref(opts), ctypes.byref(t), None, None, 0, None)
+    assert st == 6  # no workspace
+    msg = lib.nvfp4_last_error_string().decode()
+    assert "workspace" in msg
+
+
+def test_gemm_argument_errors(lib):
+    a = _tensor(128, 64)
+    b = _tensor(128, 128)
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), 0x1000, 128, 0, 1.0, 0, None) == 1  # K mismatch
+    a = _tensor(100, 64)
+    b = _tensor(128, 64)
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), 0x1000, 128, 0, 1.0, 0, None) == 2  # M % 128
+    a = _tensor(128, 64, _lib.SCALE_ROWMAJOR)
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), 0x1000, 128, 0, 1.0, 0, None) == 1  # layout
+    a = _tensor(128, 64)
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), 0x1004, 128, 0, 1.0, 0, None) == 3  # misaligned C
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), 0x1000, 128, 7, 1.0, 0, None) == 1  # dtype
+    assert lib.nvfp4_gemm(None, ctypes.byref(b), 0x1000, 128, 0, 1.0, 0, None) == 1
+
+
+def test_dequantize_argument_errors(lib):
+    q = _tensor(32, 48)
+    assert lib.nvfp4_dequantize(ctypes.byref(q), None, 48, 1, None) == 1
+    assert lib.nvfp4_dequantize(ctypes.byref(q), 0x1000, 40, 1, None) == 1
+    assert lib.nvfp4_dequantize(ctypes.byref(q), 0x1008, 48, 1, None) == 3

@@ -1,0 +1,115 @@
+"""GPU parity of the block-scaled NVFP4 GEMM (nvfp4_gemm) against the oracle's
+FP64 product of the dequantised operands.
+
+Bound: |C - C_ref| <= 1e-5 * sum_k |a_k b_k| + 1e-6 for FP32 output; the BF16
+output adds one BF16 half-ulp (2^-8 |C_ref|) for its final rounding."""
+
+import numpy as np
+import pytest
+import torch
+
+from nvfp4_pretraining_linear_b200 import api, synthetic
+from oracle import nvfp4_oracle as O
+from tests.helpers import assert_layout_equal, bf16_to_np, gemm_check
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    (128, 128, 64),       # one tile, one MMA k-step
+    (256, 256, 256),      # tiny config
+    (384, 640, 320),      # N tail of 128 (half tile), K tail of 64
+    (512, 384, 1024),
+    (256, 1280, 768),     # several N tiles, K tail of 0
+    (1152, 512, 2112),    # more tiles than one wave per CTA? K tail 64
+]
+
+
+def operands(M, N, K, seed, kind="outliers"):
+    if kind == "outliers":
+        a = synthetic.normal((M, K), 1.0, seed=seed, device="cuda", outlier_frac=0.01, outlier_mult=50.0)
+        b = synthetic.normal((N, K), 1.0, seed=seed + 1, device="cuda", outlier_frac=0.01, outlier_mult=50.0)
+    else:
+        a = synthetic.student_t((M, K), 3, 0.1, seed=seed, device="cuda")
+        b = synthetic.normal((N, K), 0.02, seed=seed + 1, device="cuda")
+    return a, b
+
+
+def quantised_pair(a, b):
+    qa, _ = api.quantize(a)
+    qb, _ = api.quantize(b)
+    ra = O.quantize(bf16_to_np(a))["row"]
+    rb = O.quantize(bf16_to_np(b))["row"]
+    assert_layout_equal(qa, ra, "A")
+    assert_layout_equal(qb, rb, "B")
+    return qa, qb, O.dequantize(*ra), O.dequantize(*rb)
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_gemm_f32_within_bound(M, N, K):
+    a, b = operands(M, N, K, seed=M + N + K)
+    qa, qb, ah, bh = quantised_pair(a, b)
+    c = api.gemm(qa, qb, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ratio = gemm_check(c.cpu().numpy(), ah, bh)
+    assert ratio <= 1.0, ratio
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES[:4])
+def test_gemm_bf16_within_bound(M, N, K):
+    a, b = operands(M, N, K, seed=7 * M + K, kind="t")
+    qa, qb, ah, bh = quantised_pair(a, b)
+    c = api.gemm(qa, qb, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ratio = gemm_check(c.float().cpu().numpy(), ah, bh, bf16=True)
+    assert ratio <= 1.0, ratio
+
+
+def test_gemm_alpha_and_accumulate():
+    M, N, K = 256, 384, 512
+    a, b = operands(M, N, K, seed=99)
+    qa, qb, ah, bh = quantised_pair(a, b)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    c0 = torch.randn((M, N), generator=g, device="cuda") * 10
+    c = c0.clone()
+    api.gemm(qa, qb, alpha=0.375, accumulate=True, out=c)
+    torch.cuda.synchronize()
+    ratio = gemm_check(c.cpu().numpy(), ah, bh, alpha=0.375, c0=c0.cpu().numpy())
+    assert ratio <= 1.0, ratio
+    cb0 = c0.to(torch.bfloat16)
+    cb = cb0.clone()
+    api.gemm(qa, qb, alpha=-2.0, accumulate=True, out=cb)
+    torch.cuda.synchronize()
+    ratio = gemm_check(cb.float().cpu().numpy(), ah, bh, alpha=-2.0, c0=cb0.float().cpu().numpy(), bf16=True)
+    assert ratio <= 1.0, ratio
+
+
+def test_gemm_strided_output_and_zero_operand():
+    M, N, K = 256, 256, 256
+    a, b = operands(M, N, K, seed=3)
+    qa, qb, ah, bh = quantised_pair(a, b)
+    big = torch.full((M, N + 64), 7.0, device="cuda")
+    out = big[:, :N]
+    api.gemm(qa, qb, out_dtype=torch.float32, out=out)
+    torch.cuda.synchronize()
+    assert gemm_check(out.cpu().numpy(), ah, bh) <= 1.0
+    assert torch.all(big[:, N:] == 7.0)
+    z = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    qz, _ = api.quantize(z)
+    cz = api.gemm(qz, qb, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(cz) == 0
+
+
+def test_gemm_large_k_accumulation():
+    # K = 16384: the FP32 tensor-memory accumulation over 256 MMA k-steps
+    M, N, K = 256, 256, 16384
+    a, b = operands(M, N, K, seed=21)
+    qa, qb, ah, bh = quantised_pair(a, b)
+    c = api.gemm(qa, qb, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ratio = gemm_check(c.cpu().numpy(), ah, bh)
+    assert ratio <= 1.0, ratio
+
+
+def test_status_clean_after_gemms():
+    api.get_status()
