@@ -155,33 +155,48 @@ def test_philox_matches_triton_interpreter():
         assert np.array_equal(ours, ref), seed
 
 
-def test_philox_words_uniform():
-    w = O.philox_words(0, 1 << 20, seed=1234, offset=0, tag=0)
-    counts = np.bincount((w >> 24).astype(np.int64), minlength=256)
-    exp = w.size / 256
+def test_philox_noise_uniform_and_stream_separation():
+    n = O.philox_noise(0, 1 << 20, seed=1234, offset=0, tag=0)
+    assert n.min() >= 0 and n.max() < 65536
+    counts = np.bincount((n >> 8).astype(np.int64), minlength=256)
+    exp = n.size / 256
     chi2 = ((counts - exp) ** 2 / exp).sum()
     assert chi2 < 350  # 255 dof: p ~ 1e-4 tail
     # tags and offsets give different streams
-    w1 = O.philox_words(0, 4096, seed=1234, offset=0, tag=1)
-    w2 = O.philox_words(0, 4096, seed=1234, offset=1, tag=0)
-    assert not np.array_equal(w[:4096], w1) and not np.array_equal(w[:4096], w2)
+    n1 = O.philox_noise(0, 4096, seed=1234, offset=0, tag=1)
+    n2 = O.philox_noise(0, 4096, seed=1234, offset=1, tag=0)
+    assert not np.array_equal(n[:4096], n1) and not np.array_equal(n[:4096], n2)
+
+
+def test_group_noise_mapping_by_hand():
+    # w = 0x12345678: bytes (low..high) 0x78 0x56 0x34 0x12
+    # n(e0) = 0x34*256 + 0x78 = 0x3478, n(e2) = 0x12*256 + 0x56 = 0x1256
+    # bit-reversed over 16 bits: 0011010001111000 -> 0001111000101100 = 0x1E2C,
+    #                            0001001001010110 -> 0110101001001000 = 0x6A48
+    assert O.group_noise(np.array([0x12345678])).tolist() == [[0x3478, 0x1E2C, 0x1256, 0x6A48]]
+    assert O.bitrev16(np.array([1, 0x00FF, 0x8000])).tolist() == [0x8000, 0xFF00, 1]
+    # the word of group g is word g % 4 of Philox call g / 4
+    w = O.philox4x32_10(3, 0, 1, 9, 77, 0)
+    n = O.philox_noise(48, 16, seed=77, offset=9, tag=1)
+    assert np.array_equal(n.reshape(4, 4), O.group_noise(np.array([int(v) for v in w])))
 
 
 # ---------------------------------------------------------------- stochastic rounding
 
 
-def test_sr_exact_count_over_all_u():
-    """Closed form: over every 24-bit u, the number of round-ups is ceil(f * 2**24)."""
+def test_sr_exact_count_over_all_noise():
+    """Closed form: over every 16-bit n, the number of round-ups is floor(f * 2**16)."""
     rng = np.random.default_rng(5)
-    ys = np.concatenate([rng.uniform(0, 6, 8), rng.uniform(0.5, 1, 2), np.array([0.3, 1.1, 2.9, 5.999])]).astype(F32)
-    u = np.arange(1 << 24, dtype=np.uint32) << np.uint32(8)
+    ys = np.concatenate([rng.uniform(0, 6, 40), rng.uniform(0.5, 1, 10), rng.uniform(0, 0.01, 5),
+                         np.array([0.3, 1.1, 2.9, 5.999, 1.0 + 2.0 ** -20, 0.25])]).astype(F32)
+    nvals = np.arange(1 << 16)
     grid = O.E2M1_MAGNITUDES
     for y in ys:
-        codes = O.e2m1_encode_sr(np.full(u.shape, y, F32), u)
+        codes = O.e2m1_encode_sr(np.full(nvals.shape, y, F32), nvals)
         lo_i = np.searchsorted(grid, float(y), side="right") - 1
         f = (float(y) - grid[lo_i]) / (grid[lo_i + 1] - grid[lo_i])
         ups = int(np.count_nonzero(codes == lo_i + 1))
-        assert ups == int(np.ceil(f * 2 ** 24)), (y, ups)
+        assert ups == int(np.floor(f * 2 ** 16)), (y, ups)
         assert np.all((codes == lo_i) | (codes == lo_i + 1))
 
 
@@ -190,17 +205,19 @@ def test_sr_unbiased_statistically():
     ys = np.concatenate([rng.uniform(-6, 6, 30), np.array([0.1, -0.3, 5.5, -2.25])]).astype(F32)
     n = 1 << 18
     for j, y in enumerate(ys):
-        w = O.philox_words(0, n, seed=99 + j, offset=j, tag=0)
-        q = O.e2m1_decode(O.e2m1_encode_sr(np.full(n, y, F32), w)).astype(np.float64)
+        noise = O.philox_noise(0, n, seed=99 + j, offset=j, tag=0)
+        q = O.e2m1_decode(O.e2m1_encode_sr(np.full(n, y, F32), noise)).astype(np.float64)
         sd = q.std() + 1e-12
-        assert abs(q.mean() - float(y)) < 5 * sd / np.sqrt(n) + 1e-6, y
+        # 16-bit noise: bias below 2**-16 of a grid step (<= 2)
+        assert abs(q.mean() - float(y)) < 5 * sd / np.sqrt(n) + 2.0 * 2 ** -16, y
 
 
 def test_sr_saturates_and_keeps_grid():
-    w = O.philox_words(0, 1024, seed=1, offset=0, tag=0)
-    assert np.all(O.e2m1_encode_sr(np.full(1024, 7.5, F32), w) == 7)
-    assert np.all(O.e2m1_encode_sr(np.full(1024, -6.0, F32), w) == 15)
-    assert np.all(O.e2m1_encode_sr(np.full(1024, 3.0, F32), w) == 5)
+    noise = O.philox_noise(0, 1024, seed=1, offset=0, tag=0)
+    assert np.all(O.e2m1_encode_sr(np.full(1024, 7.5, F32), noise) == 7)
+    assert np.all(O.e2m1_encode_sr(np.full(1024, -6.0, F32), noise) == 15)
+    assert np.all(O.e2m1_encode_sr(np.full(1024, 3.0, F32), noise) == 5)
+    assert np.all(O.e2m1_encode_sr(np.full(1024, -0.0, F32), noise) == 8)
 
 
 # ---------------------------------------------------------------- Hadamard
