@@ -427,6 +427,60 @@ def run_ours(args):
     return 0
 
 
+QUANT_MODES = {
+    "rne_row": dict(emit_row=True),
+    "rne_row_col": dict(emit_row=True, emit_col=True),
+    "act": dict(emit_row=True, emit_col=True, rht_col=True, rht_signs=RHT_SIGNS),
+    "grad": dict(emit_row=True, emit_col=True, stochastic=True, rht_col=True, seed=SR_SEED, rht_signs=RHT_SIGNS),
+    "sr_rht_both": dict(emit_row=True, emit_col=True, stochastic=True, rht_row=True, rht_col=True, seed=SR_SEED,
+                        rht_signs=RHT_SIGNS),
+    "weight": dict(emit_row=True, emit_col=True, block_2d=True),
+}
+
+
+def run_kernel(args):
+    """Single-kernel timing (GEMM or quantiser) on one GPU; used for sweeps and ncu captures."""
+    from nvfp4_pretraining_linear_b200 import api, synthetic as syn
+    torch.cuda.set_device(0)
+    dims = [int(v) for v in args.shape.split(",")]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    if args.kernel == "gemm":
+        M, N, K = dims
+        qa, _ = api.quantize(syn.normal((M, K), 1.0, seed=30, device="cuda"))
+        qb, _ = api.quantize(syn.normal((N, K), 1.0, seed=31, device="cuda"))
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: api.gemm(qa, qb, out=out)  # noqa: E731
+        work, unit = 2.0 * M * N * K, "TFLOP/s"
+    else:
+        R, C = dims
+        kw = dict(QUANT_MODES[args.mode])
+        x = syn.student_t((R, C), 3, 0.1, seed=1, device="cuda")
+        rq = api.QTensor.empty(R, C) if kw.get("emit_row") else None
+        cq = api.QTensor.empty(C, R) if kw.get("emit_col") else None
+        fn = lambda: api.quantize(x, out_row=rq, out_col=cq, **kw)  # noqa: E731
+        layouts = int(bool(kw.get("emit_row"))) + int(bool(kw.get("emit_col")))
+        work, unit = R * C * (4.0 + 0.5625 * layouts), "GB/s"
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    api.get_status()
+    ms = statistics.median(times)
+    rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    print(json.dumps({"kernel": args.kernel, "shape": dims, "mode": args.mode if args.kernel == "quantize" else None,
+                      "ms": ms, "value": rate, "unit": unit, "steps": args.steps, "l2": "flushed (256 MB write)"}),
+          flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -436,7 +490,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["step", "gemm", "quantize"], default="step",
+                    help="step: the contract benchmark; gemm/quantize: one kernel on --shape")
+    ap.add_argument("--shape", default="16384,16384,16384")
+    ap.add_argument("--mode", choices=sorted(QUANT_MODES), default="grad")
     args = ap.parse_args()
+    if args.kernel != "step":
+        return run_kernel(args)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

@@ -192,6 +192,17 @@ nvfp4_status nvfp4_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ld
 nvfp4_status nvfp4_linear_wgrad(const nvfp4_tensor* dYq_col, const nvfp4_tensor* Xq_col, void* dW,
                                 int64_t ldw, int32_t out_dtype, int32_t accumulate, void* stream);
 
+/* Self-check of the conversions the quantiser encodes with.  The kernels use
+ * the sm_100a conversion instructions for E2M1 round-to-nearest-even, E2M1
+ * stochastic rounding (the rule stated for nvfp4_quant_opts.stochastic) and
+ * E4M3 round-to-nearest-even; this call compares each with its definition on
+ * the current device and writes mismatch counts to counts (3 device uint64,
+ * 16-byte aligned): [0] E2M1 RNE over every float bit pattern, [1] E4M3 over
+ * every non-negative finite float, [2] E2M1 stochastic rounding over n_sr
+ * pseudo-random (value, random word) pairs.  All three are 0 on a conforming
+ * GPU.  Asynchronous on `stream`; a few milliseconds of GPU time. */
+nvfp4_status nvfp4_check_conversions(unsigned long long* counts, uint64_t n_sr, void* stream);
+
 /* Synchronise `stream`, then report and clear any device-side error recorded
  * by this library's kernels on the current device since the last call
  * (NVFP4_ERR_TIMEOUT), or a pending CUDA error (NVFP4_ERR_CUDA). */

@@ -5,6 +5,7 @@ torch's current stream, and every step of the computation runs in the CUDA
 library.  There is no CPU path: calls fail when the library or a GPU is missing.
 """
 
+import ctypes
 from dataclasses import dataclass
 from typing import Optional
 
@@ -18,12 +19,7 @@ _workspaces = {}
 
 def _stream_ptr(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes_void(s.cuda_stream)
-
-
-def ctypes_void(v):
-    import ctypes
-    return ctypes.c_void_p(v)
+    return ctypes.c_void_p(s.cuda_stream)
 
 
 def _ptr(t):
@@ -168,6 +164,15 @@ def linear_wgrad(dyq_col: QTensor, xq_col: QTensor, *, out_dtype=torch.bfloat16,
     _lib.check(lib.nvfp4_linear_wgrad(dyq_col.struct(), xq_col.struct(), out.data_ptr(), out.stride(0), code,
                                       int(accumulate), _stream_ptr(stream)))
     return out
+
+
+def check_conversions(n_sr=1 << 26, stream=None):
+    """nvfp4_check_conversions: mismatch counts (E2M1 RNE, E4M3, E2M1 SR) of the hardware
+    conversions against their definitions on the current device; all 0 when conforming."""
+    lib = _lib.load()
+    counts = torch.zeros(4, dtype=torch.int64, device="cuda")
+    _lib.check(lib.nvfp4_check_conversions(counts.data_ptr(), n_sr, _stream_ptr(stream)))
+    return [int(v) for v in counts[:3].cpu().tolist()]
 
 
 def get_status(stream=None):

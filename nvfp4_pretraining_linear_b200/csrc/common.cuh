@@ -78,9 +78,10 @@ __device__ __forceinline__ uint32_t e2m1_rne(float y) {
   return idx | ((__float_as_uint(y) >> 31) << 3);
 }
 
-// Stochastic rounding between the two neighbouring magnitudes lo <= |y| < hi:
-// up iff (w >> 8) * 2^-24 < (|y| - lo) / (hi - lo); |y| >= 6 gives 6.
-__device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t w) {
+// Stochastic rounding between the two neighbouring magnitudes lo <= |y| < hi
+// with a 16-bit random integer n: up iff floor(f * 2^16) + n >= 2^16, f =
+// (|y| - lo) / (hi - lo); |y| >= 6 gives 6; sign kept.
+__device__ __forceinline__ uint32_t e2m1_sr16(float y, uint32_t n) {
   const float a = fabsf(y);
   const uint32_t sign = (__float_as_uint(y) >> 31) << 3;
   if (a >= 6.0f) return 7u | sign;
@@ -88,9 +89,57 @@ __device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t w) {
                       (uint32_t)(a >= 2.0f) + (uint32_t)(a >= 3.0f) + (uint32_t)(a >= 4.0f);
   const float lo_v = lo < 4u ? __fmul_rn((float)lo, 0.5f) : (float)lo - 2.0f;   // 0,.5,1,1.5 | 2,3,4
   const float inv_step = lo < 4u ? 2.0f : (lo < 6u ? 1.0f : 0.5f);
-  const float frac = __fmul_rn(__fsub_rn(a, lo_v), inv_step);                  // exact
-  const float u = __fmul_rn((float)(w >> 8), 5.9604644775390625e-08f);         // * 2^-24, exact
-  return (lo + (u < frac ? 1u : 0u)) | sign;
+  const float frac = __fmul_rn(__fsub_rn(a, lo_v), inv_step);                  // exact, in [0, 1)
+  const uint32_t fixed = (uint32_t)__float2int_rd(__fmul_rn(frac, 65536.0f));  // exact scaling, floor
+  return (lo + (fixed + n >= 65536u ? 1u : 0u)) | sign;
+}
+
+// 16-bit reversal and the random integers of the four elements of a group.
+__device__ __forceinline__ uint32_t bitrev16(uint32_t x) { return __brev(x) >> 16; }
+
+__device__ __forceinline__ uint32_t group_noise(uint32_t w, int e) {
+  const uint32_t n0 = (((w >> 16) & 0xFFu) << 8) | (w & 0xFFu);
+  const uint32_t n2 = (((w >> 24) & 0xFFu) << 8) | ((w >> 8) & 0xFFu);
+  return e == 0 ? n0 : (e == 1 ? bitrev16(n0) : (e == 2 ? n2 : bitrev16(n2)));
+}
+
+// ----------------------------------------------------------------- hardware conversions
+//
+// The sm_100a conversions below are used by the kernels; each was checked on
+// every input it can receive against the definitions above (e2m1_rne: all 2^32
+// float patterns; e4m3_encode: all non-negative floats).
+
+// Eight floats -> eight E2M1 codes (RNE, saturating), element j in nibble j.
+__device__ __forceinline__ uint32_t e2m1x8_rn(const float* y) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+  return out;
+}
+
+// Four floats -> four E2M1 codes with stochastic rounding (element j in nibble
+// j).  The 32-bit word w supplies each element's 16-bit random integer:
+// e0: w[23:16]:w[7:0], e1: its 16-bit reversal, e2: w[31:24]:w[15:8], e3: its
+// reversal; an element rounds up iff floor(f * 2^16) + n >= 2^16.
+__device__ __forceinline__ uint32_t e2m1x4_rs(float y0, float y1, float y2, float y3, uint32_t w) {
+  uint16_t out;
+  asm("cvt.rs.satfinite.e2m1x4.f32 %0, {%1, %2, %3, %4}, %5;"
+      : "=h"(out)
+      : "f"(y3), "f"(y2), "f"(y1), "f"(y0), "r"(w));
+  return out;
+}
+
+// Non-negative float -> E4M3 byte, round to nearest even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_encode_hw(float v) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(out) : "f"(v), "f"(0.0f));
+  return out & 0xFFu;
 }
 
 // ----------------------------------------------------------------- Philox4x32-10
@@ -109,7 +158,8 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
   return c;
 }
 
-// The four random words of elements 4*ctr .. 4*ctr+3 of a layout.
+// The four random words of Philox call `ctr` of a layout: word k drives the
+// four elements 16*ctr + 4k .. 16*ctr + 4k + 3.
 __device__ __forceinline__ uint4 philox_block(uint64_t ctr, uint32_t tag, uint32_t offset,
                                               uint32_t k0, uint32_t k1) {
   return philox4x32_10(make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), tag, offset), k0, k1);
@@ -163,7 +213,7 @@ struct BlockScale {
 __device__ __forceinline__ BlockScale block_scale(float bmax, float S) {
   BlockScale out;
   const float s_f = __fdiv_rn(__fdiv_rn(bmax, 6.0f), S);
-  out.sbyte = e4m3_encode(s_f);
+  out.sbyte = e4m3_encode_hw(s_f);
   const float d = __fmul_rn(e4m3_decode(out.sbyte), S);
   const float r = __fdiv_rn(1.0f, d);
   const bool dead = (out.sbyte == 0u) || (d == 0.0f) || !isfinite(r);

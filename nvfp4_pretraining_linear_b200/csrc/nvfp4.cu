@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "gemm.cuh"
 #include "quantize.cuh"
+#include "selfcheck.cuh"
 
 namespace {
 
@@ -124,53 +125,93 @@ nvfp4::QuantLayout layout_of(const nvfp4_tensor* t) {
   L.tensor_scale = t->tensor_scale;
   L.kgroups = ceil_div(t->cols / 16, 4);
   L.mma_layout = t->scale_layout == NVFP4_SCALE_MMA;
+  L.vec16 = ((t->cols / 2) % 16) == 0;
   return L;
 }
 
-template <bool ER, bool EC, bool SR, bool RR, bool RC, bool TD>
-void launch_quant(const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
-  nvfp4::quantize_kernel<ER, EC, SR, RR, RC, TD><<<grid, nvfp4::kQuantThreads, 0, s>>>(p);
+// Each kernel instantiation needs its large dynamic shared memory opted in once
+// per device; `done` must be a distinct object per instantiation.
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel kernel, int bytes, bool (&done)[kMaxDevices], std::mutex& m) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(m);
+  if (done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
+
+template <bool AM, bool ER, bool EC, bool SR, bool RR, bool RC, bool TD>
+cudaError_t launch_tiles(const CUtensorMap& map, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  static std::mutex m;
+  auto kernel = nvfp4::quant_tile_kernel<AM, ER, EC, SR, RR, RC, TD>;
+  cudaError_t e = ensure_smem(kernel, nvfp4::kQSmemBytes, done, m);
+  if (e != cudaSuccess) return e;
+  kernel<<<grid, nvfp4::kQThreads, nvfp4::kQSmemBytes, s>>>(map, p);
+  return cudaGetLastError();
 }
 
 template <bool ER, bool EC, bool SR, bool RR, bool RC>
-void dispatch_td(bool td, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
+cudaError_t dispatch_td(bool td, const CUtensorMap& m, const nvfp4::QuantParams& p, int g, cudaStream_t s) {
   if constexpr (!SR && !RR && !RC) {
-    if (td) return launch_quant<ER, EC, false, false, false, true>(p, grid, s);
+    if (td) return launch_tiles<false, ER, EC, false, false, false, true>(m, p, g, s);
   }
-  launch_quant<ER, EC, SR, RR, RC, false>(p, grid, s);
+  return launch_tiles<false, ER, EC, SR, RR, RC, false>(m, p, g, s);
 }
 
 template <bool ER, bool EC, bool SR, bool RR>
-void dispatch_rc(bool rc, bool td, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
-  if (rc) return dispatch_td<ER, EC, SR, RR, true>(td, p, grid, s);
-  dispatch_td<ER, EC, SR, RR, false>(td, p, grid, s);
+cudaError_t dispatch_rc(bool rc, bool td, const CUtensorMap& m, const nvfp4::QuantParams& p, int g, cudaStream_t s) {
+  if (rc) return dispatch_td<ER, EC, SR, RR, true>(td, m, p, g, s);
+  return dispatch_td<ER, EC, SR, RR, false>(td, m, p, g, s);
 }
 
 template <bool ER, bool EC, bool SR>
-void dispatch_rr(bool rr, bool rc, bool td, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
-  if (rr) return dispatch_rc<ER, EC, SR, true>(rc, td, p, grid, s);
-  dispatch_rc<ER, EC, SR, false>(rc, td, p, grid, s);
+cudaError_t dispatch_rr(bool rr, bool rc, bool td, const CUtensorMap& m, const nvfp4::QuantParams& p, int g,
+                        cudaStream_t s) {
+  if (rr) return dispatch_rc<ER, EC, SR, true>(rc, td, m, p, g, s);
+  return dispatch_rc<ER, EC, SR, false>(rc, td, m, p, g, s);
 }
 
 template <bool ER, bool EC>
-void dispatch_sr(bool sr, bool rr, bool rc, bool td, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
-  if (sr) return dispatch_rr<ER, EC, true>(rr, rc, td, p, grid, s);
-  dispatch_rr<ER, EC, false>(rr, rc, td, p, grid, s);
+cudaError_t dispatch_sr(bool sr, bool rr, bool rc, bool td, const CUtensorMap& m, const nvfp4::QuantParams& p, int g,
+                        cudaStream_t s) {
+  if (sr) return dispatch_rr<ER, EC, true>(rr, rc, td, m, p, g, s);
+  return dispatch_rr<ER, EC, false>(rr, rc, td, m, p, g, s);
 }
 
-void dispatch_quant(bool er, bool ec, bool sr, bool rr, bool rc, bool td, const nvfp4::QuantParams& p, int grid,
-                    cudaStream_t s) {
-  if (er && ec) return dispatch_sr<true, true>(sr, rr, rc, td, p, grid, s);
-  if (er) return dispatch_sr<true, false>(sr, rr, rc, td, p, grid, s);
-  dispatch_sr<false, true>(sr, rr, rc, td, p, grid, s);
+cudaError_t dispatch_quant(bool er, bool ec, bool sr, bool rr, bool rc, bool td, const CUtensorMap& m,
+                           const nvfp4::QuantParams& p, int g, cudaStream_t s) {
+  if (er && ec) return dispatch_sr<true, true>(sr, rr, rc, td, m, p, g, s);
+  if (er) return dispatch_sr<true, false>(sr, rr, rc, td, m, p, g, s);
+  return dispatch_sr<false, true>(sr, rr, rc, td, m, p, g, s);
 }
 
-void launch_amax(bool rc, bool rr, const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t signs,
-                 unsigned* out, int grid, cudaStream_t s) {
-  if (rc && rr) nvfp4::amax_kernel<true, true><<<grid, nvfp4::kQuantThreads, 0, s>>>(x, rows, cols, ld, signs, out);
-  else if (rc) nvfp4::amax_kernel<true, false><<<grid, nvfp4::kQuantThreads, 0, s>>>(x, rows, cols, ld, signs, out);
-  else if (rr) nvfp4::amax_kernel<false, true><<<grid, nvfp4::kQuantThreads, 0, s>>>(x, rows, cols, ld, signs, out);
-  else nvfp4::amax_kernel<false, false><<<grid, nvfp4::kQuantThreads, 0, s>>>(x, rows, cols, ld, signs, out);
+cudaError_t dispatch_amax(bool rr, bool rc, const CUtensorMap& m, const nvfp4::QuantParams& p, int g, cudaStream_t s) {
+  if (rr && rc) return launch_tiles<true, false, false, false, true, true, false>(m, p, g, s);
+  if (rc) return launch_tiles<true, false, false, false, false, true, false>(m, p, g, s);
+  if (rr) return launch_tiles<true, false, false, false, true, false, false>(m, p, g, s);
+  return launch_tiles<true, false, false, false, false, false, false>(m, p, g, s);
+}
+
+// Tensor map of a BF16 matrix [rows][cols] with row stride ld elements: 128 x 128 tiles,
+// no swizzle, zero fill outside the matrix.
+nvfp4_status make_input_map(CUtensorMap* map, const void* x, int64_t rows, int64_t cols, int64_t ld) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  nvfp4_status st = get_encoder(&encode);
+  if (st != NVFP4_OK) return st;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)nvfp4::kTileCols, (cuuint32_t)nvfp4::kTileRows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled(input) failed (%d)", (int)r);
+  return NVFP4_OK;
 }
 
 }  // namespace
@@ -232,38 +273,42 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
   DeviceInfo* dev;
   if ((st = device_info(&dev)) != NVFP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-
-  const int64_t items = ceil_div(rows, nvfp4::kSlabRows) * ceil_div(cols, nvfp4::kSlabCols);
-  if (!amax) {
-    unsigned* ws = static_cast<unsigned*>(workspace);
-    cudaError_t e = cudaMemsetAsync(ws, 0, 3 * sizeof(unsigned), s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
-    if (items > 0) {
-      const int64_t want = ceil_div(items, nvfp4::kQuantWarps);
-      const int grid = (int)std::min<int64_t>(want, (int64_t)dev->sm_count * 8);
-      launch_amax(opts->rht_col != 0, opts->rht_row != 0, static_cast<const uint16_t*>(x), rows, cols, ld,
-                  opts->rht_signs, ws, grid, s);
-    }
-    amax = reinterpret_cast<const float*>(ws);
+  cudaError_t e;
+  if (rows == 0 || cols == 0) {
+    // nothing to encode: S = 1 for every requested layout
+    nvfp4::empty_tensor_scales_kernel<<<1, 32, 0, s>>>(out_row ? out_row->tensor_scale : nullptr,
+                                                       out_col ? out_col->tensor_scale : nullptr, opts->amax_out);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "quantize launch");
   }
+  CUtensorMap map;
+  if ((st = make_input_map(&map, x, rows, cols, ld)) != NVFP4_OK) return st;
   nvfp4::QuantParams p{};
-  p.x = static_cast<const uint16_t*>(x);
   p.rows = rows;
   p.cols = cols;
-  p.ld = ld;
+  p.tiles_c = ceil_div(cols, nvfp4::kTileCols);
+  p.tiles = ceil_div(rows, nvfp4::kTileRows) * p.tiles_c;
   p.row = layout_of(out_row);
   p.col = layout_of(out_col);
-  p.amax = amax;
   p.amax_out = opts->amax_out;
   p.key0 = (uint32_t)opts->seed;
   p.key1 = (uint32_t)(opts->seed >> 32);
   p.offset = (uint32_t)opts->offset;
   p.signs = opts->rht_signs;
-  const int64_t tiles = ceil_div(ceil_div(rows, nvfp4::kSlabRows), nvfp4::kQuantWarps) * ceil_div(cols, nvfp4::kSlabCols);
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)1 << 30));
-  dispatch_quant(out_row != nullptr, out_col != nullptr, opts->stochastic != 0, opts->rht_row != 0,
-                 opts->rht_col != 0, opts->block_2d != 0, p, grid, s);
-  cudaError_t e = cudaGetLastError();
+  const int grid = (int)std::min<int64_t>(p.tiles, (int64_t)dev->sm_count * nvfp4::kQCtasPerSm);
+  if (!amax) {
+    unsigned* acc = static_cast<unsigned*>(workspace);
+    e = cudaMemsetAsync(acc, 0, 3 * sizeof(unsigned), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+    p.amax_acc = acc;
+    e = dispatch_amax(opts->rht_row != 0, opts->rht_col != 0, map, p, grid, s);
+    if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+    amax = reinterpret_cast<const float*>(acc);
+  }
+  p.amax = amax;
+  p.amax_acc = nullptr;
+  e = dispatch_quant(out_row != nullptr, out_col != nullptr, opts->stochastic != 0, opts->rht_row != 0,
+                     opts->rht_col != 0, opts->block_2d != 0, map, p, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return NVFP4_OK;
 }
@@ -388,6 +433,20 @@ nvfp4_status nvfp4_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ld
 nvfp4_status nvfp4_linear_wgrad(const nvfp4_tensor* dYq_col, const nvfp4_tensor* Xq_col, void* dW, int64_t ldw,
                                 int32_t out_dtype, int32_t accumulate, void* stream) {
   return nvfp4_gemm(dYq_col, Xq_col, dW, ldw, out_dtype, 1.0f, accumulate, stream);
+}
+
+nvfp4_status nvfp4_check_conversions(unsigned long long* counts, uint64_t n_sr, void* stream) {
+  if (!counts) return fail(NVFP4_ERR_INVALID_ARG, "counts is NULL");
+  if (!aligned16(counts)) return fail(NVFP4_ERR_MISALIGNED, "counts is not 16-byte aligned");
+  DeviceInfo* dev;
+  nvfp4_status st = device_info(&dev);
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(counts, 0, 3 * sizeof(unsigned long long), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(counts)");
+  nvfp4::check_conversions_kernel<<<dev->sm_count * 8, 256, 0, s>>>(counts, n_sr);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "check_conversions launch");
 }
 
 nvfp4_status nvfp4_get_status(void* stream) {

@@ -1,4 +1,4 @@
-// NVFP4 quantiser kernels: the amax pass, the fused quantise pass and the
+// NVFP4 quantiser: the amax pass and the fused quantise pass, plus the
 // dequantiser.
 //
 // What they compute follows the format and recipe passages of "Preentrenamiento
@@ -7,24 +7,38 @@
 // blocks for weights; a 16x16 random Hadamard transform on the weight-gradient
 // operands; stochastic rounding for gradients only.
 //
-// Work decomposition (both passes).  A warp owns a slab of 16 rows x 256
-// columns; lane l holds the 16 x 8 sub-block at columns 8l..8l+7, loaded as
-// sixteen 16-byte vectors (each row of the slab is one 512-byte coalesced
-// segment).  The slab contains, per lane, half of 16 row blocks (the other half
-// is the neighbouring lane: one shuffle joins them) and 8 whole column blocks,
-// so the row and the col (transposed) layouts are both produced from one read
-// of the input.  A CTA of 8 warps stacks 8 slabs vertically (128 rows), so that
-// each column's col-layout codes for the CTA are one 64-byte run.
+// Work decomposition.  The input is cut into 128 x 128 BF16 tiles (32 KB).  A
+// persistent grid of CTAs (two per SM) walks the tiles; in each CTA one warp
+// streams tiles into a ring of shared-memory stages with TMA, eight compute
+// warps consume them:
+//   row pass   warp w owns tile rows 16w..16w+15; per instruction a warp reads
+//              two 256-byte rows (16 B per lane, conflict-free), a lane pair
+//              holds one 16-element row block (one shuffle joins the halves);
+//   col pass   thread t owns columns 2(t%64), 2(t%64)+1 and rows 32(t/64)..+31,
+//              reading one 32-bit word per row (a warp reads 128 contiguous
+//              bytes), so its column blocks are whole in registers.
+// Both layouts come from one read of the tile.  Codes go straight to global
+// memory (row: 4 B per lane, 64 B per row segment; col: 16 B per column);
+// block scales are gathered with shuffles into 4-byte (row) or 2-byte (col)
+// stores in the tensor-core scale order.  The same kernel, in amax mode, is the
+// first pass (maximum of |x| and of the transformed blocks).
 #pragma once
+
+#include <cuda.h>
 
 #include "common.cuh"
 
 namespace nvfp4 {
 
-constexpr int kQuantWarps = 8;
-constexpr int kQuantThreads = kQuantWarps * 32;
-constexpr int kSlabRows = 16;
-constexpr int kSlabCols = 256;
+constexpr int kTileRows = 128;
+constexpr int kTileCols = 128;
+constexpr int kTileRowBytes = kTileCols * 2;          // 256
+constexpr int kTileBytes = kTileRows * kTileRowBytes; // 32 KiB
+constexpr int kQStages = 3;
+constexpr int kQComputeWarps = 8;
+constexpr int kQThreads = 32 * (kQComputeWarps + 1);  // 288
+constexpr int kQCtasPerSm = 2;
+constexpr int kQSmemBytes = kQStages * kTileBytes + 256 + 128;
 
 struct QuantLayout {
   uint8_t* codes;       // nullptr when the layout is not emitted
@@ -32,43 +46,27 @@ struct QuantLayout {
   float* tensor_scale;
   int64_t kgroups;      // 4-block groups per row (tensor-core scale layout)
   int32_t mma_layout;   // scales in the tensor-core layout (else row-major)
+  int32_t vec16;        // rows of codes are 16-byte aligned
 };
 
 struct QuantParams {
-  const uint16_t* x;    // BF16 bits
-  int64_t rows, cols, ld;
+  int64_t rows, cols;
+  int64_t tiles_c;      // tiles along cols
+  int64_t tiles;        // total tiles
   QuantLayout row, col;
-  const float* amax;    // 3 floats: raw, transformed col layout, transformed row layout
+  const float* amax;    // quantise mode: 3 floats (raw, transformed col, transformed row)
+  unsigned* amax_acc;   // amax mode: 3 accumulators (float bits)
   float* amax_out;      // nullptr or 3 floats
   uint32_t key0, key1;  // Philox key (seed)
   uint32_t offset;      // Philox counter word 3
   uint32_t signs;       // RHT sign mask
 };
 
-__device__ __forceinline__ int64_t scale_index(const QuantLayout& L, int64_t r, int64_t j, int64_t nblk) {
-  return L.mma_layout ? mma_scale_offset(r, j, L.kgroups) : r * nblk + j;
-}
-
-// Load the 16 x 8 sub-block of lane `lane` (zero rows past `nrows`, zero lanes past `cols`).
-__device__ __forceinline__ void load_slab(const uint16_t* __restrict__ x, int64_t ld, int64_t r0, int64_t c0,
-                                          int nrows, bool active, uint4 (&raw)[16]) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    raw[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (active && i < nrows) raw[i] = __ldg(reinterpret_cast<const uint4*>(x + (r0 + i) * ld + c0));
-  }
-}
-
 __device__ __forceinline__ void unpack8(const uint4& w, float* v) {
   v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x);
   v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
   v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z);
   v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
-}
-
-__device__ __forceinline__ float column_value(const uint4& w, int j) {
-  const uint32_t word = j < 2 ? w.x : (j < 4 ? w.y : (j < 6 ? w.z : w.w));
-  return (j & 1) ? bf16_hi(word) : bf16_lo(word);
 }
 
 // Row-block transform: this lane holds elements e = 8*(lane&1) + j of a 16-group
@@ -97,202 +95,302 @@ __device__ __forceinline__ float absmax8(const float* v) {
   return m;
 }
 
-__device__ __forceinline__ unsigned float_as_ordered(float f) { return __float_as_uint(f); }
-
-// ------------------------------------------------------------------ amax pass
-//
-// out[0] = max |x|; out[1] = max over the col layout's transformed blocks;
-// out[2] = max over the row layout's transformed blocks.  Non-negative floats
-// order like their bit patterns, so atomicMax on the bits is a float max.
-template <bool RHT_COL, bool RHT_ROW>
-__global__ void __launch_bounds__(kQuantThreads) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
-                                                             int64_t cols, int64_t ld, uint32_t signs,
-                                                             unsigned* __restrict__ out) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t row_groups = (rows + kSlabRows - 1) / kSlabRows;
-  const int64_t chunks = (cols + kSlabCols - 1) / kSlabCols;
-  const int64_t items = row_groups * chunks;
-  float m_raw = 0.0f, m_col = 0.0f, m_row = 0.0f;
-  for (int64_t it = (int64_t)blockIdx.x * kQuantWarps + warp; it < items; it += (int64_t)gridDim.x * kQuantWarps) {
-    const int64_t rg = it / chunks, ch = it - rg * chunks;
-    const int64_t r0 = rg * kSlabRows, c0 = ch * kSlabCols + lane * 8;
-    const bool active = c0 < cols;
-    const int nrows = (int)(rows - r0 < kSlabRows ? rows - r0 : kSlabRows);
-    uint4 raw[16];
-    load_slab(x, ld, r0, c0, nrows, active, raw);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float v[8];
-      unpack8(raw[i], v);
-      m_raw = fmaxf(m_raw, absmax8(v));
-      if (RHT_ROW) {
-        rht16_pair(v, signs, lane);
-        m_row = fmaxf(m_row, absmax8(v));
-      }
-    }
-    if (RHT_COL) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float v[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = column_value(raw[i], j);
-        rht16(v, signs);
-        float m = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-        m_col = fmaxf(m_col, m);
-      }
-    }
-  }
-#pragma unroll
-  for (int s = 16; s > 0; s >>= 1) {
-    m_raw = fmaxf(m_raw, __shfl_xor_sync(0xFFFFFFFFu, m_raw, s));
-    if (RHT_COL) m_col = fmaxf(m_col, __shfl_xor_sync(0xFFFFFFFFu, m_col, s));
-    if (RHT_ROW) m_row = fmaxf(m_row, __shfl_xor_sync(0xFFFFFFFFu, m_row, s));
-  }
-  __shared__ float red[3][kQuantWarps];
-  if (lane == 0) {
-    red[0][warp] = m_raw;
-    red[1][warp] = m_col;
-    red[2][warp] = m_row;
-  }
-  __syncthreads();
-  if (threadIdx.x < 3) {
-    float m = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kQuantWarps; ++w) m = fmaxf(m, red[threadIdx.x][w]);
-    if (threadIdx.x == 0 || (threadIdx.x == 1 && RHT_COL) || (threadIdx.x == 2 && RHT_ROW))
-      atomicMax(out + threadIdx.x, float_as_ordered(m));
-  }
-}
-
-// ------------------------------------------------------------------ quantise pass
+__device__ __forceinline__ float absmax16(const float* v) { return fmaxf(absmax8(v), absmax8(v + 8)); }
 
 template <bool SR>
-__device__ __forceinline__ uint32_t encode8(const float* v, float r, uint4 w0, uint4 w1) {
-  uint32_t packed = 0;
-  const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+__device__ __forceinline__ uint32_t encode8(const float* v, float r, uint32_t w0, uint32_t w1) {
+  float y[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float y = __fmul_rn(v[j], r);
-    const uint32_t c = SR ? e2m1_sr(y, words[j]) : e2m1_rne(y);
-    packed |= c << (4 * j);
-  }
-  return packed;
+  for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(v[j], r);
+  if (SR) return e2m1x4_rs(y[0], y[1], y[2], y[3], w0) | (e2m1x4_rs(y[4], y[5], y[6], y[7], w1) << 16);
+  return e2m1x8_rn(y);
 }
 
-template <bool EMIT_ROW, bool EMIT_COL, bool SR, bool RHT_ROW, bool RHT_COL, bool TWO_D>
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float amax_raw = p.amax[0];
-  const float amax_col = RHT_COL ? p.amax[1] : amax_raw;
-  const float amax_row = RHT_ROW ? p.amax[2] : amax_raw;
-  const float S_row = tensor_scale_from_amax(amax_row);
-  const float S_col = tensor_scale_from_amax(amax_col);
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    if (EMIT_ROW) *p.row.tensor_scale = S_row;
-    if (EMIT_COL) *p.col.tensor_scale = S_col;
-    if (p.amax_out) {
-      p.amax_out[0] = amax_raw;
-      p.amax_out[1] = RHT_COL ? amax_col : 0.0f;
-      p.amax_out[2] = RHT_ROW ? amax_row : 0.0f;
+__device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                              uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// AMAX: first pass (maxima only).  Otherwise ER / EC emit the row / col layout,
+// SR stochastic rounding, RR / RC the transform on the row / col layout, TD
+// 16x16 blocks.
+template <bool AMAX, bool ER, bool EC, bool SR, bool RR, bool RC, bool TD>
+__global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
+    quant_tile_kernel(const __grid_constant__ CUtensorMap xmap, const QuantParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_base = smem_base + kQStages * kTileBytes;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kQStages * kTileBytes + 8 * 2 * kQStages);
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (kQStages + s); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), kQComputeWarps);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued[kQStages] = {};
+      uint32_t issued_phase[kQStages] = {};
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int64_t tr = t / p.tiles_c, tc = t - tr * p.tiles_c;
+        mbar_arrive_expect_tx(full_bar(stage), kTileBytes);
+        tma_load_tile(smem_base + stage * kTileBytes, &xmap, (int32_t)(tc * kTileCols), (int32_t)(tr * kTileRows),
+                      full_bar(stage));
+        issued[stage] = true;
+        issued_phase[stage] = phase;
+        if (++stage == kQStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        // wind down: let every load already issued land before the CTA exits
+        for (int s = 0; s < kQStages; ++s) {
+          if (!issued[s]) continue;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(full_bar(s), issued_phase[s]) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ compute warps
+  const int cw = warp - 1;                 // 0..7
+  const int ct = threadIdx.x - 32;         // 0..255
+  const int64_t rows = p.rows, cols = p.cols;
+  float S_row = 1.0f, S_col = 1.0f;
+  if (!AMAX) {
+    const float amax_raw = p.amax[0];
+    const float amax_col = RC ? p.amax[1] : amax_raw;
+    const float amax_row = RR ? p.amax[2] : amax_raw;
+    S_row = tensor_scale_from_amax(amax_row);
+    S_col = tensor_scale_from_amax(amax_col);
+    if (blockIdx.x == 0 && ct == 0) {
+      if (ER) *p.row.tensor_scale = S_row;
+      if (EC) *p.col.tensor_scale = S_col;
+      if (p.amax_out) {
+        p.amax_out[0] = amax_raw;
+        p.amax_out[1] = RC ? amax_col : 0.0f;
+        p.amax_out[2] = RR ? amax_row : 0.0f;
+      }
     }
   }
-  const int64_t rows = p.rows, cols = p.cols;
-  const int64_t row_groups = (rows + kSlabRows - 1) / kSlabRows;
-  const int64_t chunks = (cols + kSlabCols - 1) / kSlabCols;
-  const int64_t row_tiles = (row_groups + kQuantWarps - 1) / kQuantWarps;
-  const int64_t tiles = row_tiles * chunks;
+  float m_raw = 0.0f, m_col = 0.0f, m_row = 0.0f;
   const int64_t nblk_row = cols / 16, nblk_col = rows / 16;
+  const int64_t rows_padded = (rows + 127) & ~int64_t(127);
 
-  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-    const int64_t rt = t / chunks, ch = t - rt * chunks;
-    const int64_t rg = rt * kQuantWarps + warp;
-    if (rg >= row_groups) continue;                       // whole warp
-    const int64_t r0 = rg * kSlabRows, c0 = ch * kSlabCols + lane * 8;
-    const bool active = c0 < cols;
-    const int nrows = (int)(rows - r0 < kSlabRows ? rows - r0 : kSlabRows);
-    uint4 raw[16];
-    load_slab(p.x, p.ld, r0, c0, nrows, active, raw);
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x) {
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(full_bar(stage), phase, abort_flag))) break;
+    const uint8_t* in = smem + stage * kTileBytes;
+    const int64_t tr = t / p.tiles_c, tc = t - tr * p.tiles_c;
+    const int64_t r_base = tr * kTileRows, c_base = tc * kTileCols;
 
-    float tile_max = 0.0f;
-    if (TWO_D) {
+    // ---------------------------------------------------------------- row pass
+    if (AMAX || ER) {
+      const int ch = lane & 15;            // 16-byte chunk: columns 8ch .. 8ch+7
+      const int64_t c = c_base + ch * 8;
+      float tile_max = 0.0f;
+      if (TD) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float v[8];
-        unpack8(raw[i], v);
-        tile_max = fmaxf(tile_max, absmax8(v));
+        for (int it = 0; it < 8; ++it) {
+          const int rl = cw * 16 + it * 2 + (lane >> 4);
+          float v[8];
+          unpack8(*reinterpret_cast<const uint4*>(in + rl * kTileRowBytes + ch * 16), v);
+          tile_max = fmaxf(tile_max, absmax8(v));
+        }
+        tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 1));
+        tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 16));
       }
-      tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 1));
-    }
-
-    if (EMIT_ROW) {
       BlockScale tbs;
-      if (TWO_D) tbs = block_scale(tile_max, S_row);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        if (i >= nrows) break;                            // warp-uniform
-        const int64_t r = r0 + i;
+      if (TD && !AMAX) tbs = block_scale(tile_max, S_row);
+#pragma unroll 2
+      for (int it = 0; it < 8; ++it) {
+        const int rl = cw * 16 + it * 2 + (lane >> 4);
+        const int64_t r = r_base + rl;
         float v[8];
-        unpack8(raw[i], v);
-        if (RHT_ROW) rht16_pair(v, p.signs, lane);
+        unpack8(*reinterpret_cast<const uint4*>(in + rl * kTileRowBytes + ch * 16), v);
+        if (AMAX) {
+          m_raw = fmaxf(m_raw, absmax8(v));
+          if (RR) {
+            rht16_pair(v, p.signs, lane);
+            m_row = fmaxf(m_row, absmax8(v));
+          }
+          continue;
+        }
+        if (RR) rht16_pair(v, p.signs, lane);
         BlockScale bs;
-        if (TWO_D) {
+        if (TD) {
           bs = tbs;
         } else {
           float m = absmax8(v);
           m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
           bs = block_scale(m, S_row);
         }
-        uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+        uint32_t w0 = 0, w1 = 0;
         if (SR) {
-          const uint64_t ctr = (uint64_t)(r * cols + c0) >> 2;
-          w0 = philox_block(ctr, 0u, p.offset, p.key0, p.key1);
-          w1 = philox_block(ctr + 1, 0u, p.offset, p.key0, p.key1);
+          const uint4 w =
+              philox_block((uint64_t)(r * cols + c_base + (ch >> 1) * 16) >> 4, 0u, p.offset, p.key0, p.key1);
+          w0 = (ch & 1) ? w.z : w.x;
+          w1 = (ch & 1) ? w.w : w.y;
         }
         uint32_t packed = encode8<SR>(v, bs.r, w0, w1);
-        if (bs.r == 0.0f) packed = 0u;                    // dead block: all-zero codes
-        if (active) {
-          *reinterpret_cast<uint32_t*>(p.row.codes + r * (cols / 2) + c0 / 2) = packed;
-          if (!(lane & 1)) p.row.scales[scale_index(p.row, r, c0 / 16, nblk_row)] = (uint8_t)bs.sbyte;
+        if (bs.r == 0.0f) packed = 0u;                       // dead block: all-zero codes
+        const bool row_ok = r < rows;
+        if (row_ok && c < cols) *reinterpret_cast<uint32_t*>(p.row.codes + r * (cols / 2) + c / 2) = packed;
+        // block scales: the even lane of each pair holds block j = ch / 2
+        if (p.row.mma_layout) {
+          // blocks 4g .. 4g+3 are 4 consecutive bytes: gather them on lanes ch = 0 and 8
+          const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 2);
+          const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 4);
+          const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 6);
+          if ((ch & 7) == 0) {
+            const int64_t j = c_base / 16 + (ch >> 1);
+            if ((j >> 2) < p.row.kgroups && r < rows_padded)
+              *reinterpret_cast<uint32_t*>(p.row.scales + mma_scale_offset(r, j, p.row.kgroups)) =
+                  bs.sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24);
+          }
+        } else if (!(ch & 1) && row_ok && c < cols) {
+          p.row.scales[r * nblk_row + c / 16] = (uint8_t)bs.sbyte;
         }
       }
     }
 
-    if (EMIT_COL) {
-      BlockScale tbs;
-      if (TWO_D) tbs = block_scale(tile_max, S_col);
-#pragma unroll 1
-      for (int j = 0; j < 8; ++j) {
-        float v[16];
+    // ---------------------------------------------------------------- col pass
+    if ((AMAX && RC) || (!AMAX && EC)) {
+      const int cp = ct & 63, q = ct >> 6;
+      uint32_t codes[2][2][2];
+      uint32_t sb[2][2];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = column_value(raw[i], j);
-        if (RHT_COL) rht16(v, p.signs);
-        BlockScale bs;
-        if (TWO_D) {
-          bs = tbs;
+      for (int b = 0; b < 2; ++b) {
+        const int rl0 = q * 32 + b * 16;
+        float va[16], vb[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(in + (rl0 + i) * kTileRowBytes + cp * 4);
+          va[i] = bf16_lo(w);
+          vb[i] = bf16_hi(w);
+        }
+        if (RC) {
+          rht16(va, p.signs);
+          rht16(vb, p.signs);
+        }
+        if (AMAX) {
+          m_col = fmaxf(m_col, fmaxf(absmax16(va), absmax16(vb)));
+          continue;
+        }
+        float ma, mb;
+        if (TD) {
+          // the 16x16 tile spans the 8 lanes holding columns 16*(cp/8) .. +15
+          float m = fmaxf(absmax16(va), absmax16(vb));
+          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+          ma = mb = m;
         } else {
-          float m = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-          bs = block_scale(m, S_col);
+          ma = absmax16(va);
+          mb = absmax16(vb);
         }
-        const int64_t c = c0 + j;
-        uint4 w[4] = {};
-        if (SR) {
-          const uint64_t ctr = (uint64_t)(c * rows + r0) >> 2;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) w[q] = philox_block(ctr + q, 1u, p.offset, p.key0, p.key1);
+        for (int k = 0; k < 2; ++k) {
+          const float* v = k ? vb : va;
+          const BlockScale bs = block_scale(k ? mb : ma, S_col);
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (SR) {
+            const int64_t c = c_base + 2 * cp + k;
+            w = philox_block((uint64_t)(c * rows + r_base + rl0) >> 4, 1u, p.offset, p.key0, p.key1);
+          }
+          uint32_t lo = encode8<SR>(v, bs.r, w.x, w.y);
+          uint32_t hi = encode8<SR>(v + 8, bs.r, w.z, w.w);
+          if (bs.r == 0.0f) lo = hi = 0u;
+          codes[k][b][0] = lo;
+          codes[k][b][1] = hi;
+          sb[k][b] = bs.sbyte;
         }
-        uint32_t lo = encode8<SR>(v, bs.r, w[0], w[1]);
-        uint32_t hi = encode8<SR>(v + 8, bs.r, w[2], w[3]);
-        if (bs.r == 0.0f) lo = hi = 0u;
-        if (active) {
-          *reinterpret_cast<uint2*>(p.col.codes + c * (rows / 2) + r0 / 2) = make_uint2(lo, hi);
-          p.col.scales[scale_index(p.col, c, r0 / 16, nblk_col)] = (uint8_t)bs.sbyte;
+      }
+      if (!AMAX) {
+        const int64_t rg = r_base + q * 32;                  // first of this thread's 32 rows
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int64_t c = c_base + 2 * cp + k;
+          if (c >= cols || rg >= rows) continue;
+          uint8_t* dst = p.col.codes + c * (rows / 2) + rg / 2;
+          const bool both = rg + 16 < rows;
+          if (p.col.vec16 && both) {
+            *reinterpret_cast<uint4*>(dst) =
+                make_uint4(codes[k][0][0], codes[k][0][1], codes[k][1][0], codes[k][1][1]);
+          } else {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(codes[k][0][0], codes[k][0][1]);
+            if (both) *reinterpret_cast<uint2*>(dst + 8) = make_uint2(codes[k][1][0], codes[k][1][1]);
+          }
+          const int64_t j0 = rg / 16;                        // even: blocks j0, j0+1 are adjacent bytes
+          if (p.col.mma_layout) {
+            if ((j0 >> 2) < p.col.kgroups)
+              *reinterpret_cast<uint16_t*>(p.col.scales + mma_scale_offset(c, j0, p.col.kgroups)) =
+                  (uint16_t)(sb[k][0] | (sb[k][1] << 8));
+          } else {
+            p.col.scales[c * nblk_col + j0] = (uint8_t)sb[k][0];
+            if (both) p.col.scales[c * nblk_col + j0 + 1] = (uint8_t)sb[k][1];
+          }
         }
       }
     }
+
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar(stage));
+    if (++stage == kQStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+
+  if (AMAX) {
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) {
+      m_raw = fmaxf(m_raw, __shfl_xor_sync(0xFFFFFFFFu, m_raw, s));
+      m_col = fmaxf(m_col, __shfl_xor_sync(0xFFFFFFFFu, m_col, s));
+      m_row = fmaxf(m_row, __shfl_xor_sync(0xFFFFFFFFu, m_row, s));
+    }
+    if (lane == 0) {
+      // non-negative floats order like their bit patterns
+      atomicMax(p.amax_acc + 0, __float_as_uint(m_raw));
+      if (RC) atomicMax(p.amax_acc + 1, __float_as_uint(m_col));
+      if (RR) atomicMax(p.amax_acc + 2, __float_as_uint(m_row));
+    }
+  }
+}
+
+// Tensor scales of an empty tensor (no tile to visit): S = 1, maxima 0.
+__global__ void empty_tensor_scales_kernel(float* row_scale, float* col_scale, float* amax_out) {
+  if (threadIdx.x == 0) {
+    if (row_scale) *row_scale = 1.0f;
+    if (col_scale) *col_scale = 1.0f;
+    if (amax_out) amax_out[0] = amax_out[1] = amax_out[2] = 0.0f;
   }
 }
 
