@@ -192,6 +192,30 @@ nvfp4_status nvfp4_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ld
 nvfp4_status nvfp4_linear_wgrad(const nvfp4_tensor* dYq_col, const nvfp4_tensor* Xq_col, void* dW,
                                 int64_t ldw, int32_t out_dtype, int32_t accumulate, void* stream);
 
+/* nvfp4_quantize without a workspace argument, for callers that cannot
+ * allocate device memory at the point of the call -- for example a host thread
+ * that must not take the allocator's device-wide locks or trigger its implicit
+ * synchronisation, code that runs inside a fixed, pre-planned memory budget, or
+ * a foreign-language caller that has no device allocator at hand.  No
+ * counterpart on the source pages: it exists for how the library is called.
+ *   Arguments, outputs and results are those of nvfp4_quantize.
+ *   Scratch: a 256-byte array of device memory inside the library, held by
+ *   every GPU that loads it until the process exits; this call allocates and
+ *   frees nothing.  The quantiser needs 12 bytes of it for any tensor size;
+ *   a scratch requirement above 256 bytes is rejected with
+ *   NVFP4_ERR_WORKSPACE.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current and caches it; make that
+ *   first call before any stream capture.
+ *   Sharing: all calls on a device use the same array and leave their last
+ *   values in it; each call clears what it needs.  Calls whose work overlaps
+ *   on the GPU (different streams, no ordering between them) race on the
+ *   array and may produce wrong tensor scales; order them on one stream or
+ *   use nvfp4_quantize with a workspace per stream. */
+nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                    const nvfp4_quant_opts* opts, nvfp4_tensor* out_row,
+                                    nvfp4_tensor* out_col, void* stream);
+
 /* Self-check of the conversions the quantiser encodes with.  The kernels use
  * the sm_100a conversion instructions for E2M1 round-to-nearest-even, E2M1
  * stochastic rounding (the rule stated for nvfp4_quant_opts.stochastic) and

@@ -73,6 +73,7 @@ SIGNATURES = {
     "nvfp4_linear_dgrad": (c_int32, [c_void_p, c_int64, c_int64, c_int64, T_P, c_void_p, c_int64, c_int32, T_P, T_P,
                                      c_uint64, c_uint64, c_uint32, c_void_p, c_size_t, c_void_p]),
     "nvfp4_linear_wgrad": (c_int32, [T_P, T_P, c_void_p, c_int64, c_int32, c_int32, c_void_p]),
+    "nvfp4_quantize_noalloc": (c_int32, [c_void_p, c_int64, c_int64, c_int64, O_P, T_P, T_P, c_void_p]),
     "nvfp4_check_conversions": (c_int32, [c_void_p, c_uint64, c_void_p]),
     "nvfp4_get_status": (c_int32, [c_void_p]),
     "nvfp4_last_error_string": (ctypes.c_char_p, []),

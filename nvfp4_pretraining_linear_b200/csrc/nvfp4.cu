@@ -214,6 +214,35 @@ nvfp4_status make_input_map(CUtensorMap* map, const void* x, int64_t rows, int64
   return NVFP4_OK;
 }
 
+// ------------------------------------------------------------------ fixed scratch
+//
+// Scratch for nvfp4_quantize_noalloc: the quantiser's amax accumulators live in
+// this module-scope device array instead of a caller workspace.  Every GPU that
+// loads the library holds these bytes until the process exits.  In host code
+// the name is only a stand-in for the symbol: its device address is fetched
+// with cudaGetSymbolAddress once per device and cached.
+constexpr size_t kNoAllocScratchBytes = 256;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_addr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+nvfp4_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(NVFP4_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return NVFP4_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -433,6 +462,22 @@ nvfp4_status nvfp4_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ld
 nvfp4_status nvfp4_linear_wgrad(const nvfp4_tensor* dYq_col, const nvfp4_tensor* Xq_col, void* dW, int64_t ldw,
                                 int32_t out_dtype, int32_t accumulate, void* stream) {
   return nvfp4_gemm(dYq_col, Xq_col, dW, ldw, out_dtype, 1.0f, accumulate, stream);
+}
+
+nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                    const nvfp4_quant_opts* opts, nvfp4_tensor* out_row, nvfp4_tensor* out_col,
+                                    void* stream) {
+  // The scratch this call needs must fit the fixed array; it does not grow with
+  // the tensor (three amax accumulators), but the check keeps the limit explicit.
+  const size_t need = kWorkspaceBytes;
+  if (need > kNoAllocScratchBytes)
+    return fail(NVFP4_ERR_WORKSPACE, "quantize needs %zu bytes of scratch, the fixed scratch holds %zu", need,
+                kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  nvfp4_status st = noalloc_scratch(&scratch);
+  if (st != NVFP4_OK) return st;
+  // the quantiser clears the accumulators it uses at the start of every call
+  return nvfp4_quantize(x, rows, cols, ld, opts, out_row, out_col, scratch, kNoAllocScratchBytes, stream);
 }
 
 nvfp4_status nvfp4_check_conversions(unsigned long long* counts, uint64_t n_sr, void* stream) {
