@@ -11,14 +11,15 @@
 // persistent grid of CTAs (two per SM) walks the tiles; in each CTA one warp
 // streams tiles into a ring of shared-memory stages with TMA, eight compute
 // warps consume them:
-//   row pass   warp w owns tile rows 16w..16w+15; per instruction a warp reads
-//              two 256-byte rows (16 B per lane, conflict-free), a lane pair
-//              holds one 16-element row block (one shuffle joins the halves);
+//   row pass   warp w owns tile rows 16w..16w+15; a lane owns one whole
+//              16-element row block (a warp covers 4 rows x 128 columns per
+//              step, reading each 32-byte block as two 16-byte halves ordered
+//              so that every quarter-warp hits distinct banks);
 //   col pass   thread t owns columns 2(t%64), 2(t%64)+1 and rows 32(t/64)..+31,
 //              reading one 32-bit word per row (a warp reads 128 contiguous
 //              bytes), so its column blocks are whole in registers.
 // Both layouts come from one read of the tile.  Codes go straight to global
-// memory (row: 4 B per lane, 64 B per row segment; col: 16 B per column);
+// memory (row: 8 B per lane, 64 B per row segment; col: 16 B per column);
 // block scales are gathered with shuffles into 4-byte (row) or 2-byte (col)
 // stores in the tensor-core scale order.  The same kernel, in amax mode, is the
 // first pass (maximum of |x| and of the transformed blocks).
@@ -86,6 +87,22 @@ __device__ __forceinline__ void rht16_pair(float* v, uint32_t signs, int lane) {
   }
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(v[j], 0.25f);
+}
+
+// Butterfly stages h = 1, 2, 4, 8 and the 1/4 normalisation over 16 values whose
+// signs were already applied (the transform of rht16 after its sign flips).
+__device__ __forceinline__ void wht16_scaled(float* v) {
+  wht_stage<16>(v, 1);
+  wht_stage<16>(v, 2);
+  wht_stage<16>(v, 4);
+  wht_stage<16>(v, 8);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], 0.25f);
+}
+
+// Sign-flip mask for a word holding two BF16 elements that both have group index i.
+__device__ __forceinline__ uint32_t pair_sign_mask(uint32_t signs, int i) {
+  return ((signs >> i) & 1u) * 0x80008000u;
 }
 
 __device__ __forceinline__ float absmax8(const float* v) {
@@ -212,70 +229,86 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     const int64_t r_base = tr * kTileRows, c_base = tc * kTileCols;
 
     // ---------------------------------------------------------------- row pass
-    if (AMAX || ER) {
-      const int ch = lane & 15;            // 16-byte chunk: columns 8ch .. 8ch+7
-      const int64_t c = c_base + ch * 8;
+    // lane (rsub, b): 16-element block b (columns 16b..16b+15) of tile row
+    // 16cw + 4it + rsub.  The two 16-byte halves are read in the order that
+    // keeps each quarter-warp on distinct banks (blocks 4..7 read their upper
+    // half first); results are put back in element order afterwards.
+    if ((AMAX && !RC) || (AMAX && RR) || (!AMAX && ER)) {
+      const int b = lane & 7, rsub = lane >> 3;
+      const int swap = (b >> 2) & 1;
+      const int64_t c = c_base + b * 16;
       float tile_max = 0.0f;
-      if (TD) {
+      if (TD && !AMAX) {
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int rl = cw * 16 + it * 2 + (lane >> 4);
-          float v[8];
-          unpack8(*reinterpret_cast<const uint4*>(in + rl * kTileRowBytes + ch * 16), v);
-          tile_max = fmaxf(tile_max, absmax8(v));
+        for (int it = 0; it < 4; ++it) {
+          const uint8_t* src = in + (cw * 16 + it * 4 + rsub) * kTileRowBytes + b * 32;
+          float v[16];
+          unpack8(*reinterpret_cast<const uint4*>(src + 16 * swap), v);
+          unpack8(*reinterpret_cast<const uint4*>(src + 16 * (1 - swap)), v + 8);
+          tile_max = fmaxf(tile_max, absmax16(v));
         }
-        tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 1));
+        tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 8));
         tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 16));
       }
       BlockScale tbs;
       if (TD && !AMAX) tbs = block_scale(tile_max, S_row);
 #pragma unroll 2
-      for (int it = 0; it < 8; ++it) {
-        const int rl = cw * 16 + it * 2 + (lane >> 4);
+      for (int it = 0; it < 4; ++it) {
+        const int rl = cw * 16 + it * 4 + rsub;
         const int64_t r = r_base + rl;
-        float v[8];
-        unpack8(*reinterpret_cast<const uint4*>(in + rl * kTileRowBytes + ch * 16), v);
-        if (AMAX) {
-          m_raw = fmaxf(m_raw, absmax8(v));
-          if (RR) {
-            rht16_pair(v, p.signs, lane);
-            m_row = fmaxf(m_row, absmax8(v));
+        const uint8_t* src = in + rl * kTileRowBytes + b * 32;
+        uint4 h0 = *reinterpret_cast<const uint4*>(src + 16 * swap);
+        uint4 h1 = *reinterpret_cast<const uint4*>(src + 16 * (1 - swap));
+        float v[16];
+        if (RR) {
+          // the transform needs element order: undo the read order, fold in the signs
+          const uint4 lo = swap ? h1 : h0, hi = swap ? h0 : h1;
+          const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t m = (((p.signs >> (2 * k)) & 1u) << 15) | (((p.signs >> (2 * k + 1)) & 1u) << 31);
+            v[2 * k] = bf16_lo(w[k] ^ m);
+            v[2 * k + 1] = bf16_hi(w[k] ^ m);
           }
-          continue;
-        }
-        if (RR) rht16_pair(v, p.signs, lane);
-        BlockScale bs;
-        if (TD) {
-          bs = tbs;
+          if (AMAX) {
+            m_raw = fmaxf(m_raw, absmax16(v));   // the sign flips leave |x| unchanged
+            wht16_scaled(v);
+            m_row = fmaxf(m_row, absmax16(v));
+            continue;
+          }
+          wht16_scaled(v);
         } else {
-          float m = absmax8(v);
-          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-          bs = block_scale(m, S_row);
+          unpack8(h0, v);
+          unpack8(h1, v + 8);
+          if (AMAX) {
+            m_raw = fmaxf(m_raw, absmax16(v));
+            continue;
+          }
         }
-        uint32_t w0 = 0, w1 = 0;
-        if (SR) {
-          const uint4 w =
-              philox_block((uint64_t)(r * cols + c_base + (ch >> 1) * 16) >> 4, 0u, p.offset, p.key0, p.key1);
-          w0 = (ch & 1) ? w.z : w.x;
-          w1 = (ch & 1) ? w.w : w.y;
-        }
-        uint32_t packed = encode8<SR>(v, bs.r, w0, w1);
-        if (bs.r == 0.0f) packed = 0u;                       // dead block: all-zero codes
-        const bool row_ok = r < rows;
-        if (row_ok && c < cols) *reinterpret_cast<uint32_t*>(p.row.codes + r * (cols / 2) + c / 2) = packed;
-        // block scales: the even lane of each pair holds block j = ch / 2
+        const BlockScale bs = TD ? tbs : block_scale(absmax16(v), S_row);
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (SR) w = philox_block((uint64_t)(r * cols + c) >> 4, 0u, p.offset, p.key0, p.key1);
+        // v[0..7] holds the half read first; pick the matching random words
+        const bool phys_swap = swap && !RR;
+        const uint32_t wa0 = phys_swap ? w.z : w.x, wa1 = phys_swap ? w.w : w.y;
+        const uint32_t wb0 = phys_swap ? w.x : w.z, wb1 = phys_swap ? w.y : w.w;
+        const uint32_t ca = encode8<SR>(v, bs.r, wa0, wa1);
+        const uint32_t cb = encode8<SR>(v + 8, bs.r, wb0, wb1);
+        uint32_t lo = phys_swap ? cb : ca, hi = phys_swap ? ca : cb;
+        if (bs.r == 0.0f) lo = hi = 0u;                     // dead block: all-zero codes
+        if (r < rows && c < cols) *reinterpret_cast<uint2*>(p.row.codes + r * (cols / 2) + c / 2) = make_uint2(lo, hi);
         if (p.row.mma_layout) {
-          // blocks 4g .. 4g+3 are 4 consecutive bytes: gather them on lanes ch = 0 and 8
-          const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 2);
-          const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 4);
-          const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 6);
-          if ((ch & 7) == 0) {
-            const int64_t j = c_base / 16 + (ch >> 1);
+          // blocks 4g .. 4g+3 of a row are 4 consecutive bytes: gather them on lanes b = 0 and 4
+          const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 1);
+          const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 2);
+          const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 3);
+          if ((b & 3) == 0) {
+            const int64_t j = c / 16;
             if ((j >> 2) < p.row.kgroups && r < rows_padded)
               *reinterpret_cast<uint32_t*>(p.row.scales + mma_scale_offset(r, j, p.row.kgroups)) =
                   bs.sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24);
           }
-        } else if (!(ch & 1) && row_ok && c < cols) {
+        } else if (r < rows && c < cols) {
           p.row.scales[r * nblk_row + c / 16] = (uint8_t)bs.sbyte;
         }
       }
@@ -292,13 +325,15 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
         float va[16], vb[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(in + (rl0 + i) * kTileRowBytes + cp * 4);
+          uint32_t w = *reinterpret_cast<const uint32_t*>(in + (rl0 + i) * kTileRowBytes + cp * 4);
+          if (RC) w ^= pair_sign_mask(p.signs, i);        // element i of both column groups
           va[i] = bf16_lo(w);
           vb[i] = bf16_hi(w);
         }
+        if (AMAX) m_raw = fmaxf(m_raw, fmaxf(absmax16(va), absmax16(vb)));   // signs leave |x| unchanged
         if (RC) {
-          rht16(va, p.signs);
-          rht16(vb, p.signs);
+          wht16_scaled(va);
+          wht16_scaled(vb);
         }
         if (AMAX) {
           m_col = fmaxf(m_col, fmaxf(absmax16(va), absmax16(vb)));
