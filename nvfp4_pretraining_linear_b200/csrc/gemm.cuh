@@ -46,9 +46,9 @@ constexpr int TMEM_COLS = 512;
 constexpr int ACC_COL = 0;              // 256 FP32 columns
 constexpr int SFA_COL = 256;            // 4 columns per MMA k-step -> 16
 constexpr int SFB_COL = 256 + 16;       // 8 columns per MMA k-step -> 32
-constexpr int NUM_THREADS = 192;
 constexpr int EPI_WARP0 = 2;
-constexpr int NUM_EPI_WARPS = 4;
+constexpr int NUM_EPI_WARPS = 8;                  // two per tensor-memory lane quarter
+constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
 
@@ -58,7 +58,8 @@ struct Params {
   int32_t group_m;
   const uint8_t* sfa;       // tensor-core scale layout of A
   const uint8_t* sfb;
-  int64_t sf_kgroups;       // 64-element K groups per 128-row scale block (= K / 64)
+  int64_t sf_kgroups;       // 64-element K groups per 128-row scale block of B (= K / 64)
+  int64_t sf_kgroups_a;     // the same for A
   const float* scale_a;
   const float* scale_b;
   float alpha;
@@ -125,7 +126,8 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
 }
 
 // 32 lanes x 32 columns of 32-bit accumulator: lane i of the warp gets row i.
-__device__ __forceinline__ void tc_load_32cols(uint32_t taddr, uint32_t (&r)[32]) {
+// Asynchronous: the registers are valid after tc_wait_loads().
+__device__ __forceinline__ void tc_load_32cols(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -135,7 +137,49 @@ __device__ __forceinline__ void tc_load_32cols(uint32_t taddr, uint32_t (&r)[32]
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_wait_loads() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Scale 32 accumulator columns by g and store them (BF16 or FP32, optionally
+// adding the existing values) at crow (row-major C, 16-byte aligned).
+__device__ __forceinline__ void store_32cols(const Params& p, const uint32_t* r, float g, void* crow_v) {
+  if (p.out_f32) {
+    float* crow = static_cast<float*>(crow_v);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float4 v = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), g), __fmul_rn(__uint_as_float(r[4 * q + 1]), g),
+                             __fmul_rn(__uint_as_float(r[4 * q + 2]), g), __fmul_rn(__uint_as_float(r[4 * q + 3]), g));
+      if (p.accumulate) {
+        const float4 o = reinterpret_cast<const float4*>(crow)[q];
+        v.x = __fadd_rn(v.x, o.x);
+        v.y = __fadd_rn(v.y, o.y);
+        v.z = __fadd_rn(v.z, o.z);
+        v.w = __fadd_rn(v.w, o.w);
+      }
+      reinterpret_cast<float4*>(crow)[q] = v;
+    }
+  } else {
+    uint16_t* crow = static_cast<uint16_t*>(crow_v);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t w[4];
+      uint4 old = make_uint4(0u, 0u, 0u, 0u);
+      if (p.accumulate) old = reinterpret_cast<const uint4*>(crow)[q];
+      const uint32_t oldw[4] = {old.x, old.y, old.z, old.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v0 = __fmul_rn(__uint_as_float(r[8 * q + 2 * e]), g);
+        float v1 = __fmul_rn(__uint_as_float(r[8 * q + 2 * e + 1]), g);
+        if (p.accumulate) {
+          v0 = __fadd_rn(v0, bf16_lo(oldw[e]));
+          v1 = __fadd_rn(v1, bf16_hi(oldw[e]));
+        }
+        w[e] = f32_to_bf16_bits(v0) | (f32_to_bf16_bits(v1) << 16);
+      }
+      reinterpret_cast<uint4*>(crow)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
 }
 
 // Wait with a time limit only (teardown after an abort).
@@ -304,64 +348,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;                  // tensor-memory lanes 32*quarter ..
+    // Warp w reads tensor-memory lanes 32*(w%4).. (its hardware lane quarter)
+    // and one half of the 256 accumulator columns.  It copies its whole share to
+    // registers, hands the accumulator back to the MMA warp at once, and then
+    // scales, converts and stores while the next tile's main loop runs.
+    const int ew = warp - EPI_WARP0;               // 0..7
+    const int quarter = warp & 3;
+    const int half = ew >> 2;                      // accumulator columns 128*half ..
     const int row_in_tile = quarter * 32 + lane;
     const float g = __fmul_rn(__fmul_rn(*p.scale_a, *p.scale_b), p.alpha);
     uint32_t acc_phase = 0;
     for (int32_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       const TileCoord tc = tile_coord(p, t);
       const int n_cols = min(BN, p.N - tc.n_blk * BN);
+      const bool mine = n_cols > half * 128;
       // every lane polls; the warp proceeds (converged) only if all saw the phase complete
       const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, acc_phase, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const int64_t m = (int64_t)tc.m_blk * BM + row_in_tile;
-      for (int chunk = 0; chunk < n_cols / 32; ++chunk) {
-        uint32_t r[32];
-        tc_load_32cols(tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + chunk * 32, r);
-        const int64_t n0 = (int64_t)tc.n_blk * BN + chunk * 32;
-        if (p.out_f32) {
-          float* crow = static_cast<float*>(p.C) + m * p.ldc + n0;
+      uint32_t r[128];
+      if (mine) {
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + half * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 v = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), g), __fmul_rn(__uint_as_float(r[4 * q + 1]), g),
-                                   __fmul_rn(__uint_as_float(r[4 * q + 2]), g),
-                                   __fmul_rn(__uint_as_float(r[4 * q + 3]), g));
-            if (p.accumulate) {
-              const float4 o = reinterpret_cast<const float4*>(crow)[q];
-              v.x = __fadd_rn(v.x, o.x);
-              v.y = __fadd_rn(v.y, o.y);
-              v.z = __fadd_rn(v.z, o.z);
-              v.w = __fadd_rn(v.w, o.w);
-            }
-            reinterpret_cast<float4*>(crow)[q] = v;
-          }
-        } else {
-          uint16_t* crow = static_cast<uint16_t*>(p.C) + m * p.ldc + n0;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w[4];
-            uint4 old = make_uint4(0u, 0u, 0u, 0u);
-            if (p.accumulate) old = reinterpret_cast<const uint4*>(crow)[q];
-            const uint32_t oldw[4] = {old.x, old.y, old.z, old.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float v0 = __fmul_rn(__uint_as_float(r[8 * q + 2 * e]), g);
-              float v1 = __fmul_rn(__uint_as_float(r[8 * q + 2 * e + 1]), g);
-              if (p.accumulate) {
-                v0 = __fadd_rn(v0, bf16_lo(oldw[e]));
-                v1 = __fadd_rn(v1, bf16_hi(oldw[e]));
-              }
-              w[e] = f32_to_bf16_bits(v0) | (f32_to_bf16_bits(v1) << 16);
-            }
-            reinterpret_cast<uint4*>(crow)[q] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
+        for (int k = 0; k < 4; ++k) tc_load_32cols(taddr + 32 * k, r + 32 * k);
+        tc_wait_loads();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
       acc_phase ^= 1u;
+      if (mine) {
+        const int64_t m = (int64_t)tc.m_blk * BM + row_in_tile;
+        const int64_t n0 = (int64_t)tc.n_blk * BN + half * 128;
+        const size_t esz = p.out_f32 ? 4 : 2;
+        uint8_t* crow = static_cast<uint8_t*>(p.C) + (size_t)(m * p.ldc + n0) * esz;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) store_32cols(p, r + 32 * k, g, crow + (size_t)32 * k * esz);
+      }
     }
   }
 
@@ -374,5 +397,271 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+
+// =====================================================================================
+// CTA-pair variant (cta_group::2): one 256 x 256 output tile per pair of SMs.
+//
+// CTA r of the pair (r = 0 leads) loads A rows 128r.. of the tile, B rows 128r..
+// (its half of N), the block scales of its A rows and the scales of all 256 B
+// rows; the leader alone issues tcgen05.cp / tcgen05.mma with cta_group::2
+// (M = 256, N = 256, K = 64), which read each CTA's shared memory at the same
+// offsets and accumulate rows 128r.. of the tile in CTA r's tensor memory.  Each
+// CTA streams 38 KB per K-stage (the single-CTA kernel streams 54 KB for half the
+// work), so a 5-stage ring covers more memory latency.  All loads are TMA tile
+// loads without multicast; the pair's loads complete on the leader's stage
+// barrier, the leader's commits arrive on both CTAs' barriers.
+// =====================================================================================
+
+constexpr int P_STAGES = 5;
+constexpr int P_A_BYTES = 128 * BK_BYTES;                           // 16 KiB, own A rows
+constexpr int P_B_BYTES = 128 * BK_BYTES;                           // 16 KiB, own half of B
+constexpr int P_SFA_BYTES = (BK / MMA_K) * SF_ATOM;                 // 2 KiB
+constexpr int P_SFB_BYTES = 2 * (BK / MMA_K) * SF_ATOM;             // 4 KiB, all 256 B rows
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES + P_SFA_BYTES + P_SFB_BYTES;   // 38 KiB
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + BAR_BYTES + 1024;
+constexpr int P_BM = 256;                                           // tile rows per pair
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
+  return out;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA tile load whose completion is signalled on `bar`, which may be the peer CTA's barrier.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                                 uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_copy_scales_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor of the pair MMA: M = 256, N = 256.
+__host__ __device__ constexpr uint32_t make_idesc_pair() {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
+__device__ __forceinline__ TileCoord pair_tile_coord(const Params& p, int32_t t) {
+  // p.num_m counts 256-row tiles here
+  return tile_coord(p, t);
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_kernel_pair(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                     const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
+                     const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  uint8_t* bar_area = smem + P_STAGES * P_STAGE_BYTES;
+  const uint32_t bar_base = smem_u32(bar_area);
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (P_STAGES + s); };
+  const uint32_t acc_full = bar_base + 8u * (2 * P_STAGES);
+  const uint32_t acc_empty = bar_base + 8u * (2 * P_STAGES + 1);
+  const uint32_t mma_done = bar_base + 8u * (2 * P_STAGES + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (2 * P_STAGES + 3));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * P_STAGES + 3) + 4);
+
+  auto a_smem = [&](int s) { return smem_base + (uint32_t)(s * P_STAGE_BYTES); };
+  auto b_smem = [&](int s) { return smem_base + (uint32_t)(s * P_STAGE_BYTES + P_A_BYTES); };
+  auto sfa_smem = [&](int s) { return smem_base + (uint32_t)(s * P_STAGE_BYTES + P_A_BYTES + P_B_BYTES); };
+  auto sfb_smem = [&](int s) {
+    return smem_base + (uint32_t)(s * P_STAGE_BYTES + P_A_BYTES + P_B_BYTES + P_SFA_BYTES);
+  };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();           // 0 = leader
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * NUM_EPI_WARPS);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync();                                     // barriers of both CTAs initialised
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int32_t num_tiles = p.num_m * p.num_n;
+  const int32_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  const uint32_t leader_full0 = map_to_cta(full_bar(0), 0);
+  const uint32_t leader_acc_empty = map_to_cta(acc_empty, 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
+        const TileCoord tc = pair_tile_coord(p, t);
+        for (int ks = 0; ks < p.num_k_stages; ++ks) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = leader_full0 + 8u * stage;
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * P_STAGE_BYTES);
+          const int32_t kx = ks * BK_BYTES;
+          tma_load_2d_pair(a_smem(stage), &tma_a, kx, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
+          tma_load_2d_pair(b_smem(stage), &tma_b, kx, tc.n_blk * BN + (int32_t)rank * 128, fb);
+          const int32_t katom = ks * (BK / MMA_K);
+          tma_load_2d_pair(sfa_smem(stage), &tma_sfa, 0,
+                           (int32_t)((tc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + katom, fb);
+          tma_load_2d_pair(sfb_smem(stage), &tma_sfb, 0, (int32_t)((tc.n_blk * 2) * p.sf_kgroups) + katom, fb);
+          tma_load_2d_pair(sfb_smem(stage) + (BK / MMA_K) * SF_ATOM, &tma_sfb, 0,
+                           (int32_t)((tc.n_blk * 2 + 1) * p.sf_kgroups) + katom, fb);
+          if (++stage == P_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      const uint32_t idesc = make_idesc_pair();
+      for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
+        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int ks = 0; ks < p.num_k_stages; ++ks) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
+          for (int kk = 0; kk < atoms; ++kk) {
+            tc_copy_scales_pair(tmem + SFA_COL + 4 * kk, sf_desc(sfa_smem(stage) + kk * SF_ATOM));
+            tc_copy_scales_pair(tmem + SFB_COL + 8 * kk, sf_desc(sfb_smem(stage) + kk * SF_ATOM));
+            tc_copy_scales_pair(tmem + SFB_COL + 8 * kk + 4,
+                                sf_desc(sfb_smem(stage) + ((BK / MMA_K) + kk) * SF_ATOM));
+            tc_mma_pair(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * (MMA_K / 2)),
+                        sw128_desc(b_smem(stage) + kk * (MMA_K / 2)), idesc, (ks | kk) != 0 ? 1u : 0u,
+                        tmem + SFA_COL + 4 * kk, tmem + SFB_COL + 8 * kk);
+          }
+          tc_commit_pair(empty_bar(stage));
+          if (++stage == P_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(acc_full);
+        acc_phase ^= 1u;
+      }
+      // every MMA this thread issued has finished once mma_done flips
+      asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mma_done)
+                   : "memory");
+      mbar_wait_drain(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int ew = warp - EPI_WARP0;
+    const int quarter = warp & 3;
+    const int half = ew >> 2;
+    const int row_in_tile = (int)rank * 128 + quarter * 32 + lane;
+    const float g = __fmul_rn(__fmul_rn(*p.scale_a, *p.scale_b), p.alpha);
+    uint32_t acc_phase = 0;
+    for (int32_t t = pair; t < num_tiles; t += num_pairs) {
+      const TileCoord tc = pair_tile_coord(p, t);
+      const int n_cols = min(BN, p.N - tc.n_blk * BN);
+      const int64_t m = (int64_t)tc.m_blk * P_BM + row_in_tile;
+      const bool mine = n_cols > half * 128;
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, acc_phase, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t r[128];
+      if (mine) {
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + half * 128;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) tc_load_32cols(taddr + 32 * k, r + 32 * k);
+        tc_wait_loads();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_acc_empty);
+      acc_phase ^= 1u;
+      if (mine && m < p.M) {
+        const int64_t n0 = (int64_t)tc.n_blk * BN + half * 128;
+        const size_t esz = p.out_f32 ? 4 : 2;
+        uint8_t* crow = static_cast<uint8_t*>(p.C) + (size_t)(m * p.ldc + n0) * esz;
+        const int chunks = min(4, (n_cols - half * 128) / 32);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (k < chunks) store_32cols(p, r + 32 * k, g, crow + (size_t)32 * k * esz);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                     // the leader's MMAs are done with both CTAs
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
 }  // namespace gemm
 }  // namespace nvfp4

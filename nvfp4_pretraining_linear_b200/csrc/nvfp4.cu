@@ -45,6 +45,7 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 struct DeviceInfo {
   int sm_count = 0;
   bool gemm_attr = false;
+  int pair_clusters = 0;    // co-resident CTA pairs of the pair GEMM kernel
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -64,6 +65,24 @@ nvfp4_status device_info(DeviceInfo** out) {
     e = cudaFuncSetAttribute(nvfp4::gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              nvfp4::gemm::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
+    e = cudaFuncSetAttribute(nvfp4::gemm::gemm_kernel_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             nvfp4::gemm::P_SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (d.sm_count / 2), 1, 1);
+    cfg.blockDim = dim3(nvfp4::gemm::NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = nvfp4::gemm::P_SMEM_BYTES;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, nvfp4::gemm::gemm_kernel_pair, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+    d.pair_clusters = clusters;
     d.gemm_attr = true;
   }
   *out = &d;
@@ -100,6 +119,24 @@ nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t, uint32_t box
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return NVFP4_OK;
+}
+
+// Tensor map over the tensor-core scale layout viewed as rows of 512-byte
+// atoms (128 x 32-bit words): box of 4 atoms = one 128-row block x 256 K.
+nvfp4_status make_scale_map(CUtensorMap* map, const nvfp4_tensor* t) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  nvfp4_status st = get_encoder(&encode);
+  if (st != NVFP4_OK) return st;
+  const int64_t atoms = ceil_div(t->rows, 128) * ceil_div(t->cols / 16, 4);
+  const cuuint64_t dims[2] = {128u, (cuuint64_t)atoms};
+  const cuuint64_t strides[1] = {512u};
+  const cuuint32_t box[2] = {128u, 4u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, t->scales, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled(scales) failed (%d)", (int)r);
   return NVFP4_OK;
 }
 
@@ -394,22 +431,18 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, i
   }
   DeviceInfo* dev;
   if ((st = device_info(&dev)) != NVFP4_OK) return st;
-  CUtensorMap map_a, map_b;
-  if ((st = make_code_map(&map_a, A, nvfp4::gemm::BM)) != NVFP4_OK) return st;
-  if ((st = make_code_map(&map_b, B, nvfp4::gemm::BN)) != NVFP4_OK) return st;
   nvfp4::gemm::Params p{};
   p.M = (int32_t)M;
   p.N = (int32_t)N;
   p.K = (int32_t)K;
-  p.num_m = (int32_t)(M / nvfp4::gemm::BM);
   p.num_n = (int32_t)ceil_div(N, nvfp4::gemm::BN);
   p.num_k_stages = (int32_t)ceil_div(K, nvfp4::gemm::BK);
   const int64_t tail = K % nvfp4::gemm::BK;
   p.tail_atoms = tail ? (int32_t)(tail / nvfp4::gemm::MMA_K) : nvfp4::gemm::BK / nvfp4::gemm::MMA_K;
-  p.group_m = 16;
   p.sfa = A->scales;
   p.sfb = B->scales;
   p.sf_kgroups = K / 64;
+  p.sf_kgroups_a = K / 64;
   p.scale_a = A->tensor_scale;
   p.scale_b = B->tensor_scale;
   p.alpha = alpha;
@@ -417,10 +450,42 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, i
   p.ldc = ldc;
   p.out_f32 = out_dtype == NVFP4_OUT_F32;
   p.accumulate = accumulate != 0;
-  const int64_t tiles = (int64_t)p.num_m * p.num_n;
-  const int grid = (int)std::min<int64_t>(tiles, dev->sm_count);
-  nvfp4::gemm::gemm_kernel<<<grid, nvfp4::gemm::NUM_THREADS, nvfp4::gemm::SMEM_BYTES, s>>>(map_a, map_b, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (M >= 256 && dev->pair_clusters > 0) {
+    // CTA pairs, 256 x 256 tiles
+    CUtensorMap map_a, map_b, map_sfa, map_sfb;
+    if ((st = make_code_map(&map_a, A, 128)) != NVFP4_OK) return st;
+    if ((st = make_code_map(&map_b, B, 128)) != NVFP4_OK) return st;
+    if ((st = make_scale_map(&map_sfa, A)) != NVFP4_OK) return st;
+    if ((st = make_scale_map(&map_sfb, B)) != NVFP4_OK) return st;
+    p.num_m = (int32_t)ceil_div(M, nvfp4::gemm::P_BM);
+    p.group_m = 8;
+    const int64_t tiles = (int64_t)p.num_m * p.num_n;
+    const int pairs = (int)std::min<int64_t>(tiles, dev->pair_clusters);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(nvfp4::gemm::NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = nvfp4::gemm::P_SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, nvfp4::gemm::gemm_kernel_pair, map_a, map_b, map_sfa, map_sfb, p);
+  } else {
+    CUtensorMap map_a, map_b;
+    if ((st = make_code_map(&map_a, A, nvfp4::gemm::BM)) != NVFP4_OK) return st;
+    if ((st = make_code_map(&map_b, B, nvfp4::gemm::BN)) != NVFP4_OK) return st;
+    p.num_m = (int32_t)(M / nvfp4::gemm::BM);
+    p.group_m = 16;
+    const int64_t tiles = (int64_t)p.num_m * p.num_n;
+    const int grid = (int)std::min<int64_t>(tiles, dev->sm_count);
+    nvfp4::gemm::gemm_kernel<<<grid, nvfp4::gemm::NUM_THREADS, nvfp4::gemm::SMEM_BYTES, s>>>(map_a, map_b, p);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return NVFP4_OK;
 }
