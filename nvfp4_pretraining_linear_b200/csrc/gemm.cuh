@@ -420,6 +420,8 @@ constexpr int P_SFB_BYTES = 2 * (BK / MMA_K) * SF_ATOM;             // 4 KiB, al
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES + P_SFA_BYTES + P_SFB_BYTES;   // 38 KiB
 constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + BAR_BYTES + 1024;
 constexpr int P_BM = 256;                                           // tile rows per pair
+constexpr int P_ISSUER2 = EPI_WARP0 + NUM_EPI_WARPS;                // warp 10: second MMA issuer
+constexpr int P_NUM_THREADS = 32 * (P_ISSUER2 + 1);                 // 352
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -484,7 +486,7 @@ __device__ __forceinline__ TileCoord pair_tile_coord(const Params& p, int32_t t)
   return tile_coord(p, t);
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(P_NUM_THREADS, 1)
     gemm_kernel_pair(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                      const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
                      const Params p) {
@@ -498,8 +500,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t acc_full = bar_base + 8u * (2 * P_STAGES);
   const uint32_t acc_empty = bar_base + 8u * (2 * P_STAGES + 1);
   const uint32_t mma_done = bar_base + 8u * (2 * P_STAGES + 2);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (2 * P_STAGES + 3));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * P_STAGES + 3) + 4);
+  const uint32_t mma_done2 = bar_base + 8u * (2 * P_STAGES + 3);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (2 * P_STAGES + 4));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * P_STAGES + 4) + 4);
 
   auto a_smem = [&](int s) { return smem_base + (uint32_t)(s * P_STAGE_BYTES); };
   auto b_smem = [&](int s) { return smem_base + (uint32_t)(s * P_STAGE_BYTES + P_A_BYTES); };
@@ -520,6 +523,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * NUM_EPI_WARPS);
     mbar_init(mma_done, 1);
+    mbar_init(mma_done2, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -571,49 +575,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader only)
-    if (leader && lane == 0) {
+  } else if (warp == 1 || warp == P_ISSUER2) {
+    // ------------------------------------------------------------ MMA issuers (leader only)
+    // Two warps take the K-stages in turn (stage sequence q over all tiles of this
+    // pair: warp 1 issues even q, warp 10 odd q).  An issuer waits for its stage's
+    // data while the other warp's MMAs keep the tensor pipe busy -- a thread that
+    // polls an mbarrier stalls its own MMA issue, so one issuer alone cannot keep
+    // the pipe full.  Named barriers hand the turn over (1: warp 1 -> warp 10,
+    // 2: warp 10 -> warp 1), which keeps the MMAs in stage order; the tensor fences
+    // around them order the tensor-memory accesses across the two issuers.  After
+    // a failed wait an issuer keeps taking part in the hand-over (so the other
+    // issuer is never left waiting at a named barrier) but issues nothing.
+    if (leader) {
+      const int me = warp == 1 ? 0 : 1;
+      const uint32_t idesc = make_idesc_pair();
+      bool ok = true;
+      int64_t q = 0;                                    // stage sequence number
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
-      const uint32_t idesc = make_idesc_pair();
-      for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
-        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        for (int ks = 0; ks < p.num_k_stages; ++ks) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag)) {
-            ok = false;
-            break;
+      const int64_t my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
+      const int64_t total = my_tiles * p.num_k_stages;
+      for (int32_t t = pair; t < num_tiles; t += num_pairs) {
+        for (int ks = 0; ks < p.num_k_stages; ++ks, ++q) {
+          if ((q & 1) == me) {
+            if (ok && ks == 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag));
+            if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(full_bar(stage), phase, abort_flag));
+            if (q > 0) asm volatile("bar.sync %0, 64;" ::"r"(me == 0 ? 2 : 1) : "memory");
+            tc_fence_after();
+            if (ok && lane == 0) {
+              const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
+              for (int kk = 0; kk < atoms; ++kk) {
+                tc_copy_scales_pair(tmem + SFA_COL + 4 * kk, sf_desc(sfa_smem(stage) + kk * SF_ATOM));
+                tc_copy_scales_pair(tmem + SFB_COL + 8 * kk, sf_desc(sfb_smem(stage) + kk * SF_ATOM));
+                tc_copy_scales_pair(tmem + SFB_COL + 8 * kk + 4,
+                                    sf_desc(sfb_smem(stage) + ((BK / MMA_K) + kk) * SF_ATOM));
+                tc_mma_pair(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * (MMA_K / 2)),
+                            sw128_desc(b_smem(stage) + kk * (MMA_K / 2)), idesc, (ks | kk) != 0 ? 1u : 0u,
+                            tmem + SFA_COL + 4 * kk, tmem + SFB_COL + 8 * kk);
+              }
+              tc_commit_pair(empty_bar(stage));
+              if (ks == p.num_k_stages - 1) tc_commit_pair(acc_full);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (q + 1 < total) asm volatile("bar.arrive %0, 64;" ::"r"(me == 0 ? 1 : 2) : "memory");
           }
-          tc_fence_after();
-          const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
-          for (int kk = 0; kk < atoms; ++kk) {
-            tc_copy_scales_pair(tmem + SFA_COL + 4 * kk, sf_desc(sfa_smem(stage) + kk * SF_ATOM));
-            tc_copy_scales_pair(tmem + SFB_COL + 8 * kk, sf_desc(sfb_smem(stage) + kk * SF_ATOM));
-            tc_copy_scales_pair(tmem + SFB_COL + 8 * kk + 4,
-                                sf_desc(sfb_smem(stage) + ((BK / MMA_K) + kk) * SF_ATOM));
-            tc_mma_pair(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * (MMA_K / 2)),
-                        sw128_desc(b_smem(stage) + kk * (MMA_K / 2)), idesc, (ks | kk) != 0 ? 1u : 0u,
-                        tmem + SFA_COL + 4 * kk, tmem + SFB_COL + 8 * kk);
-          }
-          tc_commit_pair(empty_bar(stage));
           if (++stage == P_STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (!ok) break;
-        tc_commit_pair(acc_full);
         acc_phase ^= 1u;
       }
-      // every MMA this thread issued has finished once mma_done flips
-      asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mma_done)
-                   : "memory");
-      mbar_wait_drain(mma_done, 0);
+      // every MMA this warp issued has finished once mma_done flips (one barrier per issuer)
+      if (lane == 0) {
+        const uint32_t done = me == 0 ? mma_done : mma_done2;
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(done)
+                     : "memory");
+        mbar_wait_drain(done, 0);
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)

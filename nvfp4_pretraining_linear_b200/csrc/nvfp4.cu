@@ -75,7 +75,7 @@ nvfp4_status device_info(DeviceInfo** out) {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * (d.sm_count / 2), 1, 1);
-    cfg.blockDim = dim3(nvfp4::gemm::NUM_THREADS, 1, 1);
+    cfg.blockDim = dim3(nvfp4::gemm::P_NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = nvfp4::gemm::P_SMEM_BYTES;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -469,7 +469,7 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, i
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(nvfp4::gemm::NUM_THREADS, 1, 1);
+    cfg.blockDim = dim3(nvfp4::gemm::P_NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = nvfp4::gemm::P_SMEM_BYTES;
     cfg.stream = s;
     cfg.attrs = attr;
