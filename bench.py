@@ -464,6 +464,7 @@ def run_kernel(args):
         fn()
     torch.cuda.synchronize()
     times = []
+    clocks = ClockSampler(0)
     for _ in range(args.steps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -472,11 +473,13 @@ def run_kernel(args):
         b.record()
         b.synchronize()
         times.append(a.elapsed_time(b))
+    clock_info = clocks.stop()
     api.get_status()
     ms = statistics.median(times)
     rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
     print(json.dumps({"kernel": args.kernel, "shape": dims, "mode": args.mode if args.kernel == "quantize" else None,
-                      "ms": ms, "value": rate, "unit": unit, "steps": args.steps, "l2": "flushed (256 MB write)"}),
+                      "ms": ms, "value": rate, "unit": unit, "steps": args.steps, "l2": "flushed (256 MB write)",
+                      "clocks": clock_info}),
           flush=True)
     return 0
 

@@ -403,25 +403,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 //
 // CTA r of the pair (r = 0 leads) loads A rows 128r.. of the tile, B rows 128r..
 // (its half of N), the block scales of its A rows and the scales of all 256 B
-// rows; the leader alone issues tcgen05.cp / tcgen05.mma with cta_group::2
-// (M = 256, N = 256, K = 64), which read each CTA's shared memory at the same
-// offsets and accumulate rows 128r.. of the tile in CTA r's tensor memory.  Each
-// CTA streams 38 KB per K-stage (the single-CTA kernel streams 54 KB for half the
-// work), so a 5-stage ring covers more memory latency.  All loads are TMA tile
-// loads without multicast; the pair's loads complete on the leader's stage
-// barrier, the leader's commits arrive on both CTAs' barriers.
+// rows; the leader alone issues tcgen05.mma with cta_group::2 (M = 256, N = 256,
+// K = 64), which reads each CTA's shared memory at the same offsets and
+// accumulates rows 128r.. of the tile in CTA r's tensor memory.  Each CTA streams
+// 38 KB per K-stage (the single-CTA kernel streams 54 KB for half the work), so a
+// 5-stage ring covers more memory latency.  All loads are TMA tile loads without
+// multicast; the pair's operand loads complete on the leader's stage barrier, each
+// CTA's scale loads on its own; the leader's commits arrive on both CTAs' barriers.
+//
+// Block scales reach tensor memory through tcgen05.st from four scale-writer warps
+// per CTA (one per 32-lane quarter), not through tcgen05.cp from the MMA thread:
+// copies issued between the MMAs stretch each M256N256K64 MMA from 128 to about
+// 275 cycles on random operands, while stores from other warps leave the MMA
+// stream at 128.  Each operand stage has its own scale slot in tensor memory (48
+// columns: 16 of A scales, 32 of B scales), freed with the stage.  The layout
+// written is the one a 32x128b.warpx4 copy of the 512-byte scale tile gives:
+// every quarter holds the same 32 lanes x 4 columns per tile.  The scales stream
+// through a shared-memory ring of their own, deeper than the operand ring and fed
+// by a second producer warp, so that a stage's scales are in shared memory before
+// its tensor-memory slot frees.  The writers' hand-over to the MMA issuers is a
+// relaxed cluster-scope arrival: ordering tensor-memory accesses takes only the
+// tcgen05 fences around it, and a release arrival costs over a thousand cycles.
 // =====================================================================================
 
-constexpr int P_STAGES = 5;
+constexpr int P_STAGES = 5;                                         // operand ring
+constexpr int P_SF_STAGES = 8;                                      // scale ring
 constexpr int P_A_BYTES = 128 * BK_BYTES;                           // 16 KiB, own A rows
 constexpr int P_B_BYTES = 128 * BK_BYTES;                           // 16 KiB, own half of B
 constexpr int P_SFA_BYTES = (BK / MMA_K) * SF_ATOM;                 // 2 KiB
 constexpr int P_SFB_BYTES = 2 * (BK / MMA_K) * SF_ATOM;             // 4 KiB, all 256 B rows
-constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES + P_SFA_BYTES + P_SFB_BYTES;   // 38 KiB
-constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + BAR_BYTES + 1024;
+constexpr int P_AB_BYTES = P_A_BYTES + P_B_BYTES;                   // operand bytes per CTA and stage
+constexpr int P_SF_BYTES = P_SFA_BYTES + P_SFB_BYTES;               // scale bytes per CTA and stage
+constexpr int P_SF_OFFSET = P_STAGES * P_AB_BYTES;                  // scale ring after the operands
+constexpr int P_BAR_OFFSET = P_SF_OFFSET + P_SF_STAGES * P_SF_BYTES;
+constexpr int P_NUM_BARS = 3 * P_STAGES + 2 * P_SF_STAGES + 4;
+constexpr int P_BAR_BYTES = 512;
+constexpr int P_SMEM_BYTES = P_BAR_OFFSET + P_BAR_BYTES + 1024;
 constexpr int P_BM = 256;                                           // tile rows per pair
 constexpr int P_ISSUER2 = EPI_WARP0 + NUM_EPI_WARPS;                // warp 10: second MMA issuer
-constexpr int P_NUM_THREADS = 32 * (P_ISSUER2 + 1);                 // 352
+constexpr int P_WRITER0 = P_ISSUER2 + 1;                            // warps 11..14: scale writers
+constexpr int P_NUM_WRITERS = 4;
+constexpr int P_SF_PRODUCER = P_WRITER0 + P_NUM_WRITERS;            // warp 15: scale loads
+constexpr int P_NUM_THREADS = 32 * (P_SF_PRODUCER + 1);             // 512
+constexpr int P_SF_COL0 = 256;                                      // scale slot s at 256 + 48 s
+constexpr int P_SF_SLOT_COLS = 48;                                  // 16 A-scale + 32 B-scale columns
+static_assert(P_SF_COL0 + P_STAGES * P_SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed tensor memory");
+static_assert(8 * P_NUM_BARS + 8 <= P_BAR_BYTES, "barrier area too small");
+static_assert(P_SMEM_BYTES <= 232448, "shared memory above the sm_100 limit");
+static_assert(P_SF_BYTES % 128 == 0 && P_AB_BYTES % 1024 == 0, "ring alignment");
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -444,6 +473,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Arrival that only hands over tensor-memory accesses: the arriving warp has waited
+// for its tcgen05.ld / tcgen05.st (wait::ld / wait::st) and issued
+// tcgen05.fence::before_thread_sync; the waiter issues tcgen05.fence::after_thread_sync
+// before its next tcgen05 operation.  No generic-memory release is needed, and the
+// cluster-scope release costs over a thousand cycles per arrival.
+__device__ __forceinline__ void mbar_arrive_cluster_tc(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // TMA tile load whose completion is signalled on `bar`, which may be the peer CTA's barrier.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
                                                  uint32_t bar) {
@@ -459,10 +497,6 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
       "h"((uint16_t)3)
       : "memory");
-}
-
-__device__ __forceinline__ void tc_copy_scales_pair(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -493,23 +527,26 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t smem_base = smem_u32(smem);
-  uint8_t* bar_area = smem + P_STAGES * P_STAGE_BYTES;
+  uint8_t* bar_area = smem + P_BAR_OFFSET;
   const uint32_t bar_base = smem_u32(bar_area);
+  // operand ring: full (leader; both CTAs' loads complete on it), empty (MMA commits, both CTAs)
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (P_STAGES + s); };
-  const uint32_t acc_full = bar_base + 8u * (2 * P_STAGES);
-  const uint32_t acc_empty = bar_base + 8u * (2 * P_STAGES + 1);
-  const uint32_t mma_done = bar_base + 8u * (2 * P_STAGES + 2);
-  const uint32_t mma_done2 = bar_base + 8u * (2 * P_STAGES + 3);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (2 * P_STAGES + 4));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * P_STAGES + 4) + 4);
+  auto sf_ready_bar = [&](int s) { return bar_base + 8u * (2 * P_STAGES + s); };   // scales in TMEM (leader)
+  // scale ring (each CTA its own): landed in shared memory / written to TMEM by the four writers
+  auto sf_full_bar = [&](int j) { return bar_base + 8u * (3 * P_STAGES + j); };
+  auto sf_empty_bar = [&](int j) { return bar_base + 8u * (3 * P_STAGES + P_SF_STAGES + j); };
+  const uint32_t acc_full = bar_base + 8u * (P_NUM_BARS - 4);
+  const uint32_t acc_empty = bar_base + 8u * (P_NUM_BARS - 3);
+  const uint32_t mma_done = bar_base + 8u * (P_NUM_BARS - 2);
+  const uint32_t mma_done2 = bar_base + 8u * (P_NUM_BARS - 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * P_NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * P_NUM_BARS + 4);
 
-  auto a_smem = [&](int s) { return smem_base + (uint32_t)(s * P_STAGE_BYTES); };
-  auto b_smem = [&](int s) { return smem_base + (uint32_t)(s * P_STAGE_BYTES + P_A_BYTES); };
-  auto sfa_smem = [&](int s) { return smem_base + (uint32_t)(s * P_STAGE_BYTES + P_A_BYTES + P_B_BYTES); };
-  auto sfb_smem = [&](int s) {
-    return smem_base + (uint32_t)(s * P_STAGE_BYTES + P_A_BYTES + P_B_BYTES + P_SFA_BYTES);
-  };
+  auto a_smem = [&](int s) { return smem_base + (uint32_t)(s * P_AB_BYTES); };
+  auto b_smem = [&](int s) { return smem_base + (uint32_t)(s * P_AB_BYTES + P_A_BYTES); };
+  auto sfa_smem = [&](int j) { return smem_base + (uint32_t)(P_SF_OFFSET + j * P_SF_BYTES); };
+  auto sfb_smem = [&](int j) { return smem_base + (uint32_t)(P_SF_OFFSET + j * P_SF_BYTES + P_SFA_BYTES); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();           // 0 = leader
@@ -519,6 +556,11 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     for (int s = 0; s < P_STAGES; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
+      mbar_init(sf_ready_bar(s), 2 * P_NUM_WRITERS);
+    }
+    for (int j = 0; j < P_SF_STAGES; ++j) {
+      mbar_init(sf_full_bar(j), 1);
+      mbar_init(sf_empty_bar(j), P_NUM_WRITERS);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * NUM_EPI_WARPS);
@@ -545,7 +587,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
   const uint32_t leader_acc_empty = map_to_cta(acc_empty, 0);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (both CTAs)
+    // ------------------------------------------------------------ operand producer (both CTAs)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -558,16 +600,10 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             break;
           }
           const uint32_t fb = leader_full0 + 8u * stage;
-          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * P_STAGE_BYTES);
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * P_AB_BYTES);
           const int32_t kx = ks * BK_BYTES;
           tma_load_2d_pair(a_smem(stage), &tma_a, kx, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
           tma_load_2d_pair(b_smem(stage), &tma_b, kx, tc.n_blk * BN + (int32_t)rank * 128, fb);
-          const int32_t katom = ks * (BK / MMA_K);
-          tma_load_2d_pair(sfa_smem(stage), &tma_sfa, 0,
-                           (int32_t)((tc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + katom, fb);
-          tma_load_2d_pair(sfb_smem(stage), &tma_sfb, 0, (int32_t)((tc.n_blk * 2) * p.sf_kgroups) + katom, fb);
-          tma_load_2d_pair(sfb_smem(stage) + (BK / MMA_K) * SF_ATOM, &tma_sfb, 0,
-                           (int32_t)((tc.n_blk * 2 + 1) * p.sf_kgroups) + katom, fb);
           if (++stage == P_STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -600,19 +636,16 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           if ((q & 1) == me) {
             if (ok && ks == 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag));
             if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(full_bar(stage), phase, abort_flag));
+            if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(sf_ready_bar(stage), phase, abort_flag));
             if (q > 0) asm volatile("bar.sync %0, 64;" ::"r"(me == 0 ? 2 : 1) : "memory");
             tc_fence_after();
             if (ok && lane == 0) {
               const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
-              for (int kk = 0; kk < atoms; ++kk) {
-                tc_copy_scales_pair(tmem + SFA_COL + 4 * kk, sf_desc(sfa_smem(stage) + kk * SF_ATOM));
-                tc_copy_scales_pair(tmem + SFB_COL + 8 * kk, sf_desc(sfb_smem(stage) + kk * SF_ATOM));
-                tc_copy_scales_pair(tmem + SFB_COL + 8 * kk + 4,
-                                    sf_desc(sfb_smem(stage) + ((BK / MMA_K) + kk) * SF_ATOM));
+              const uint32_t sfa = tmem + P_SF_COL0 + P_SF_SLOT_COLS * stage, sfb = sfa + 16;
+              for (int kk = 0; kk < atoms; ++kk)
                 tc_mma_pair(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * (MMA_K / 2)),
                             sw128_desc(b_smem(stage) + kk * (MMA_K / 2)), idesc, (ks | kk) != 0 ? 1u : 0u,
-                            tmem + SFA_COL + 4 * kk, tmem + SFB_COL + 8 * kk);
-              }
+                            sfa + 4 * kk, sfb + 8 * kk);
               tc_commit_pair(empty_bar(stage));
               if (ks == p.num_k_stages - 1) tc_commit_pair(acc_full);
             }
@@ -635,6 +668,101 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
         mbar_wait_drain(done, 0);
       }
     }
+  } else if (warp == P_SF_PRODUCER) {
+    // ------------------------------------------------------------ scale producer (both CTAs)
+    // Each CTA loads the scales of its own A rows and of all 256 B rows of the tile,
+    // up to P_SF_STAGES stages ahead; a slot is reused once the four writers of this
+    // CTA have stored it to tensor memory.
+    if (lane == 0) {
+      int j = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
+        const TileCoord tc = pair_tile_coord(p, t);
+        for (int ks = 0; ks < p.num_k_stages; ++ks) {
+          if (!mbar_wait(sf_empty_bar(j), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sb = sf_full_bar(j);
+          mbar_arrive_expect_tx(sb, (uint32_t)P_SF_BYTES);
+          const int32_t katom = ks * (BK / MMA_K);
+          tma_load_2d(sfa_smem(j), &tma_sfa, 0, (int32_t)((tc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + katom,
+                      sb);
+          tma_load_2d(sfb_smem(j), &tma_sfb, 0, (int32_t)((tc.n_blk * 2) * p.sf_kgroups) + katom, sb);
+          tma_load_2d(sfb_smem(j) + (BK / MMA_K) * SF_ATOM, &tma_sfb, 0,
+                      (int32_t)((tc.n_blk * 2 + 1) * p.sf_kgroups) + katom, sb);
+          if (++j == P_SF_STAGES) {
+            j = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp >= P_WRITER0) {
+    // ------------------------------------------------------------ scale writers (both CTAs)
+    // Warp w writes lane quarter w % 4 of each stage's scale slot: lane i takes row i
+    // of every 512-byte scale tile of the stage (16 bytes = 4 columns per tile) and
+    // stores them with tcgen05.st; then it tells the leader's MMA issuers and frees
+    // the shared-memory slot (the stores have consumed the loaded registers, so the
+    // loads are complete).  The tensor-memory slot of operand stage s is free once the
+    // MMAs of its previous use have completed (the commit that frees the operand stage).
+    const int quarter = warp & 3;
+    const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t leader_ready0 = map_to_cta(sf_ready_bar(0), 0);
+    const uint32_t own_empty0 = map_to_cta(sf_empty_bar(0), rank);
+    int stage = 0, j = 0;
+    uint32_t phase = 0, sf_phase = 0;
+    bool ok = true;
+    for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
+      for (int ks = 0; ks < p.num_k_stages; ++ks) {
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(sf_full_bar(j), sf_phase, abort_flag));
+        if (!ok) break;
+        const uint8_t* sa = smem + P_SF_OFFSET + j * P_SF_BYTES + lane * 16;
+        uint32_t v[48];
+#pragma unroll
+        for (int kk = 0; kk < BK / MMA_K; ++kk) {
+          const uint4 xa = *reinterpret_cast<const uint4*>(sa + kk * SF_ATOM);
+          const uint4 x0 = *reinterpret_cast<const uint4*>(sa + P_SFA_BYTES + kk * SF_ATOM);
+          const uint4 x1 = *reinterpret_cast<const uint4*>(sa + P_SFA_BYTES + ((BK / MMA_K) + kk) * SF_ATOM);
+          v[4 * kk] = xa.x, v[4 * kk + 1] = xa.y, v[4 * kk + 2] = xa.z, v[4 * kk + 3] = xa.w;
+          v[16 + 8 * kk] = x0.x, v[17 + 8 * kk] = x0.y, v[18 + 8 * kk] = x0.z, v[19 + 8 * kk] = x0.w;
+          v[20 + 8 * kk] = x1.x, v[21 + 8 * kk] = x1.y, v[22 + 8 * kk] = x1.z, v[23 + 8 * kk] = x1.w;
+        }
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t slot = tq + P_SF_COL0 + P_SF_SLOT_COLS * stage;
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+                     "%15,%16};" ::"r"(slot),
+                     "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+                     "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+                     : "memory");
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+                     "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(slot + 16),
+                     "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]),
+                     "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]),
+                     "r"(v[30]), "r"(v[31]), "r"(v[32]), "r"(v[33]), "r"(v[34]), "r"(v[35]), "r"(v[36]),
+                     "r"(v[37]), "r"(v[38]), "r"(v[39]), "r"(v[40]), "r"(v[41]), "r"(v[42]), "r"(v[43]),
+                     "r"(v[44]), "r"(v[45]), "r"(v[46]), "r"(v[47])
+                     : "memory");
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster_tc(leader_ready0 + 8u * stage);
+          mbar_arrive_cluster_tc(own_empty0 + 8u * j);
+        }
+        if (++stage == P_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if (++j == P_SF_STAGES) {
+          j = 0;
+          sf_phase ^= 1u;
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int ew = warp - EPI_WARP0;
@@ -642,6 +770,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     const int half = ew >> 2;
     const int row_in_tile = (int)rank * 128 + quarter * 32 + lane;
     const float g = __fmul_rn(__fmul_rn(*p.scale_a, *p.scale_b), p.alpha);
+    const bool packed = !p.out_f32 && !p.accumulate;
     uint32_t acc_phase = 0;
     for (int32_t t = pair; t < num_tiles; t += num_pairs) {
       const TileCoord tc = pair_tile_coord(p, t);
@@ -651,26 +780,57 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, acc_phase, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t r[128];
-      if (mine) {
-        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + half * 128;
+      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + half * 128;
+      const int64_t n0 = (int64_t)tc.n_blk * BN + half * 128;
+      const int chunks = mine ? min(4, (n_cols - half * 128) / 32) : 0;
+      if (packed) {
+        // BF16 without accumulation: scale and round while reading, so the 128
+        // columns of this warp stay in 64 registers; release, then store.
+        uint32_t pk[64];
+        if (mine) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) tc_load_32cols(taddr + 32 * k, r + 32 * k);
-        tc_wait_loads();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_acc_empty);
-      acc_phase ^= 1u;
-      if (mine && m < p.M) {
-        const int64_t n0 = (int64_t)tc.n_blk * BN + half * 128;
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t r[64];
+            tc_load_32cols(taddr + 64 * hh, r);
+            tc_load_32cols(taddr + 64 * hh + 32, r + 32);
+            tc_wait_loads();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              pk[32 * hh + j] = f32_to_bf16_bits(__fmul_rn(__uint_as_float(r[2 * j]), g)) |
+                                (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r[2 * j + 1]), g)) << 16);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_tc(leader_acc_empty);
+        if (m < p.M) {
+          uint4* crow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.C) + (size_t)(m * p.ldc + n0));
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (k < chunks)
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                crow[4 * k + q] = make_uint4(pk[16 * k + 4 * q], pk[16 * k + 4 * q + 1], pk[16 * k + 4 * q + 2],
+                                             pk[16 * k + 4 * q + 3]);
+        }
+      } else {
+        // FP32 output or accumulation into C: 32 columns at a time, released at the end.
         const size_t esz = p.out_f32 ? 4 : 2;
         uint8_t* crow = static_cast<uint8_t*>(p.C) + (size_t)(m * p.ldc + n0) * esz;
-        const int chunks = min(4, (n_cols - half * 128) / 32);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (k < chunks) store_32cols(p, r + 32 * k, g, crow + (size_t)32 * k * esz);
+        if (mine) {
+#pragma unroll 1
+          for (int k = 0; k < 4; ++k) {
+            uint32_t r[32];
+            tc_load_32cols(taddr + 32 * k, r);
+            tc_wait_loads();
+            if (k < chunks && m < p.M) store_32cols(p, r, g, crow + (size_t)32 * k * esz);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_tc(leader_acc_empty);
       }
+      acc_phase ^= 1u;
     }
   }
 
