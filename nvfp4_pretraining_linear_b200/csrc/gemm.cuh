@@ -426,8 +426,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // tcgen05 fences around it, and a release arrival costs over a thousand cycles.
 // =====================================================================================
 
-constexpr int P_STAGES = 5;                                         // operand ring
-constexpr int P_SF_STAGES = 8;                                      // scale ring
+constexpr int P_STAGES = 6;                                         // operand ring
+constexpr int P_SF_STAGES = 4;                                      // scale ring (shared memory)
+constexpr int P_SF_SLOTS = 5;                                       // scale slots in tensor memory
 constexpr int P_A_BYTES = 128 * BK_BYTES;                           // 16 KiB, own A rows
 constexpr int P_B_BYTES = 128 * BK_BYTES;                           // 16 KiB, own half of B
 constexpr int P_SFA_BYTES = (BK / MMA_K) * SF_ATOM;                 // 2 KiB
@@ -447,7 +448,9 @@ constexpr int P_SF_PRODUCER = P_WRITER0 + P_NUM_WRITERS;            // warp 15: 
 constexpr int P_NUM_THREADS = 32 * (P_SF_PRODUCER + 1);             // 512
 constexpr int P_SF_COL0 = 256;                                      // scale slot s at 256 + 48 s
 constexpr int P_SF_SLOT_COLS = 48;                                  // 16 A-scale + 32 B-scale columns
-static_assert(P_SF_COL0 + P_STAGES * P_SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed tensor memory");
+constexpr int P_PREFETCH = 8;                                       // next-tile stages warmed in L2
+static_assert(P_SF_COL0 + P_SF_SLOTS * P_SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed tensor memory");
+static_assert(P_SF_SLOTS < P_STAGES, "a scale slot must free no later than the operand stage it serves");
 static_assert(8 * P_NUM_BARS + 8 <= P_BAR_BYTES, "barrier area too small");
 static_assert(P_SMEM_BYTES <= 232448, "shared memory above the sm_100 limit");
 static_assert(P_SF_BYTES % 128 == 0 && P_AB_BYTES % 1024 == 0, "ring alignment");
@@ -490,6 +493,21 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
           dst),
       "l"(map), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+// Warm L2 with a tile that a later TMA load will read (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
+}
+
+// Two FP32 values scaled by g, rounded to BF16 (nearest even) and packed, lo in the low half.
+__device__ __forceinline__ uint32_t scale_pack_bf16x2(uint32_t lo, uint32_t hi, float g) {
+  uint32_t out;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+      : "=r"(out)
+      : "f"(__fmul_rn(__uint_as_float(hi), g)), "f"(__fmul_rn(__uint_as_float(lo), g)));
+  return out;
 }
 
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
@@ -592,8 +610,14 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // During the last P_PREFETCH stages of a tile, the first stages of the pair's next
+      // tile are prefetched into L2: every pair starts its next tile at about the same
+      // time, and without this those first loads all miss L2 at once.
+      const int pf_n = min(P_PREFETCH, p.num_k_stages);
       for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
         const TileCoord tc = pair_tile_coord(p, t);
+        const bool has_next = t + num_pairs < num_tiles;
+        const TileCoord nc = pair_tile_coord(p, has_next ? t + num_pairs : t);
         for (int ks = 0; ks < p.num_k_stages; ++ks) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
             ok = false;
@@ -604,6 +628,11 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           const int32_t kx = ks * BK_BYTES;
           tma_load_2d_pair(a_smem(stage), &tma_a, kx, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
           tma_load_2d_pair(b_smem(stage), &tma_b, kx, tc.n_blk * BN + (int32_t)rank * 128, fb);
+          const int pf = ks - (p.num_k_stages - pf_n);
+          if (has_next && pf >= 0) {
+            tma_prefetch_2d(&tma_a, pf * BK_BYTES, nc.m_blk * P_BM + (int32_t)rank * 128);
+            tma_prefetch_2d(&tma_b, pf * BK_BYTES, nc.n_blk * BN + (int32_t)rank * 128);
+          }
           if (++stage == P_STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -627,7 +656,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       const uint32_t idesc = make_idesc_pair();
       bool ok = true;
       int64_t q = 0;                                    // stage sequence number
-      int stage = 0;
+      int stage = 0, slot = 0;                          // operand stage, scale slot (q % P_SF_SLOTS)
       uint32_t phase = 0, acc_phase = 0;
       const int64_t my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
       const int64_t total = my_tiles * p.num_k_stages;
@@ -641,7 +670,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             tc_fence_after();
             if (ok && lane == 0) {
               const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
-              const uint32_t sfa = tmem + P_SF_COL0 + P_SF_SLOT_COLS * stage, sfb = sfa + 16;
+              const uint32_t sfa = tmem + P_SF_COL0 + P_SF_SLOT_COLS * slot, sfb = sfa + 16;
               for (int kk = 0; kk < atoms; ++kk)
                 tc_mma_pair(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * (MMA_K / 2)),
                             sw128_desc(b_smem(stage) + kk * (MMA_K / 2)), idesc, (ks | kk) != 0 ? 1u : 0u,
@@ -657,6 +686,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             stage = 0;
             phase ^= 1u;
           }
+          if (++slot == P_SF_SLOTS) slot = 0;
         }
         acc_phase ^= 1u;
       }
@@ -677,9 +707,19 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       int j = 0;
       uint32_t phase = 0;
       bool ok = true;
+      const int pf_n = min(P_PREFETCH, p.num_k_stages);
       for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
         const TileCoord tc = pair_tile_coord(p, t);
+        const bool has_next = t + num_pairs < num_tiles;
+        const TileCoord nc = pair_tile_coord(p, has_next ? t + num_pairs : t);
         for (int ks = 0; ks < p.num_k_stages; ++ks) {
+          const int pf = ks - (p.num_k_stages - pf_n);
+          if (has_next && pf >= 0) {             // the next tile's scales, as for the operands
+            const int32_t pk = pf * (BK / MMA_K);
+            tma_prefetch_2d(&tma_sfa, 0, (int32_t)((nc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + pk);
+            tma_prefetch_2d(&tma_sfb, 0, (int32_t)((nc.n_blk * 2) * p.sf_kgroups) + pk);
+            tma_prefetch_2d(&tma_sfb, 0, (int32_t)((nc.n_blk * 2 + 1) * p.sf_kgroups) + pk);
+          }
           if (!mbar_wait(sf_empty_bar(j), phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -705,17 +745,22 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     // of every 512-byte scale tile of the stage (16 bytes = 4 columns per tile) and
     // stores them with tcgen05.st; then it tells the leader's MMA issuers and frees
     // the shared-memory slot (the stores have consumed the loaded registers, so the
-    // loads are complete).  The tensor-memory slot of operand stage s is free once the
-    // MMAs of its previous use have completed (the commit that frees the operand stage).
+    // loads are complete).  Stage q uses tensor-memory slot q % P_SF_SLOTS, free once
+    // the MMAs of stage q - P_SF_SLOTS have completed: the commit that frees operand
+    // stage (q - P_SF_SLOTS) % P_STAGES, phase (q - P_SF_SLOTS) / P_STAGES.  That
+    // barrier cannot be a phase behind (the MMAs of stage q - 1 - P_SF_SLOTS, older,
+    // are complete: this warp waited for them) nor a phase ahead (stage q + 1 needs
+    // this warp's scales), so its parity names the phase.
     const int quarter = warp & 3;
     const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t leader_ready0 = map_to_cta(sf_ready_bar(0), 0);
     const uint32_t own_empty0 = map_to_cta(sf_empty_bar(0), rank);
-    int stage = 0, j = 0;
-    uint32_t phase = 0, sf_phase = 0;
+    int stage = 0, j = 0, slot = 0, lag_stage = 0;
+    uint32_t sf_phase = 0, lag_phase = 0;
+    int64_t q = 0;
     bool ok = true;
     for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
-      for (int ks = 0; ks < p.num_k_stages; ++ks) {
+      for (int ks = 0; ks < p.num_k_stages; ++ks, ++q) {
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(sf_full_bar(j), sf_phase, abort_flag));
         if (!ok) break;
         const uint8_t* sa = smem + P_SF_OFFSET + j * P_SF_BYTES + lane * 16;
@@ -729,17 +774,23 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           v[16 + 8 * kk] = x0.x, v[17 + 8 * kk] = x0.y, v[18 + 8 * kk] = x0.z, v[19 + 8 * kk] = x0.w;
           v[20 + 8 * kk] = x1.x, v[21 + 8 * kk] = x1.y, v[22 + 8 * kk] = x1.z, v[23 + 8 * kk] = x1.w;
         }
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag));
-        if (!ok) break;
+        if (q >= P_SF_SLOTS) {
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(lag_stage), lag_phase, abort_flag));
+          if (!ok) break;
+          if (++lag_stage == P_STAGES) {
+            lag_stage = 0;
+            lag_phase ^= 1u;
+          }
+        }
         tc_fence_after();
-        const uint32_t slot = tq + P_SF_COL0 + P_SF_SLOT_COLS * stage;
+        const uint32_t taddr = tq + P_SF_COL0 + P_SF_SLOT_COLS * slot;
         asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-                     "%15,%16};" ::"r"(slot),
+                     "%15,%16};" ::"r"(taddr),
                      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
                      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
                      : "memory");
         asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-                     "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(slot + 16),
+                     "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr + 16),
                      "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]),
                      "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]),
                      "r"(v[30]), "r"(v[31]), "r"(v[32]), "r"(v[33]), "r"(v[34]), "r"(v[35]), "r"(v[36]),
@@ -753,10 +804,8 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           mbar_arrive_cluster_tc(leader_ready0 + 8u * stage);
           mbar_arrive_cluster_tc(own_empty0 + 8u * j);
         }
-        if (++stage == P_STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        if (++stage == P_STAGES) stage = 0;
+        if (++slot == P_SF_SLOTS) slot = 0;
         if (++j == P_SF_STAGES) {
           j = 0;
           sf_phase ^= 1u;
@@ -795,9 +844,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             tc_load_32cols(taddr + 64 * hh + 32, r + 32);
             tc_wait_loads();
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              pk[32 * hh + j] = f32_to_bf16_bits(__fmul_rn(__uint_as_float(r[2 * j]), g)) |
-                                (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r[2 * j + 1]), g)) << 16);
+            for (int j = 0; j < 32; ++j) pk[32 * hh + j] = scale_pack_bf16x2(r[2 * j], r[2 * j + 1], g);
           }
         }
         tc_fence_before();
