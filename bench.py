@@ -61,6 +61,33 @@ def dist_env():
     return rank, world, local
 
 
+# ----------------------------------------------------------------------------- traffic
+
+GEMM_SOURCE = os.path.join(ROOT, "nvfp4_pretraining_linear_b200", "csrc", "gemm.cuh")
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "gemm_pair_hybrid12b_step_traffic.txt")
+
+
+def gemm_traffic_per_launch():
+    """DRAM bytes (read + write) per GEMM launch of this step, from the committed ncu
+    summary; None when there is none or when the GEMM source changed since it was taken
+    (the summary records the SHA-256 of gemm.cuh it was measured with)."""
+    import hashlib
+    try:
+        fields = {}
+        with open(TRAFFIC_PROFILE) as f:
+            for line in f:
+                if ":" in line:
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip()
+        with open(GEMM_SOURCE, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        if fields.get("gemm_source_sha256") != sha:
+            return None
+        return int(fields["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 # ----------------------------------------------------------------------------- clocks
 
 
@@ -351,14 +378,7 @@ def run_ours(args):
     quant_gbs = qbytes / (quant_ms * 1e-3) / 1e9
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     gemm_launches = 3 * len(linears)
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "gemm_traffic.json")
-    if os.path.exists(prof):
-        try:
-            with open(prof) as f:
-                traffic = json.load(f).get("bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = gemm_traffic_per_launch()
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -411,7 +431,7 @@ def run_ours(args):
             "gemm": {"tflops": gemm_tflops, "frac_fp4_peak": gemm_tflops / fp4_peak, "ms_per_step": gemm_ms},
             "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": gemm_tflops / fp4_peak, "traffic": traffic,
-                         "kernel": "nvfp4::gemm::gemm_kernel",
+                         "kernel": "nvfp4::gemm::gemm_kernel_pair",
                          "peak_source": "%s bf16 sustained x %.0f (nominal FP4/BF16 ratio), of %s" % (
                              peak_src, FP4_OVER_BF16, peak_src)},
             "clocks": clock_info,
