@@ -91,13 +91,28 @@ __device__ __forceinline__ void rht16_pair(float* v, uint32_t signs, int lane) {
 
 // Butterfly stages h = 1, 2, 4, 8 and the 1/4 normalisation over 16 values whose
 // signs were already applied (the transform of rht16 after its sign flips).
+// Stage 1 pairs neighbours, so it runs on scalars; after it, elements 2p and 2p+1
+// share register pair p, and stages 2, 4, 8 combine pairs p and p + h/2 lane by
+// lane with packed FP32 instructions (same operations, same order per element).
 __device__ __forceinline__ void wht16_scaled(float* v) {
   wht_stage<16>(v, 1);
-  wht_stage<16>(v, 2);
-  wht_stage<16>(v, 4);
-  wht_stage<16>(v, 8);
+  uint64_t pr[8];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], 0.25f);
+  for (int p = 0; p < 8; ++p) pr[p] = f2_pack(v[2 * p], v[2 * p + 1]);
+#pragma unroll
+  for (int hp = 1; hp < 8; hp <<= 1) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      if (!(p & hp)) {
+        const uint64_t a = pr[p], b = pr[p + hp];
+        pr[p] = f2_add(a, b);
+        pr[p + hp] = f2_sub(a, b);
+      }
+    }
+  }
+  const uint64_t quarter = f2_pack(0.25f, 0.25f);
+#pragma unroll
+  for (int p = 0; p < 8; ++p) f2_unpack(f2_mul(pr[p], quarter), v[2 * p], v[2 * p + 1]);
 }
 
 // Sign-flip mask for a word holding two BF16 elements that both have group index i.
@@ -117,8 +132,9 @@ __device__ __forceinline__ float absmax16(const float* v) { return fmaxf(absmax8
 template <bool SR>
 __device__ __forceinline__ uint32_t encode8(const float* v, float r, uint32_t w0, uint32_t w1) {
   float y[8];
+  const uint64_t rr = f2_pack(r, r);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(v[j], r);
+  for (int j = 0; j < 8; j += 2) f2_unpack(f2_mul(f2_pack(v[j], v[j + 1]), rr), y[j], y[j + 1]);
   if (SR) return e2m1x4_rs(y[0], y[1], y[2], y[3], w0) | (e2m1x4_rs(y[4], y[5], y[6], y[7], w1) << 16);
   return e2m1x8_rn(y);
 }
