@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // tcgen05 fences around it, and a release arrival costs over a thousand cycles.
 // =====================================================================================
 
-constexpr int P_STAGES = 6;                                         // operand ring
+constexpr int P_STAGES = 5;                                         // operand ring
 constexpr int P_SF_STAGES = 4;                                      // scale ring (shared memory)
 constexpr int P_SF_SLOTS = 5;                                       // scale slots in tensor memory
 constexpr int P_A_BYTES = 128 * BK_BYTES;                           // 16 KiB, own A rows
@@ -436,7 +436,10 @@ constexpr int P_SFB_BYTES = 2 * (BK / MMA_K) * SF_ATOM;             // 4 KiB, al
 constexpr int P_AB_BYTES = P_A_BYTES + P_B_BYTES;                   // operand bytes per CTA and stage
 constexpr int P_SF_BYTES = P_SFA_BYTES + P_SFB_BYTES;               // scale bytes per CTA and stage
 constexpr int P_SF_OFFSET = P_STAGES * P_AB_BYTES;                  // scale ring after the operands
-constexpr int P_BAR_OFFSET = P_SF_OFFSET + P_SF_STAGES * P_SF_BYTES;
+constexpr int P_EPI_BOX_COLS = 64;                                  // BF16 output box: 64 columns x 32 rows
+constexpr int P_EPI_BOX_BYTES = 32 * P_EPI_BOX_COLS * 2;            // 4 KiB, one per epilogue warp
+constexpr int P_EPI_OFFSET = P_SF_OFFSET + P_SF_STAGES * P_SF_BYTES;
+constexpr int P_BAR_OFFSET = P_EPI_OFFSET + NUM_EPI_WARPS * P_EPI_BOX_BYTES;
 constexpr int P_NUM_BARS = 3 * P_STAGES + 2 * P_SF_STAGES + 4;
 constexpr int P_BAR_BYTES = 512;
 constexpr int P_SMEM_BYTES = P_BAR_OFFSET + P_BAR_BYTES + 1024;
@@ -450,7 +453,7 @@ constexpr int P_SF_COL0 = 256;                                      // scale slo
 constexpr int P_SF_SLOT_COLS = 48;                                  // 16 A-scale + 32 B-scale columns
 constexpr int P_PREFETCH = 8;                                       // next-tile stages warmed in L2
 static_assert(P_SF_COL0 + P_SF_SLOTS * P_SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed tensor memory");
-static_assert(P_SF_SLOTS < P_STAGES, "a scale slot must free no later than the operand stage it serves");
+static_assert(P_SF_SLOTS <= P_STAGES, "a scale slot must free no later than the operand stage it serves");
 static_assert(8 * P_NUM_BARS + 8 <= P_BAR_BYTES, "barrier area too small");
 static_assert(P_SMEM_BYTES <= 232448, "shared memory above the sm_100 limit");
 static_assert(P_SF_BYTES % 128 == 0 && P_AB_BYTES % 1024 == 0, "ring alignment");
@@ -501,6 +504,18 @@ __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t 
                : "memory");
 }
 
+// TMA store of a tile from shared memory (bulk async group of the issuing thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int32_t x, int32_t y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(x),
+               "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the shared memory of every committed store has been read (it may be reused).
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until every committed store has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Two FP32 values scaled by g, rounded to BF16 (nearest even) and packed, lo in the low half.
 __device__ __forceinline__ uint32_t scale_pack_bf16x2(uint32_t lo, uint32_t hi, float g) {
   uint32_t out;
@@ -541,7 +556,7 @@ __device__ __forceinline__ TileCoord pair_tile_coord(const Params& p, int32_t t)
 __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     gemm_kernel_pair(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                      const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
-                     const Params p) {
+                     const __grid_constant__ CUtensorMap tma_c, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t smem_base = smem_u32(smem);
@@ -834,7 +849,12 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       const int chunks = mine ? min(4, (n_cols - half * 128) / 32) : 0;
       if (packed) {
         // BF16 without accumulation: scale and round while reading, so the 128
-        // columns of this warp stay in 64 registers; release, then store.
+        // columns of this warp stay in 64 registers; release the accumulator, then
+        // write the warp's 32 x 128 block out as two 32 x 64 TMA stores staged in
+        // its own 4 KB of shared memory (128-byte swizzle: lane r puts 16-byte chunk
+        // c of its row at chunk c ^ (r % 8), which keeps each quarter-warp on
+        // distinct banks).  Whole-line bulk stores instead of per-row 16-byte
+        // stores keep the output burst at every tile change off the operand loads.
         uint32_t pk[64];
         if (mine) {
 #pragma unroll
@@ -850,15 +870,24 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster_tc(leader_acc_empty);
-        if (m < p.M) {
-          uint4* crow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.C) + (size_t)(m * p.ldc + n0));
+        const int32_t m0 = tc.m_blk * P_BM + (int32_t)rank * 128 + quarter * 32;
+        uint8_t* stg = smem + P_EPI_OFFSET + ew * P_EPI_BOX_BYTES;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            if (k < chunks)
+        for (int hh = 0; hh < 2; ++hh) {
+          if (n_cols <= half * 128 + hh * P_EPI_BOX_COLS || m0 >= p.M) continue;   // box outside C
+          if (lane == 0) bulk_wait_read();                                 // staging buffer free again
+          __syncwarp();
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-                crow[4 * k + q] = make_uint4(pk[16 * k + 4 * q], pk[16 * k + 4 * q + 1], pk[16 * k + 4 * q + 2],
-                                             pk[16 * k + 4 * q + 3]);
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(pk[32 * hh + 4 * c], pk[32 * hh + 4 * c + 1], pk[32 * hh + 4 * c + 2],
+                           pk[32 * hh + 4 * c + 3]);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tma_c, (int32_t)n0 + hh * P_EPI_BOX_COLS, m0, smem_u32(stg));
+            bulk_commit();
+          }
         }
       } else {
         // FP32 output or accumulation into C: 32 columns at a time, released at the end.
@@ -879,6 +908,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       }
       acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();                   // this warp's output stores have landed
   }
 
   tc_fence_before();

@@ -122,6 +122,23 @@ nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t, uint32_t box
   return NVFP4_OK;
 }
 
+// Tensor map of a BF16 output C [M x N] (row stride ldc elements) for the pair
+// GEMM's epilogue stores: boxes of 32 rows x 64 columns, 128-byte swizzle.
+nvfp4_status make_out_map(CUtensorMap* map, void* C, int64_t M, int64_t N, int64_t ldc) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  nvfp4_status st = get_encoder(&encode);
+  if (st != NVFP4_OK) return st;
+  const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)ldc * 2u};
+  const cuuint32_t box[2] = {(cuuint32_t)nvfp4::gemm::P_EPI_BOX_COLS, 32u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled(C) failed (%d)", (int)r);
+  return NVFP4_OK;
+}
+
 // Tensor map over the tensor-core scale layout viewed as rows of 512-byte
 // atoms (128 x 32-bit words): box of 4 atoms = one 128-row block x 256 K.
 nvfp4_status make_scale_map(CUtensorMap* map, const nvfp4_tensor* t) {
@@ -453,11 +470,15 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, i
   cudaError_t e;
   if (M >= 256 && dev->pair_clusters > 0) {
     // CTA pairs, 256 x 256 tiles
-    CUtensorMap map_a, map_b, map_sfa, map_sfb;
+    CUtensorMap map_a, map_b, map_sfa, map_sfb, map_c;
     if ((st = make_code_map(&map_a, A, 128)) != NVFP4_OK) return st;
     if ((st = make_code_map(&map_b, B, 128)) != NVFP4_OK) return st;
     if ((st = make_scale_map(&map_sfa, A)) != NVFP4_OK) return st;
     if ((st = make_scale_map(&map_sfb, B)) != NVFP4_OK) return st;
+    // the BF16 store map is only read by the BF16, non-accumulating epilogue
+    std::memset(&map_c, 0, sizeof(map_c));
+    if (out_dtype == NVFP4_OUT_BF16 && !accumulate && (st = make_out_map(&map_c, C, M, N, ldc)) != NVFP4_OK)
+      return st;
     p.num_m = (int32_t)ceil_div(M, nvfp4::gemm::P_BM);
     p.group_m = 8;
     const int64_t tiles = (int64_t)p.num_m * p.num_n;
@@ -474,7 +495,7 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, i
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, nvfp4::gemm::gemm_kernel_pair, map_a, map_b, map_sfa, map_sfb, p);
+    e = cudaLaunchKernelEx(&cfg, nvfp4::gemm::gemm_kernel_pair, map_a, map_b, map_sfa, map_sfb, map_c, p);
   } else {
     CUtensorMap map_a, map_b;
     if ((st = make_code_map(&map_a, A, nvfp4::gemm::BM)) != NVFP4_OK) return st;
