@@ -256,6 +256,23 @@ __device__ __forceinline__ BlockScale block_scale(float bmax, float S) {
   return out;
 }
 
+// The encode multiplier of an E4M3 scale byte under tensor scale S, with the
+// dead-block rule of block_scale (0 when s == 0, s * S == 0 or 1 / (s * S) is not
+// finite).  A kernel tabulates it for all 128 non-negative bytes once per S.
+__device__ __forceinline__ float scale_multiplier(uint32_t sbyte, float S) {
+  const float d = __fmul_rn(e4m3_decode(sbyte), S);
+  const float r = __fdiv_rn(1.0f, d);
+  return (sbyte == 0u || d == 0.0f || !isfinite(r)) ? 0.0f : r;
+}
+
+// block_scale with the multiplier looked up in such a table (bit-identical).
+__device__ __forceinline__ BlockScale block_scale_tab(float bmax, float S, const float* rtab) {
+  BlockScale out;
+  out.sbyte = e4m3_encode_hw(__fdiv_rn(__fdiv_rn(bmax, 6.0f), S));
+  out.r = rtab[out.sbyte & 0x7Fu];
+  return out;
+}
+
 // Byte offset of block scale (row r, block j) in the tensor-core scale layout:
 // tiles of 128 rows x 4 blocks, tile-major along the blocks.
 __device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t j, int64_t kgroups) {

@@ -6,6 +6,11 @@
 // accumulator is FP32 in tensor memory and the global scales are applied once,
 // in the epilogue.
 //
+// Two kernels.  gemm_kernel_pair (further below) serves M >= 256: CTA pairs
+// (cta_group::2) on 256 x 256 output tiles, block scales stored into tensor memory
+// by writer warps, two MMA-issuing warps, BF16 output through TMA stores.
+// gemm_kernel serves M = 128 and devices that cannot co-schedule a pair:
+//
 // Structure (one CTA per SM, persistent over output tiles of 128 x 256):
 //   warp 0      TMA producer: per K-stage of 256 elements, one tiled TMA load of
 //               A (128 rows x 128 bytes) and of B (256 x 128 bytes), 128-byte
@@ -16,7 +21,7 @@
 //               block16 (M=128, N=256, K=64) into an FP32 accumulator in tensor
 //               memory; tcgen05.commit frees the stage and, after the last one,
 //               hands the accumulator to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter of the
+//   warps 2..9  epilogue: tcgen05.ld of their 32-lane quarter of the
 //               accumulator, scale by alpha*S_A*S_B, round to BF16 (or keep FP32),
 //               store; then release the accumulator.
 // All waits are bounded (see mbar_wait): a stuck pipeline records an error

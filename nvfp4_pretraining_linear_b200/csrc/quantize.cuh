@@ -39,7 +39,7 @@ constexpr int kQStages = 3;
 constexpr int kQComputeWarps = 8;
 constexpr int kQThreads = 32 * (kQComputeWarps + 1);  // 288
 constexpr int kQCtasPerSm = 2;
-constexpr int kQSmemBytes = kQStages * kTileBytes + 256 + 128;
+constexpr int kQSmemBytes = kQStages * kTileBytes + 256 + 1024 + 128;   // tiles, barriers, scale tables
 
 struct QuantLayout {
   uint8_t* codes;       // nullptr when the layout is not emitted
@@ -222,6 +222,11 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     const float amax_row = RR ? p.amax[2] : amax_raw;
     S_row = tensor_scale_from_amax(amax_row);
     S_col = tensor_scale_from_amax(amax_col);
+    // encode multipliers of all E4M3 scale bytes for both tensor scales
+    float* tab = reinterpret_cast<float*>(smem + kQStages * kTileBytes + 256);
+    if (ct < 128) tab[ct] = scale_multiplier((uint32_t)ct, S_row);
+    else tab[ct] = scale_multiplier((uint32_t)(ct - 128), S_col);
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kQComputeWarps) : "memory");
     if (blockIdx.x == 0 && ct == 0) {
       if (ER) *p.row.tensor_scale = S_row;
       if (EC) *p.col.tensor_scale = S_col;
@@ -232,6 +237,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
       }
     }
   }
+  const float* rtab_row = reinterpret_cast<const float*>(smem + kQStages * kTileBytes + 256);
+  const float* rtab_col = rtab_row + 128;
   float m_raw = 0.0f, m_col = 0.0f, m_row = 0.0f;
   const int64_t nblk_row = cols / 16, nblk_col = rows / 16;
   const int64_t rows_padded = (rows + 127) & ~int64_t(127);
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
         tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 16));
       }
       BlockScale tbs;
-      if (TD && !AMAX) tbs = block_scale(tile_max, S_row);
+      if (TD && !AMAX) tbs = block_scale_tab(tile_max, S_row, rtab_row);
 #pragma unroll 2
       for (int it = 0; it < 4; ++it) {
         const int rl = cw * 16 + it * 4 + rsub;
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
             continue;
           }
         }
-        const BlockScale bs = TD ? tbs : block_scale(absmax16(v), S_row);
+        const BlockScale bs = TD ? tbs : block_scale_tab(absmax16(v), S_row, rtab_row);
         uint4 w = make_uint4(0u, 0u, 0u, 0u);
         if (SR) w = philox_block((uint64_t)(r * cols + c) >> 4, 0u, p.offset, p.key0, p.key1);
         // v[0..7] holds the half read first; pick the matching random words
@@ -370,7 +377,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const float* v = k ? vb : va;
-          const BlockScale bs = block_scale(k ? mb : ma, S_col);
+          const BlockScale bs = block_scale_tab(k ? mb : ma, S_col, rtab_col);
           uint4 w = make_uint4(0u, 0u, 0u, 0u);
           if (SR) {
             const int64_t c = c_base + 2 * cp + k;
