@@ -156,6 +156,23 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor* q, void* out, int64_t ldo, int
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc,
                         int32_t out_dtype, float alpha, int32_t accumulate, void* stream);
 
+/* nvfp4_gemm with BF16 output that also reports, from its epilogue, the maxima the
+ * next quantisation of C needs, so that quantisation can skip its amax pass (pass
+ * amax_out as its nvfp4_quant_opts.amax_in).  The tensor scales of the format
+ * passage of the 12B NVFP4 page come from these maxima; the page's recipe applies
+ * the 16x16 random Hadamard transform to the weight-gradient operands, which for an
+ * output that becomes the next linear's activations is its col layout.
+ *   amax_out : 3 device floats, written by this call (stream-ordered):
+ *              [0] max |C| over the stored BF16 values,
+ *              [1] max |RHT16(C)| over C's col layout (16-row groups along M, sign
+ *                  mask rht_signs, the transform of nvfp4_quantize's rht_col),
+ *              [2] 0 (no row transform).
+ * C is BF16 without accumulation; requires M >= 256 (the CTA-pair kernel) besides
+ * the conditions of nvfp4_gemm.  Extends the hot path of the pages (the GEMM
+ * epilogue feeding the next quantiser); the pages describe no such fusion. */
+nvfp4_status nvfp4_gemm_amax(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc,
+                             float alpha, uint32_t rht_signs, float* amax_out, void* stream);
+
 /* Linear forward (fprop): Y [M x N] = Q(X) . Q(W)^T.
  *   X      : BF16 [M x K] activations (device, row stride ldx), quantised here
  *            row-wise with round-to-nearest-even into Xq_row (caller buffers,

@@ -68,6 +68,7 @@ SIGNATURES = {
     "nvfp4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_int64, O_P, T_P, T_P, c_void_p, c_size_t, c_void_p]),
     "nvfp4_dequantize": (c_int32, [T_P, c_void_p, c_int64, c_int32, c_void_p]),
     "nvfp4_gemm": (c_int32, [T_P, T_P, c_void_p, c_int64, c_int32, c_float, c_int32, c_void_p]),
+    "nvfp4_gemm_amax": (c_int32, [T_P, T_P, c_void_p, c_int64, c_float, c_uint32, c_void_p, c_void_p]),
     "nvfp4_linear_fwd": (c_int32, [c_void_p, c_int64, c_int64, c_int64, T_P, c_void_p, c_int64, c_int32, T_P, T_P,
                                    c_uint32, c_void_p, c_size_t, c_void_p]),
     "nvfp4_linear_dgrad": (c_int32, [c_void_p, c_int64, c_int64, c_int64, T_P, c_void_p, c_int64, c_int32, T_P, T_P,

@@ -105,6 +105,20 @@ def gemm(A: QTensor, B: QTensor, out_dtype=torch.bfloat16, alpha=1.0, accumulate
     return out
 
 
+def gemm_amax(A: QTensor, B: QTensor, alpha=1.0, rht_signs=0, out: Optional[torch.Tensor] = None,
+              amax: Optional[torch.Tensor] = None, stream=None):
+    """nvfp4_gemm_amax: BF16 C = alpha * S_A * S_B * A . B^T and the maxima its next
+    quantisation needs, as a 3-float device tensor usable as quantize(amax_in=...)."""
+    lib = _lib.load()
+    if out is None:
+        out = torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=A.codes.device)
+    if amax is None:
+        amax = torch.empty(3, dtype=torch.float32, device=A.codes.device)
+    _lib.check(lib.nvfp4_gemm_amax(A.struct(), B.struct(), out.data_ptr(), out.stride(0), alpha, rht_signs & 0xFFFF,
+                                   amax.data_ptr(), _stream_ptr(stream)))
+    return out, amax
+
+
 def quantize_weight(w: torch.Tensor, stream=None):
     """2D 16x16-block quantisation of a weight [N, K]: (row layout [N x K], col layout [K x N])."""
     return quantize(w, emit_row=True, emit_col=True, block_2d=True, stream=stream)

@@ -72,6 +72,8 @@ struct Params {
   int64_t ldc;
   int32_t out_f32;
   int32_t accumulate;
+  unsigned* amax_acc;       // nullptr, or 2 words receiving max|C| and max|RHT16 col(C)| (float bits)
+  uint32_t rht_signs;       // sign mask of that transform
 };
 
 // Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), UE4M3
@@ -521,6 +523,45 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 // Wait until every committed store has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Maxima of a staged 32 x 64 BF16 output box (rows 128 bytes, 128-byte swizzle) that
+// the next quantiser of C needs, folded into mraw / mrht: max |x|, and max |w| over
+// the 16-point Walsh-Hadamard transforms w (before their 1/4) of each 16-row group
+// of each column, signs applied first -- the col layout's transform, blocks along M.
+// Lane t takes columns 2t and 2t+1 (one word per row); the butterflies run on the
+// column pair as packed FP32, in the transform's own order (stages 1, 2, 4, 8).
+__device__ __forceinline__ void box_amax(const uint8_t* stg, int lane, uint32_t signs, float& mraw, float& mrht) {
+  const uint32_t chunk = (uint32_t)lane >> 2, wsub = ((uint32_t)lane & 3u) * 4u;
+#pragma unroll
+  for (int grp = 0; grp < 2; ++grp) {
+    uint64_t pr[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int r = 16 * grp + i;
+      uint32_t w = *reinterpret_cast<const uint32_t*>(stg + r * 128 + ((chunk ^ (uint32_t)(r & 7)) << 4) + wsub);
+      mraw = fmaxf(mraw, fmaxf(fabsf(bf16_lo(w)), fabsf(bf16_hi(w))));
+      w ^= ((signs >> i) & 1u) * 0x80008000u;
+      pr[i] = f2_pack(bf16_lo(w), bf16_hi(w));
+    }
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (!(i & h)) {
+          const uint64_t a = pr[i], b = pr[i + h];
+          pr[i] = f2_add(a, b);
+          pr[i + h] = f2_sub(a, b);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float lo, hi;
+      f2_unpack(pr[i], lo, hi);
+      mrht = fmaxf(mrht, fmaxf(fabsf(lo), fabsf(hi)));
+    }
+  }
+}
+
 // Two FP32 values scaled by g, rounded to BF16 (nearest even) and packed, lo in the low half.
 __device__ __forceinline__ uint32_t scale_pack_bf16x2(uint32_t lo, uint32_t hi, float g) {
   uint32_t out;
@@ -877,6 +918,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
         if (lane == 0) mbar_arrive_cluster_tc(leader_acc_empty);
         const int32_t m0 = tc.m_blk * P_BM + (int32_t)rank * 128 + quarter * 32;
         uint8_t* stg = smem + P_EPI_OFFSET + ew * P_EPI_BOX_BYTES;
+        float mraw = 0.0f, mrht = 0.0f;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           if (n_cols <= half * 128 + hh * P_EPI_BOX_COLS || m0 >= p.M) continue;   // box outside C
@@ -892,6 +934,22 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           if (lane == 0) {
             tma_store_2d(&tma_c, (int32_t)n0 + hh * P_EPI_BOX_COLS, m0, smem_u32(stg));
             bulk_commit();
+          }
+          if (p.amax_acc) box_amax(stg, lane, p.rht_signs, mraw, mrht);
+        }
+        if (p.amax_acc) {
+          // boxes past the end of C hold zeros (their operand rows were zero-filled), so
+          // the maxima need no masking; 0.25 * max |w| = max |w / 4| (scaling by 1/4 is
+          // monotonic in round-to-nearest)
+          mrht = __fmul_rn(mrht, 0.25f);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            mraw = fmaxf(mraw, __shfl_xor_sync(0xFFFFFFFFu, mraw, o));
+            mrht = fmaxf(mrht, __shfl_xor_sync(0xFFFFFFFFu, mrht, o));
+          }
+          if (lane == 0) {
+            atomicMax(p.amax_acc, __float_as_uint(mraw));          // non-negative floats order as their bits
+            atomicMax(p.amax_acc + 1, __float_as_uint(mrht));
           }
         }
       } else {

@@ -417,8 +417,10 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor* q, void* out, int64_t ldo, int
   return NVFP4_OK;
 }
 
-nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc, int32_t out_dtype,
-                        float alpha, int32_t accumulate, void* stream) {
+namespace {
+// nvfp4_gemm, and with amax_out (3 floats) the maxima of nvfp4_gemm_amax.
+nvfp4_status gemm_impl(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc, int32_t out_dtype,
+                       float alpha, int32_t accumulate, float* amax_out, uint32_t rht_signs, void* stream) {
   nvfp4_status st;
   if ((st = check_tensor(A, "A")) != NVFP4_OK) return st;
   if ((st = check_tensor(B, "B")) != NVFP4_OK) return st;
@@ -432,13 +434,20 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, i
                 (long long)M, (long long)N, (long long)K);
   if (M > (1ll << 31) - 128 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256)
     return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "GEMM extent above 2^31");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (amax_out) {
+    if (out_dtype != NVFP4_OUT_BF16 || accumulate)
+      return fail(NVFP4_ERR_INVALID_ARG, "the output maxima need BF16 output without accumulation");
+    if (M != 0 && M < 256) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the output maxima need M >= 256");
+    const cudaError_t e = cudaMemsetAsync(amax_out, 0, 3 * sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(amax_out)");
+  }
   if (M == 0 || N == 0) return NVFP4_OK;
   if (!C) return fail(NVFP4_ERR_INVALID_ARG, "C is NULL");
   if (ldc < N) return fail(NVFP4_ERR_INVALID_ARG, "ldc < N");
   if (!aligned16(C) || (ldc * (out_dtype == NVFP4_OUT_F32 ? 4 : 2)) % 16)
     return fail(NVFP4_ERR_MISALIGNED, "C rows are not 16-byte aligned");
   if (!aligned16(A->scales) || !aligned16(B->scales)) return fail(NVFP4_ERR_MISALIGNED, "scales not 16-byte aligned");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (K == 0) {
     // empty contraction: C = 0 (or unchanged when accumulating)
     if (accumulate) return NVFP4_OK;
@@ -467,7 +476,11 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, i
   p.ldc = ldc;
   p.out_f32 = out_dtype == NVFP4_OUT_F32;
   p.accumulate = accumulate != 0;
+  p.amax_acc = reinterpret_cast<unsigned*>(amax_out);
+  p.rht_signs = rht_signs & 0xFFFFu;
   cudaError_t e;
+  if (amax_out && dev->pair_clusters == 0)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the output maxima need the CTA-pair GEMM, not available on this device");
   if (M >= 256 && dev->pair_clusters > 0) {
     // CTA pairs, 256 x 256 tiles
     CUtensorMap map_a, map_b, map_sfa, map_sfb, map_c;
@@ -509,6 +522,19 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, i
   }
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return NVFP4_OK;
+}
+}  // namespace
+
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc, int32_t out_dtype,
+                        float alpha, int32_t accumulate, void* stream) {
+  return gemm_impl(A, B, C, ldc, out_dtype, alpha, accumulate, nullptr, 0u, stream);
+}
+
+nvfp4_status nvfp4_gemm_amax(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc, float alpha,
+                             uint32_t rht_signs, float* amax_out, void* stream) {
+  if (!amax_out) return fail(NVFP4_ERR_INVALID_ARG, "amax_out is NULL");
+  if (reinterpret_cast<uintptr_t>(amax_out) % 4) return fail(NVFP4_ERR_MISALIGNED, "amax_out is not 4-byte aligned");
+  return gemm_impl(A, B, C, ldc, NVFP4_OUT_BF16, alpha, 0, amax_out, rht_signs, stream);
 }
 
 nvfp4_status nvfp4_linear_fwd(const void* X, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* Wq_row, void* Y,
