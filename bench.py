@@ -494,6 +494,8 @@ def run_kernel(args):
     torch.cuda.set_device(0)
     dims = [int(v) for v in args.shape.split(",")]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    if args.kernel == "chain":
+        return run_chain(args, dims, flush)
     if args.kernel == "gemm":
         M, N, K = dims
         qa, _ = api.quantize(syn.normal((M, K), 1.0, seed=30, device="cuda"))
@@ -534,6 +536,51 @@ def run_kernel(args):
     return 0
 
 
+def run_chain(args, dims, flush):
+    """A GEMM whose BF16 output is quantised next (row + RHT col, as the next linear's
+    activations): nvfp4_gemm then the two-pass quantiser, against nvfp4_gemm_amax then
+    the quantiser given the epilogue's maxima (no amax pass)."""
+    from nvfp4_pretraining_linear_b200 import api, synthetic as syn
+    M, N, K = dims
+    qa, _ = api.quantize(syn.normal((M, K), 1.0, seed=30, device="cuda"))
+    qb, _ = api.quantize(syn.normal((N, K), 1.0, seed=31, device="cuda"))
+    c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    amax = torch.empty(3, dtype=torch.float32, device="cuda")
+    rq, cq = api.QTensor.empty(M, N), api.QTensor.empty(N, M)
+    qkw = dict(emit_row=True, emit_col=True, rht_col=True, rht_signs=RHT_SIGNS, out_row=rq, out_col=cq)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    t_gemm = timed(lambda: api.gemm(qa, qb, out=c))
+    t_gemm_amax = timed(lambda: api.gemm_amax(qa, qb, rht_signs=RHT_SIGNS, out=c, amax=amax))
+    t_quant = timed(lambda: api.quantize(c, **qkw))
+    t_quant_in = timed(lambda: api.quantize(c, amax_in=amax, **qkw))
+    t_plain = timed(lambda: (api.gemm(qa, qb, out=c), api.quantize(c, **qkw)))
+    t_fused = timed(lambda: (api.gemm_amax(qa, qb, rht_signs=RHT_SIGNS, out=c, amax=amax),
+                             api.quantize(c, amax_in=amax, **qkw)))
+    api.get_status()
+    flops = 2.0 * M * N * K
+    print(json.dumps({"kernel": "chain", "shape": dims, "gemm_ms": t_gemm, "gemm_amax_ms": t_gemm_amax,
+                      "gemm_tflops": flops / t_gemm / 1e9, "gemm_amax_tflops": flops / t_gemm_amax / 1e9,
+                      "quantize_two_pass_ms": t_quant, "quantize_amax_in_ms": t_quant_in,
+                      "chain_plain_ms": t_plain, "chain_fused_ms": t_fused,
+                      "steps": args.steps, "l2": "flushed (256 MB write)"}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -543,8 +590,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["step", "gemm", "quantize"], default="step",
-                    help="step: the contract benchmark; gemm/quantize: one kernel on --shape")
+    ap.add_argument("--kernel", choices=["step", "gemm", "quantize", "chain"], default="step",
+                    help="step: the contract benchmark; gemm/quantize: one kernel on --shape; chain: GEMM then "
+                         "quantise its output, plain against epilogue-fused amax (--shape M,N,K)")
     ap.add_argument("--shape", default="16384,16384,16384")
     ap.add_argument("--mode", choices=sorted(QUANT_MODES), default="grad")
     args = ap.parse_args()
