@@ -15,6 +15,12 @@ c_size_t = ctypes.c_size_t
 c_float = ctypes.c_float
 
 NVFP4_OK = 0
+NVFP4_ERR_INVALID_ARG = 1
+NVFP4_ERR_UNSUPPORTED_SHAPE = 2
+NVFP4_ERR_MISALIGNED = 3
+NVFP4_ERR_CUDA = 4
+NVFP4_ERR_TIMEOUT = 5
+NVFP4_ERR_WORKSPACE = 6
 STATUS_NAMES = {
     0: "NVFP4_OK",
     1: "NVFP4_ERR_INVALID_ARG",

@@ -9,6 +9,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -198,6 +199,18 @@ cudaError_t ensure_smem(Kernel kernel, int bytes, bool (&done)[kMaxDevices], std
   return e;
 }
 
+// Host-side fault injection for failure-detection tests: with NVFP4_INJECT_SKIP_TILE=n
+// in the environment, the quantise pass never loads its tile n, so a compute warp's
+// bounded wait expires and nvfp4_get_status reports NVFP4_ERR_TIMEOUT.  Nothing
+// faults, traps or hangs; unset (the default) it costs one getenv per call.
+int64_t injected_skip_tile() {
+  const char* v = std::getenv("NVFP4_INJECT_SKIP_TILE");
+  if (!v || !*v) return -1;
+  char* end = nullptr;
+  const long long n = std::strtoll(v, &end, 10);
+  return (end && *end == '\0' && n >= 0) ? (int64_t)n : -1;
+}
+
 template <bool AM, bool ER, bool EC, bool SR, bool RR, bool RC, bool TD>
 cudaError_t launch_tiles(const CUtensorMap& map, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
   static bool done[kMaxDevices] = {};
@@ -378,6 +391,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
   p.key1 = (uint32_t)(opts->seed >> 32);
   p.offset = (uint32_t)opts->offset;
   p.signs = opts->rht_signs;
+  p.skip_tile = -1;
   const int grid = (int)std::min<int64_t>(p.tiles, (int64_t)dev->sm_count * nvfp4::kQCtasPerSm);
   if (!amax) {
     unsigned* acc = static_cast<unsigned*>(workspace);
@@ -390,6 +404,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
   }
   p.amax = amax;
   p.amax_acc = nullptr;
+  p.skip_tile = injected_skip_tile();
   e = dispatch_quant(out_row != nullptr, out_col != nullptr, opts->stochastic != 0, opts->rht_row != 0,
                      opts->rht_col != 0, opts->block_2d != 0, map, p, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");

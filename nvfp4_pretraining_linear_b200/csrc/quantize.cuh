@@ -61,6 +61,7 @@ struct QuantParams {
   uint32_t key0, key1;  // Philox key (seed)
   uint32_t offset;      // Philox counter word 3
   uint32_t signs;       // RHT sign mask
+  int64_t skip_tile;    // fault injection: the producer never loads this tile (-1: off)
 };
 
 __device__ __forceinline__ void unpack8(const uint4& w, float* v) {
@@ -188,6 +189,16 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
           break;
         }
         const int64_t tr = t / p.tiles_c, tc = t - tr * p.tiles_c;
+        if (t == p.skip_tile) {
+          // fault injection: this stage's data never arrives, so the compute warps'
+          // bounded wait on it expires and records kErrTimeout; nothing is in flight
+          issued[stage] = false;
+          if (++stage == kQStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          continue;
+        }
         mbar_arrive_expect_tx(full_bar(stage), kTileBytes);
         tma_load_tile(smem_base + stage * kTileBytes, &xmap, (int32_t)(tc * kTileCols), (int32_t)(tr * kTileRows),
                       full_bar(stage));
