@@ -290,6 +290,15 @@ def time_oracle(min_seconds=10.0, min_steps=3):
             "sample": desc + "; median of %d steps, %.2f s each" % (len(times), t)}
 
 
+def step_config(world):
+    """The `config` of the bench line: the 12B hybrid MLP step, the same for both arms."""
+    from nvfp4_pretraining_linear_b200 import synthetic as syn
+    return {"workload": WORKLOAD, "tokens_per_gpu": syn.HYBRID12B["tokens"], "hidden": syn.HYBRID12B["hidden"],
+            "ffn": syn.HYBRID12B["ffn"], "linears": ["up 5120->20480", "down 20480->5120"],
+            "gemms_per_step": 6, "parallelism": "dp%d" % world,
+            "l2": "every input larger than the 126 MB L2; no flush"}
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -305,7 +314,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantise / f64 GEMM",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "sample": desc},
+            "data": "synthetic", "config": step_config(args.gpus),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -377,7 +386,6 @@ def run_ours(args):
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
     quant_gbs = qbytes / (quant_ms * 1e-3) / 1e9
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    gemm_launches = 3 * len(linears)
     traffic = gemm_traffic_per_launch()
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
@@ -449,10 +457,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3 block scales, fp32 accumulate), bf16 in/out",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "tokens_per_gpu": linears[0].M, "hidden": linears[0].K,
-                       "ffn": linears[0].N, "linears": ["up 5120->20480", "down 20480->5120"],
-                       "gemms_per_step": gemm_launches, "parallelism": "dp%d" % world,
-                       "l2": "every input larger than the 126 MB L2; no flush"},
+            "config": step_config(world),
             "gpu_launches": LAUNCHES_PER_LINEAR * len(linears) * args.steps,
             "quantizer": {"gbs": quant_gbs, "frac_hbm": quant_gbs / hbm, "hbm_peak_gbs": hbm,
                           "peak_source": peak_src, "ms_per_step": quant_ms,
