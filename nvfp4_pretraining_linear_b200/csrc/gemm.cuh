@@ -458,7 +458,7 @@ constexpr int P_SF_PRODUCER = P_WRITER0 + P_NUM_WRITERS;            // warp 15: 
 constexpr int P_NUM_THREADS = 32 * (P_SF_PRODUCER + 1);             // 512
 constexpr int P_SF_COL0 = 256;                                      // scale slot s at 256 + 48 s
 constexpr int P_SF_SLOT_COLS = 48;                                  // 16 A-scale + 32 B-scale columns
-constexpr int P_PREFETCH = 8;                                       // next-tile stages warmed in L2
+constexpr int P_PREFETCH = 4;                                       // next-tile stages warmed in L2
 static_assert(P_SF_COL0 + P_SF_SLOTS * P_SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed tensor memory");
 static_assert(P_SF_SLOTS <= P_STAGES, "a scale slot must free no later than the operand stage it serves");
 static_assert(8 * P_NUM_BARS + 8 <= P_BAR_BYTES, "barrier area too small");

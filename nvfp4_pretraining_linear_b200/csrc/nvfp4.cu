@@ -508,7 +508,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, in
     if (out_dtype == NVFP4_OUT_BF16 && !accumulate && (st = make_out_map(&map_c, C, M, N, ldc)) != NVFP4_OK)
       return st;
     p.num_m = (int32_t)ceil_div(M, nvfp4::gemm::P_BM);
-    p.group_m = 8;
+    p.group_m = 16;
     const int64_t tiles = (int64_t)p.num_m * p.num_n;
     const int pairs = (int)std::min<int64_t>(tiles, dev->pair_clusters);
     cudaLaunchConfig_t cfg = {};
