@@ -514,9 +514,16 @@ def run_kernel(args):
         x = syn.student_t((R, C), 3, 0.1, seed=1, device="cuda")
         rq = api.QTensor.empty(R, C) if kw.get("emit_row") else None
         cq = api.QTensor.empty(C, R) if kw.get("emit_col") else None
-        fn = lambda: api.quantize(x, out_row=rq, out_col=cq, **kw)  # noqa: E731
         layouts = int(bool(kw.get("emit_row"))) + int(bool(kw.get("emit_col")))
-        work, unit = R * C * (4.0 + 0.5625 * layouts), "GB/s"
+        if args.amax_in:
+            # given maxima (delayed scaling, or the previous GEMM's epilogue): no amax pass
+            amax = torch.zeros(3, dtype=torch.float32, device="cuda")
+            api.quantize(x, out_row=rq, out_col=cq, amax_out=amax, **kw)
+            fn = lambda: api.quantize(x, out_row=rq, out_col=cq, amax_in=amax, **kw)  # noqa: E731
+            work, unit = R * C * (2.0 + 0.5625 * layouts), "GB/s"
+        else:
+            fn = lambda: api.quantize(x, out_row=rq, out_col=cq, **kw)  # noqa: E731
+            work, unit = R * C * (4.0 + 0.5625 * layouts), "GB/s"
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
@@ -535,6 +542,7 @@ def run_kernel(args):
     ms = statistics.median(times)
     rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
     print(json.dumps({"kernel": args.kernel, "shape": dims, "mode": args.mode if args.kernel == "quantize" else None,
+                      "amax_in": bool(args.amax_in) if args.kernel == "quantize" else None,
                       "ms": ms, "value": rate, "unit": unit, "steps": args.steps, "l2": "flushed (256 MB write)",
                       "clocks": clock_info}),
           flush=True)
@@ -600,6 +608,8 @@ def main():
                          "quantise its output, plain against epilogue-fused amax (--shape M,N,K)")
     ap.add_argument("--shape", default="16384,16384,16384")
     ap.add_argument("--mode", choices=sorted(QUANT_MODES), default="grad")
+    ap.add_argument("--amax-in", action="store_true",
+                    help="--kernel quantize: given maxima, no amax pass (2 B read + 0.5625 B per layout per element)")
     args = ap.parse_args()
     if args.kernel != "step":
         return run_kernel(args)
