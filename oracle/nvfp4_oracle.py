@@ -69,9 +69,24 @@ stated where it is used:
    and col layouts hold the same codes and scales, transposed.
 10. GEMM reference: C = A_hat . B_hat^T in FP64 from the dequantised FP32
     operands x_hat = (code * s) * S.
+11. Newton-Schulz in NVFP4.  [Full-Stack FP4]'s optimizer passage runs the
+    Newton-Schulz iterations of the Muon optimizer natively in NVFP4 but gives no
+    coefficients, iteration count or precision plan.  Reading: the coefficient-free
+    cubic Newton-Schulz iteration for the orthogonal polar factor (Bjorck and Bowie,
+    "An iterative algorithm for computing the best estimate of an orthogonal
+    matrix", SIAM J. Numer. Anal. 8 (1971); Higham, "Functions of Matrices" (2008),
+    ch. 8), X <- 3/2 X - 1/2 X X^T X, written in the equivalent residual form
+    X <- X + 1/2 R X with R = I - X X^T.  Both products are NVFP4 GEMMs (1D blocks of
+    16, round-to-nearest-even, no transform: the iterates are not gradients); the
+    iterate X and the residual R are held in BF16.  X_0 = G / ||G||_F, the norm from
+    the exactly rounded FP64 sum of squares, then rounded to FP32.  A product that
+    adds into a BF16 matrix C rounds as C <- BF16(fl32(fl32(alpha * sum) + C)), the
+    sum taken exactly and rounded once to FP32.
 """
 
 from __future__ import annotations
+
+import math
 
 import numpy as np
 
@@ -480,3 +495,68 @@ def linear_wgrad_ref(dyq: dict, xq: dict):
     a_hat = dequantize(*dyq["col"])
     b_hat = dequantize(*xq["col"])
     return gemm_ref(a_hat, b_hat), (a_hat, b_hat)
+
+
+# ---------------------------------------------------------------------------
+# Newton-Schulz orthogonalisation with NVFP4 products (reading 11)
+# ---------------------------------------------------------------------------
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """float32 -> the float32 value of its BF16 rounding (nearest even)."""
+    return bf16_bits_to_f32(f32_to_bf16_bits(x))
+
+
+def frobenius_norm(g: np.ndarray) -> np.float32:
+    """||G||_F: square root of the exactly rounded FP64 sum of squares, in FP64, then
+    rounded to FP32 (the squares of BF16 values are exact in FP64)."""
+    g64 = np.asarray(g, dtype=np.float64).ravel()
+    return F32(math.sqrt(math.fsum(g64 * g64)))
+
+
+def ns_normalize(g: np.ndarray):
+    """X_0 = BF16(fl32(G / ||G||_F)) and the norm; a zero G gives X_0 = 0."""
+    g = np.asarray(g, dtype=F32)
+    nrm = frobenius_norm(g)
+    if nrm == 0:
+        return np.zeros_like(g), nrm
+    return bf16_round((g / nrm).astype(F32)), nrm
+
+
+def add_product_bf16(prod64: np.ndarray, c: np.ndarray) -> np.ndarray:
+    """C <- BF16(fl32(fl32(P) + C)) for an exact product P (FP64) and a BF16 C."""
+    p32 = np.asarray(prod64, dtype=np.float64).astype(F32)
+    return bf16_round((p32 + np.asarray(c, dtype=F32)).astype(F32))
+
+
+def ns_step(x: np.ndarray):
+    """One NVFP4 Newton-Schulz step on a BF16 iterate X [m x n] (values in float32).
+
+    R = BF16(I - Xh Xh^T) with Xh the row layout of X (blocks along n); then
+    X' = BF16(X + 1/2 Rh Xh) with Rh the row layout of R and Xh now the col layout
+    of X (blocks along m).  Returns X' and the intermediates.
+    """
+    x = np.asarray(x, dtype=F32)
+    m = x.shape[0]
+    q = quantize(x, emit_row=True, emit_col=True)
+    x_row = dequantize(*q["row"])                 # [m x n]
+    x_col = dequantize(*q["col"])                 # [n x m]: X^T, blocks along m
+    r = add_product_bf16(gemm_ref(x_row, x_row, -1.0), np.eye(m, dtype=F32))
+    rq = quantize(r, emit_row=True)["row"]
+    r_hat = dequantize(*rq)
+    x_new = add_product_bf16(gemm_ref(r_hat, x_col, 0.5), x)
+    return x_new, {"q": q, "x_row": x_row, "x_col": x_col, "r": r, "rq": rq, "r_hat": r_hat}
+
+
+def newton_schulz(g: np.ndarray, iters: int, normalize: bool = True):
+    """X_iters of the NVFP4 Newton-Schulz iteration from G [m x n] (BF16 values).
+
+    Returns (X, ||G||_F or None)."""
+    g = np.asarray(g, dtype=F32)
+    if normalize:
+        x, nrm = ns_normalize(g)
+    else:
+        x, nrm = bf16_round(g), None
+    for _ in range(iters):
+        x, _ = ns_step(x)
+    return x, nrm
