@@ -501,6 +501,8 @@ def run_kernel(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     if args.kernel == "chain":
         return run_chain(args, dims, flush)
+    if args.kernel == "ns":
+        return run_ns(args, dims, flush)
     if args.kernel == "gemm":
         M, N, K = dims
         qa, _ = api.quantize(syn.normal((M, K), 1.0, seed=30, device="cuda"))
@@ -594,6 +596,142 @@ def run_chain(args, dims, flush):
     return 0
 
 
+def run_ns(args, dims, flush):
+    """nvfp4_newton_schulz on a Gaussian [m x n] matrix: the whole call (normalisation and
+    --iters steps, L2 flushed before each call) and, from the final iterate, each stage of
+    one step timed alone: quantise X (row + col), the GEMM adding -X X^T into R, quantise
+    R (row), the GEMM adding R X / 2 into X."""
+    from nvfp4_pretraining_linear_b200 import api, synthetic as syn
+    m, n = dims[:2]
+    iters = args.iters
+    g = syn.normal((m, n), 1.0, seed=44, device="cuda")
+    x = torch.empty_like(g)
+    ws = api.newton_schulz_workspace(m, n)
+    norm = torch.empty(1, dtype=torch.float32, device="cuda")
+
+    def timed(fn, flush_each=True):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            if flush_each:
+                flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    clocks = ClockSampler(0)
+    t_ns = timed(lambda: api.newton_schulz(g, iters, out=x, norm=norm, workspace=ws))
+    clock_info = clocks.stop()
+    xs = x.clone()
+    xr, xc = api.QTensor.empty(m, n), api.QTensor.empty(n, m)
+    r = torch.eye(m, dtype=torch.bfloat16, device="cuda")
+    rr = api.QTensor.empty(m, m)
+    api.quantize(xs, emit_row=True, emit_col=True, out_row=xr, out_col=xc)
+    t_qx = timed(lambda: api.quantize(xs, emit_row=True, emit_col=True, out_row=xr, out_col=xc))
+    t_g1 = timed(lambda: api.gemm(xr, xr, alpha=-1.0, accumulate=True, out=r))
+    api.quantize(r, out_row=rr)
+    t_qr = timed(lambda: api.quantize(r, out_row=rr))
+    t_g2 = timed(lambda: api.gemm(rr, xc, alpha=0.5, accumulate=True, out=xs))
+    api.get_status()
+    step_flops = 4.0 * m * m * n
+    print(json.dumps({
+        "kernel": "ns", "shape": [m, n], "iters": iters, "ms": t_ns, "ms_per_iter": t_ns / max(iters, 1),
+        "value": step_flops * iters / (t_ns * 1e-3) / 1e12, "unit": "TFLOP/s (4 m^2 n per step)",
+        "stages_ms": {"quantize_x_row_col": t_qx, "gemm_x_xt": t_g1,
+                      "quantize_r_row": t_qr, "gemm_r_x": t_g2},
+        "gemm_tflops": {"x_xt": 2.0 * m * m * n / t_g1 / 1e9, "r_x": 2.0 * m * m * n / t_g2 / 1e9},
+        "quantize_gbs": {"x": m * n * 5.125 / t_qx / 1e6, "r": m * m * 4.5625 / t_qr / 1e6},
+        "steps": args.steps, "l2": "flushed (256 MB write) before each timed call", "clocks": clock_info}),
+        flush=True)
+    return 0
+
+
+def run_layer(args):
+    """The four linears of a 3B-class decoder layer at 32768 tokens (QKV 3072->9216, O
+    3072->3072, gate-up 3072->16384, down 8192->3072): forward through the layer, then
+    backward in reverse, every linear with W quantised (2D), fprop, dgrad and wgrad.
+    Timed two ways on one GPU: everything in order on one stream, and each wgrad on a
+    second stream so it can fill the SMs that the next dgrad's quantiser and GEMM leave
+    idle.  Inputs are resident and each larger than L2."""
+    from nvfp4_pretraining_linear_b200 import api, synthetic as syn
+    torch.cuda.set_device(0)
+    names = list(syn.LAYER3B["linears"])
+    linears = [Linear(n, *syn.layer3b_linear(n, device="cuda")) for n in names]
+    flops = sum(L.gemm_flops() for L in linears)
+    side = torch.cuda.Stream()
+
+    def forward(ev):
+        for L in linears:
+            ev.mark("q")
+            api.quantize(L.w, emit_row=True, emit_col=True, block_2d=True, out_row=L.wq_row, out_col=L.wq_col)
+            api.quantize(L.x, emit_row=True, emit_col=True, rht_col=True, rht_signs=RHT_SIGNS, out_row=L.xq_row,
+                         out_col=L.xq_col)
+            ev.mark("g")
+            api.gemm(L.xq_row, L.wq_row, out=L.y)
+
+    def step_in_order(ev):
+        forward(ev)
+        for L in reversed(linears):
+            ev.mark("q")
+            api.quantize(L.dy, emit_row=True, emit_col=True, stochastic=True, rht_col=True, seed=SR_SEED,
+                         rht_signs=RHT_SIGNS, out_row=L.dyq_row, out_col=L.dyq_col)
+            ev.mark("g")
+            api.gemm(L.dyq_row, L.wq_col, out=L.dx)
+            api.gemm(L.dyq_col, L.xq_col, out=L.dw)
+        ev.mark("end")
+
+    def step_side_stream(ev):
+        main = torch.cuda.current_stream()
+        forward(PhaseEvents(False))
+        for L in reversed(linears):
+            api.linear_dgrad(L.dy, L.wq_col, seed=SR_SEED, rht_signs=RHT_SIGNS, out=L.dx, dyq_row=L.dyq_row,
+                             dyq_col=L.dyq_col)
+            ready = torch.cuda.Event()
+            ready.record(main)
+            side.wait_event(ready)
+            api.linear_wgrad(L.dyq_col, L.xq_col, out=L.dw, stream=side)
+        done = torch.cuda.Event()
+        done.record(side)
+        main.wait_event(done)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn(PhaseEvents(False))
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn(PhaseEvents(False))
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    clocks = ClockSampler(0)
+    t_seq = timed(step_in_order)
+    clock_info = clocks.stop()
+    t_side = timed(step_side_stream)
+    ev = PhaseEvents(True)
+    step_in_order(ev)
+    torch.cuda.synchronize()
+    phases = ev.totals()
+    api.get_status()
+    print(json.dumps({
+        "kernel": "layer", "workload": "layer3b-decoder-linears-32768-tokens", "gemm_tflop_per_step": flops / 1e12,
+        "ms_in_order": t_seq, "ms_wgrad_side_stream": t_side, "value": flops / (t_seq * 1e-3) / 1e12,
+        "unit": "TFLOP/s (12 GEMMs, 2MNK each, per step time)", "phase_ms": phases,
+        "gemm_tflops_in_step": flops / (phases.get("g", float("nan")) * 1e-3) / 1e12,
+        "steps": args.steps, "l2": "inputs larger than L2, no flush", "clocks": clock_info}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -603,14 +741,19 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["step", "gemm", "quantize", "chain"], default="step",
+    ap.add_argument("--kernel", choices=["step", "gemm", "quantize", "chain", "ns", "layer"], default="step",
                     help="step: the contract benchmark; gemm/quantize: one kernel on --shape; chain: GEMM then "
-                         "quantise its output, plain against epilogue-fused amax (--shape M,N,K)")
+                         "quantise its output, plain against epilogue-fused amax (--shape M,N,K); ns: NVFP4 "
+                         "Newton-Schulz on a Gaussian --shape m,n for --iters steps; layer: the four linears of a "
+                         "3B decoder layer at 32768 tokens, in order and with wgrad on a side stream")
+    ap.add_argument("--iters", type=int, default=16, help="--kernel ns: Newton-Schulz steps per call")
     ap.add_argument("--shape", default="16384,16384,16384")
     ap.add_argument("--mode", choices=sorted(QUANT_MODES), default="grad")
     ap.add_argument("--amax-in", action="store_true",
                     help="--kernel quantize: given maxima, no amax pass (2 B read + 0.5625 B per layout per element)")
     args = ap.parse_args()
+    if args.kernel == "layer":
+        return run_layer(args)
     if args.kernel != "step":
         return run_kernel(args)
     if args.warmup < 3:

@@ -209,6 +209,46 @@ nvfp4_status nvfp4_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ld
 nvfp4_status nvfp4_linear_wgrad(const nvfp4_tensor* dYq_col, const nvfp4_tensor* Xq_col, void* dW,
                                 int64_t ldw, int32_t out_dtype, int32_t accumulate, void* stream);
 
+/* Bytes of device workspace that nvfp4_newton_schulz needs for an [m x n] matrix
+ * (256-byte aligned; contents need not be initialised): the NVFP4 row and col
+ * layouts of X, the BF16 residual R [m x m] and its row layout, and a few scalars.
+ * 0 for a shape that nvfp4_newton_schulz rejects. */
+size_t nvfp4_newton_schulz_workspace_size(int64_t m, int64_t n);
+
+/* Newton-Schulz orthogonalisation with NVFP4 products.  The optimizer passage of
+ * "Full-Stack FP4: Preentrenamiento Estable de LLM" runs the Newton-Schulz
+ * iterations of the Muon optimizer natively in NVFP4 and gives no coefficients;
+ * this is the coefficient-free cubic iteration for the orthogonal polar factor
+ * (Bjorck and Bowie, SIAM J. Numer. Anal. 8, 1971), X <- 3/2 X - 1/2 X X^T X, in
+ * residual form:
+ *   X_0 = BF16(G / ||G||_F)     (normalize != 0; else X_0 = G)
+ *   repeat iters times:
+ *     Xr, Xc = nvfp4_quantize(X): row layout (blocks along n) and col layout
+ *              (blocks along m), 1D, round-to-nearest-even, no transform
+ *     R      = BF16(I - Xr . Xr^T)            an NVFP4 GEMM adding into I
+ *     Rr     = nvfp4_quantize(R) row layout
+ *     X      = BF16(X + 1/2 Rr . Xc^T)        an NVFP4 GEMM adding into X
+ * Each GEMM that adds into a BF16 matrix rounds as BF16(fl32(fl32(product) + C)).
+ * Singular values of G/||G||_F in (0, 1] converge towards 1; the 4-bit operands
+ * leave them within about 10 % of 1.
+ *   G        : BF16 [m x n] (device, row stride ldg elements).  Pass the wide
+ *              orientation (m <= n): the work is 4 m^2 n FLOP per iteration.
+ *   X        : BF16 [m x n] output (device, row stride ldx); may be G itself when
+ *              ldx == ldg (in place); must not otherwise overlap G.
+ *   iters    : number of iterations, >= 0.
+ *   norm_out : NULL, or one device float receiving ||G||_F (normalize != 0): the
+ *              square root of the FP64 sum of squares, rounded to FP32.
+ *   workspace: nvfp4_newton_schulz_workspace_size(m, n) bytes of device memory,
+ *              256-byte aligned.
+ * Requires m % 128 == 0, n % 128 == 0, ldg and ldx multiples of 8, G and X
+ * 16-byte aligned.  Extends the hot path of the pages (the optimizer step
+ * around the linear layer); enqueues 2 + 7 * iters of this library's kernels
+ * (sum of squares and normalisation; per iteration two quantiser passes over X,
+ * the identity, two over R and the two GEMMs) and small memsets on `stream`. */
+nvfp4_status nvfp4_newton_schulz(const void* G, int64_t m, int64_t n, int64_t ldg, void* X, int64_t ldx,
+                                 int32_t iters, int32_t normalize, float* norm_out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
 /* nvfp4_quantize without a workspace argument, for callers that cannot
  * allocate device memory at the point of the call -- for example a host thread
  * that must not take the allocator's device-wide locks or trigger its implicit

@@ -180,6 +180,34 @@ def linear_wgrad(dyq_col: QTensor, xq_col: QTensor, *, out_dtype=torch.bfloat16,
     return out
 
 
+def newton_schulz_workspace(m, n, device=None):
+    """A device buffer of nvfp4_newton_schulz_workspace_size(m, n) bytes (256-byte aligned)."""
+    nbytes = _lib.load().nvfp4_newton_schulz_workspace_size(m, n)
+    if nbytes == 0:
+        raise NVFP4Error(_lib.NVFP4_ERR_UNSUPPORTED_SHAPE, "no Newton-Schulz workspace for %dx%d" % (m, n))
+    return torch.empty(nbytes, dtype=torch.uint8, device=device if device is not None else "cuda")
+
+
+def newton_schulz(g: torch.Tensor, iters=5, *, normalize=True, out: Optional[torch.Tensor] = None,
+                  norm: Optional[torch.Tensor] = None, workspace=None, stream=None):
+    """nvfp4_newton_schulz on a BF16 [m, n] CUDA tensor: returns (X, ||G||_F as a 1-float
+    device tensor, or None without normalisation).  out may be g itself (in place)."""
+    lib = _lib.load()
+    if g.dtype != torch.bfloat16 or not g.is_cuda or g.dim() != 2 or g.stride(1) != 1:
+        raise ValueError("g must be a 2-D BF16 CUDA tensor with a contiguous last dimension")
+    m, n = g.shape
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=g.device)
+    if normalize and norm is None:
+        norm = torch.empty(1, dtype=torch.float32, device=g.device)
+    if workspace is None:
+        workspace = newton_schulz_workspace(m, n, g.device)
+    _lib.check(lib.nvfp4_newton_schulz(g.data_ptr(), m, n, g.stride(0), out.data_ptr(), out.stride(0), int(iters),
+                                       int(normalize), _ptr(norm) if normalize else None, workspace.data_ptr(),
+                                       workspace.numel(), _stream_ptr(stream)))
+    return out, (norm if normalize else None)
+
+
 def check_conversions(n_sr=1 << 26, stream=None):
     """nvfp4_check_conversions: mismatch counts (E2M1 RNE, E4M3, E2M1 SR) of the hardware
     conversions against their definitions on the current device; all 0 when conforming."""

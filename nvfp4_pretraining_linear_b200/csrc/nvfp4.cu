@@ -2,8 +2,8 @@
 //
 // Host side only: argument validation, tensor-map construction for the GEMM's
 // TMA loads, and kernel launches on the caller's stream.  One translation unit
-// holds every kernel (quantize.cuh, gemm.cuh) so that the module-scope device
-// error word is shared by all of them.
+// holds every kernel (quantize.cuh, gemm.cuh, ns.cuh) so that the module-scope
+// device error word is shared by all of them.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -17,6 +17,7 @@
 #include "nvfp4.h"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "ns.cuh"
 #include "quantize.cuh"
 #include "selfcheck.cuh"
 
@@ -314,7 +315,7 @@ nvfp4_status noalloc_scratch(void** out) {
 
 extern "C" {
 
-int nvfp4_version(void) { return 100; }
+int nvfp4_version(void) { return 200; }
 
 size_t nvfp4_workspace_size(void) { return kWorkspaceBytes; }
 
@@ -589,6 +590,110 @@ nvfp4_status nvfp4_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ld
 nvfp4_status nvfp4_linear_wgrad(const nvfp4_tensor* dYq_col, const nvfp4_tensor* Xq_col, void* dW, int64_t ldw,
                                 int32_t out_dtype, int32_t accumulate, void* stream) {
   return nvfp4_gemm(dYq_col, Xq_col, dW, ldw, out_dtype, 1.0f, accumulate, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace of nvfp4_newton_schulz, each part 256-byte aligned: the quantiser's
+// scratch, the scalars (FP64 sum of squares, three tensor scales), the NVFP4 row
+// and col layouts of X [m x n], the BF16 residual R [m x m] and its row layout.
+struct NsLayout {
+  size_t quant_ws, scalars, xr_codes, xr_scales, xc_codes, xc_scales, r, rr_codes, rr_scales, total;
+};
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+NsLayout ns_layout(int64_t m, int64_t n) {
+  NsLayout L{};
+  size_t o = 0;
+  auto take = [&o](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.quant_ws = take(kWorkspaceBytes);
+  L.scalars = take(64);
+  L.xr_codes = take((size_t)m * (size_t)n / 2);
+  L.xr_scales = take(nvfp4_scales_bytes(m, n, NVFP4_SCALE_MMA));
+  L.xc_codes = take((size_t)n * (size_t)m / 2);
+  L.xc_scales = take(nvfp4_scales_bytes(n, m, NVFP4_SCALE_MMA));
+  L.r = take((size_t)m * (size_t)m * 2);
+  L.rr_codes = take((size_t)m * (size_t)m / 2);
+  L.rr_scales = take(nvfp4_scales_bytes(m, m, NVFP4_SCALE_MMA));
+  L.total = o;
+  return L;
+}
+
+bool ns_shape_ok(int64_t m, int64_t n) {
+  return m > 0 && n > 0 && m % 128 == 0 && n % 128 == 0 && m < (1ll << 30) && n < (1ll << 30);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_newton_schulz_workspace_size(int64_t m, int64_t n) {
+  return ns_shape_ok(m, n) ? ns_layout(m, n).total : 0;
+}
+
+nvfp4_status nvfp4_newton_schulz(const void* G, int64_t m, int64_t n, int64_t ldg, void* X, int64_t ldx, int32_t iters,
+                                 int32_t normalize, float* norm_out, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (!ns_shape_ok(m, n))
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Newton-Schulz needs m, n > 0 and multiples of 128 (got %lld, %lld)",
+                (long long)m, (long long)n);
+  if (!G || !X) return fail(NVFP4_ERR_INVALID_ARG, "G or X is NULL");
+  if (iters < 0) return fail(NVFP4_ERR_INVALID_ARG, "iters %d < 0", iters);
+  if (ldg < n || ldx < n) return fail(NVFP4_ERR_INVALID_ARG, "ldg or ldx < n");
+  if (!aligned16(G) || !aligned16(X) || ldg % 8 || ldx % 8)
+    return fail(NVFP4_ERR_MISALIGNED, "G and X rows must be 16-byte aligned");
+  if (G == X && ldg != ldx) return fail(NVFP4_ERR_INVALID_ARG, "in-place use needs ldg == ldx");
+  if (norm_out && reinterpret_cast<uintptr_t>(norm_out) % 4) return fail(NVFP4_ERR_MISALIGNED, "norm_out alignment");
+  const NsLayout L = ns_layout(m, n);
+  if (!workspace || workspace_bytes < L.total)
+    return fail(NVFP4_ERR_WORKSPACE, "Newton-Schulz needs %zu bytes of workspace", L.total);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(NVFP4_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+  DeviceInfo* dev;
+  nvfp4_status st = device_info(&dev);
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  double* ssq = reinterpret_cast<double*>(ws + L.scalars);
+  float* scales = reinterpret_cast<float*>(ws + L.scalars + 16);
+  uint16_t* x = static_cast<uint16_t*>(X);
+  uint16_t* r = reinterpret_cast<uint16_t*>(ws + L.r);
+  nvfp4_tensor xr{ws + L.xr_codes, ws + L.xr_scales, scales + 0, m, n, NVFP4_SCALE_MMA, 0};
+  nvfp4_tensor xc{ws + L.xc_codes, ws + L.xc_scales, scales + 1, n, m, NVFP4_SCALE_MMA, 0};
+  nvfp4_tensor rr{ws + L.rr_codes, ws + L.rr_scales, scales + 2, m, m, NVFP4_SCALE_MMA, 0};
+  const int grid_x = (int)std::min<int64_t>(m, (int64_t)dev->sm_count * 8);
+  cudaError_t e;
+  if (normalize) {
+    e = cudaMemsetAsync(ssq, 0, sizeof(double), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(sum of squares)");
+    nvfp4::ns::sumsq_kernel<<<grid_x, nvfp4::ns::kThreads, 0, s>>>(static_cast<const uint16_t*>(G), m, n, ldg, ssq);
+    nvfp4::ns::normalize_kernel<<<grid_x, nvfp4::ns::kThreads, 0, s>>>(static_cast<const uint16_t*>(G), ldg, x, ldx, m,
+                                                                        n, ssq, norm_out);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "normalisation launch");
+  } else if (G != X) {
+    e = cudaMemcpy2DAsync(X, (size_t)ldx * 2, G, (size_t)ldg * 2, (size_t)n * 2, (size_t)m, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy2DAsync(G -> X)");
+  }
+  const nvfp4_quant_opts rne{};
+  void* qws = ws + L.quant_ws;
+  const int grid_r = (int)std::min<int64_t>(m, (int64_t)dev->sm_count * 8);
+  for (int32_t it = 0; it < iters; ++it) {
+    if ((st = nvfp4_quantize(X, m, n, ldx, &rne, &xr, &xc, qws, kWorkspaceBytes, stream)) != NVFP4_OK) return st;
+    nvfp4::ns::identity_kernel<<<grid_r, nvfp4::ns::kThreads, 0, s>>>(r, m, m);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "identity launch");
+    if ((st = gemm_impl(&xr, &xr, r, m, NVFP4_OUT_BF16, -1.0f, 1, nullptr, 0u, stream)) != NVFP4_OK) return st;
+    if ((st = nvfp4_quantize(r, m, m, m, &rne, &rr, nullptr, qws, kWorkspaceBytes, stream)) != NVFP4_OK) return st;
+    if ((st = gemm_impl(&rr, &xc, X, ldx, NVFP4_OUT_BF16, 0.5f, 1, nullptr, 0u, stream)) != NVFP4_OK) return st;
+  }
+  return NVFP4_OK;
 }
 
 nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,

@@ -15,6 +15,9 @@ NVFP4 pretraining summary, plus a tiny case and a quantiser sweep):
             W_down [5120 x 20480] ~ N(0,0.014); X [16384 x 5120] and the
             down-projection input [16384 x 20480] ~ N(0,1) with 0.1 % x100
             outliers; dY ~ N(0,1e-3); seeds 10..
+  spectrum  [m x n] = U diag(sigma) V^T with orthonormal U, V from seeded
+            Gaussians and sigma evenly spaced in [smin, smax] (Newton-Schulz
+            inputs with a known polar factor)
   layer3b   32768 tokens: QKV 3072->9216, O 3072->3072, gate-up 3072->16384,
             down 8192->3072 (weights N(0,0.02), activations N(0,1), dY
             N(0,1e-3)); seeds 20..; square GEMMs n^3, n in 4096..32768, seeds 30+i
@@ -96,3 +99,12 @@ def layer3b_linear(name, device="cpu"):
 
 def square(n, i=0, device="cpu"):
     return normal((n, n), 1.0, seed=30 + 2 * i, device=device), normal((n, n), 1.0, seed=31 + 2 * i, device=device)
+
+
+def spectrum(m, n, smin=0.1, smax=1.0, seed=0, device="cpu"):
+    """[m x n], m <= n: U diag(sigma) V^T with sigma evenly spaced in [smin, smax]."""
+    g = _gen(seed, "cpu")
+    u, _ = torch.linalg.qr(torch.randn((m, m), generator=g, dtype=torch.float64))
+    v, _ = torch.linalg.qr(torch.randn((n, m), generator=g, dtype=torch.float64))
+    sigma = torch.linspace(smin, smax, m, dtype=torch.float64)
+    return ((u * sigma) @ v.T).to(torch.float32).to(torch.bfloat16).to(device)

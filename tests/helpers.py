@@ -60,3 +60,22 @@ def gemm_check(c_gpu: np.ndarray, a_hat, b_hat, alpha=1.0, c0=None, bf16=False):
     err = np.abs(c_gpu.astype(np.float64) - ref)
     ratio = float((err / bound).max()) if err.size else 0.0
     return ratio
+
+
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
+
+
+def exact_operand(rows, cols, seed, device="cuda"):
+    """A BF16 matrix that NVFP4 holds exactly: values code * u, u per 16-block in
+    {1/8, 1/4, 1/2}, one block per tensor at u = 7/8 holding +-5.25, every block holding
+    a +-6 code.  The tensor scale is then 2^-9 and every block scale a power of two or
+    448, so dequantisation returns the input and products of such matrices have few
+    significant bits.  Returns (BF16 tensor on device, float32 numpy values)."""
+    rng = np.random.default_rng(seed)
+    v = E2M1_GRID[rng.integers(0, 8, (rows, cols))] * rng.choice([-1.0, 1.0], (rows, cols))
+    blocks = v.reshape(rows, cols // 16, 16)
+    blocks[:, :, 0] = 6.0 * rng.choice([-1.0, 1.0], (rows, cols // 16))      # every block max is 6u
+    u = rng.choice([0.125, 0.25, 0.5], (rows, cols // 16))
+    u[rng.integers(0, rows), rng.integers(0, cols // 16)] = 0.875              # tensor amax 5.25 -> S = 2^-9
+    x = (blocks * u[:, :, None]).reshape(rows, cols)
+    return torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).to(device), x.astype(np.float32)

@@ -104,3 +104,29 @@ def test_dequantize_argument_errors(lib):
     assert lib.nvfp4_dequantize(ctypes.byref(q), None, 48, 1, None) == 1
     assert lib.nvfp4_dequantize(ctypes.byref(q), 0x1000, 40, 1, None) == 1
     assert lib.nvfp4_dequantize(ctypes.byref(q), 0x1008, 48, 1, None) == 3
+
+
+def test_newton_schulz_workspace_and_argument_errors(lib):
+    m, n = 256, 512
+    need = lib.nvfp4_newton_schulz_workspace_size(m, n)
+    parts = (m * n // 2 + m * n // 16) * 2 + m * m * 2 + m * m // 2 + m * m // 16      # X row+col, R, R row
+    assert parts <= need <= parts + 16 * 256
+    assert lib.nvfp4_newton_schulz_workspace_size(200, 512) == 0
+    assert lib.nvfp4_newton_schulz_workspace_size(256, 0) == 0
+    g, x, ws = 0x100000, 0x200000, 0x300000
+
+    def call(*, g=g, m=m, n=n, ldg=n, x=x, ldx=n, iters=1, ws=ws, wsb=need, norm=None):
+        return lib.nvfp4_newton_schulz(g, m, n, ldg, x, ldx, iters, 1, norm, ws, wsb, None)
+
+    assert call(m=192) == 2                     # m % 128
+    assert call(n=320) == 2                     # n % 128
+    assert call(g=None) == 1
+    assert call(iters=-1) == 1
+    assert call(ldx=n - 8) == 1
+    assert call(x=0x200008) == 3                # X not 16-byte aligned
+    assert call(ldg=n + 4) == 3                 # row stride not 16 bytes
+    assert call(x=g, ldx=n + 8) == 1            # in place with different strides
+    assert call(norm=0x400002) == 3
+    assert call(wsb=need - 1) == 6
+    assert call(ws=0x300010) == 3               # workspace not 256-byte aligned
+    assert "workspace" in lib.nvfp4_last_error_string().decode()

@@ -16,23 +16,11 @@ import torch
 
 from nvfp4_pretraining_linear_b200 import api, synthetic
 from oracle import nvfp4_oracle as O
-from tests.helpers import assert_layout_equal, bf16_to_np
+from tests.helpers import assert_layout_equal, bf16_to_np, exact_operand
 
 pytestmark = pytest.mark.gpu
 
-GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
 SIGNS = 0x5A3C
-
-
-def exact_operand(rows, cols, seed):
-    rng = np.random.default_rng(seed)
-    v = GRID[rng.integers(0, 8, (rows, cols))] * rng.choice([-1.0, 1.0], (rows, cols))
-    blocks = v.reshape(rows, cols // 16, 16)
-    blocks[:, :, 0] = 6.0 * rng.choice([-1.0, 1.0], (rows, cols // 16))      # every block max is 6u
-    u = rng.choice([0.125, 0.25, 0.5], (rows, cols // 16))
-    u[rng.integers(0, rows), rng.integers(0, cols // 16)] = 0.875              # tensor amax 5.25 -> S = 2^-9
-    x = (blocks * u[:, :, None]).reshape(rows, cols)
-    return torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).cuda(), x.astype(np.float32)
 
 
 @pytest.mark.parametrize("M,N,K", [(256, 256, 256), (512, 384, 512), (768, 640, 1024)])
