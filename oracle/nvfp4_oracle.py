@@ -82,6 +82,18 @@ stated where it is used:
     the exactly rounded FP64 sum of squares, then rounded to FP32.  A product that
     adds into a BF16 matrix C rounds as C <- BF16(fl32(fl32(alpha * sum) + C)), the
     sum taken exactly and rounded once to FP32.
+12. LoRA-SVD linear.  [Full-Stack FP4] splits each linear projection's weight with a
+    light LoRA-SVD decomposition so that 4-bit quantisation noise falls on a smaller
+    residual; it gives neither the rank nor how the factors are refreshed.  Reading:
+    W = W_res + L R with caller-supplied BF16 factors L [N x r], R [r x K] (e.g. the
+    top-r singular triplets of W), W_res = BF16(fl32(W - s)) where s accumulates
+    L[n, j] R[j, k] in FP32 over j = 0, 1, ... (each product of BF16 values exact).
+    W_res takes the NVFP4 path of the linear layer (2D blocks); the low-rank part
+    stays in BF16:  Y = BF16(fl32(Y4 + V)) with Y4 = BF16(Q(X) Q(W_res)^T) and
+    V = fl32((BF16(X R^T)) L^T);  dX = BF16(fl32(dX4 + V')) with dX4 the NVFP4
+    dgrad against W_res and V' = fl32((BF16(dY L)) R).  The weight gradient is that
+    of W itself (the NVFP4 wgrad, unchanged).  Products of the low-rank branch are
+    taken exactly and rounded once (the hardware accumulates in FP32).
 """
 
 from __future__ import annotations
@@ -560,3 +572,60 @@ def newton_schulz(g: np.ndarray, iters: int, normalize: bool = True):
     for _ in range(iters):
         x, _ = ns_step(x)
     return x, nrm
+
+
+# ---------------------------------------------------------------------------
+# LoRA-SVD linear: NVFP4 residual weight plus a BF16 low-rank branch (reading 12)
+# ---------------------------------------------------------------------------
+
+
+def lora_residual(w: np.ndarray, l: np.ndarray, r: np.ndarray) -> np.ndarray:
+    """W_res = BF16(fl32(W - s)), s = sum_j L[:, j] R[j, :] accumulated in FP32 in order."""
+    w = np.asarray(w, dtype=F32)
+    l = np.asarray(l, dtype=F32)
+    r = np.asarray(r, dtype=F32)
+    s = np.zeros(w.shape, dtype=F32)
+    for j in range(l.shape[1]):
+        s = (s + (l[:, j:j + 1] * r[j:j + 1, :]).astype(F32)).astype(F32)
+    return bf16_round((w - s).astype(F32))
+
+
+def lora_project(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """U = BF16(A B^T): A [M x K], B [r x K]; exact sum rounded to FP32, then to BF16."""
+    return bf16_round(gemm_ref(a, b).astype(F32))
+
+
+def lora_expand_add(y: np.ndarray, u: np.ndarray, c: np.ndarray) -> np.ndarray:
+    """Y <- BF16(fl32(Y + fl32(U C^T))): Y [M x N] BF16, U [M x r], C [N x r]."""
+    return add_product_bf16(gemm_ref(u, c), y)
+
+
+def lora_linear_fwd(x: np.ndarray, w_res_q: dict, l: np.ndarray, r: np.ndarray, rht_signs: int = 0,
+                    quantize_operands: bool = True):
+    """Y = BF16(fl32(Y4 + fl32(U L^T))), U = BF16(X R^T), Y4 = BF16(Q(X) Q(W_res)^T).
+
+    w_res_q is quantize_weight(W_res); with quantize_operands=False it is W_res itself
+    and Y4 uses the unquantised values (the identity check of the decomposition)."""
+    x = np.asarray(x, dtype=F32)
+    if quantize_operands:
+        y4_exact, (a_hat, b_hat), xq = linear_fwd_ref(x, w_res_q, rht_signs=rht_signs)
+    else:
+        y4_exact, (a_hat, b_hat), xq = gemm_ref(x, w_res_q), (x, w_res_q), None
+    y4 = bf16_round(y4_exact.astype(F32))
+    u = lora_project(x, r)
+    return lora_expand_add(y4, u, l), {"y4": y4, "y4_exact": y4_exact, "u": u, "a_hat": a_hat,
+                                       "b_hat": b_hat, "xq": xq}
+
+
+def lora_linear_dgrad(dy: np.ndarray, w_res_q: dict, l: np.ndarray, r: np.ndarray, seed: int, offset: int,
+                      rht_signs: int = 0, quantize_operands: bool = True):
+    """dX = BF16(fl32(dX4 + fl32(U' R))), U' = BF16(dY L), dX4 = BF16(Q_sr(dY) Q(W_res))."""
+    dy = np.asarray(dy, dtype=F32)
+    if quantize_operands:
+        dx4_exact, (a_hat, b_hat), dyq = linear_dgrad_ref(dy, w_res_q, seed, offset, rht_signs=rht_signs)
+    else:
+        dx4_exact, (a_hat, b_hat), dyq = gemm_ref(dy, np.asarray(w_res_q, dtype=F32).T), (dy, None), None
+    dx4 = bf16_round(dx4_exact.astype(F32))
+    u = lora_project(dy, np.asarray(l, dtype=F32).T)
+    return lora_expand_add(dx4, u, np.asarray(r, dtype=F32).T), {"dx4": dx4, "dx4_exact": dx4_exact, "u": u,
+                                                                  "a_hat": a_hat, "b_hat": b_hat, "dyq": dyq}
