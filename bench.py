@@ -503,6 +503,8 @@ def run_kernel(args):
         return run_chain(args, dims, flush)
     if args.kernel == "ns":
         return run_ns(args, dims, flush)
+    if args.kernel == "lora":
+        return run_lora(args, dims, flush)
     if args.kernel == "gemm":
         M, N, K = dims
         qa, _ = api.quantize(syn.normal((M, K), 1.0, seed=30, device="cuda"))
@@ -652,6 +654,63 @@ def run_ns(args, dims, flush):
     return 0
 
 
+def run_lora(args, dims, flush):
+    """The LoRA-SVD linear against the plain NVFP4 linear on one layer shape (M tokens,
+    N outputs, K inputs, --rank): fprop and dgrad each way, and the low-rank kernels
+    alone (residual, projection, expansion), L2 flushed before each timed call."""
+    from nvfp4_pretraining_linear_b200 import api, synthetic as syn
+    M, N, K = dims
+    rank = args.rank
+    x = syn.normal((M, K), 1.0, seed=12, device="cuda", outlier_frac=0.001, outlier_mult=100.0)
+    w = syn.normal((N, K), 0.014, seed=10, device="cuda")
+    dy = syn.normal((M, N), 1e-3, seed=14, device="cuda")
+    l = syn.normal((N, rank), 0.05, seed=15, device="cuda")
+    r = syn.normal((rank, K), 0.05, seed=16, device="cuda")
+    w_res = api.lora_residual(w, l, r)
+    wq_row, wq_col = api.quantize_weight(w_res)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    u = torch.empty((M, rank), dtype=torch.bfloat16, device="cuda")
+    xr, xc = api.QTensor.empty(M, K), api.QTensor.empty(K, M)
+    dr, dc = api.QTensor.empty(M, N), api.QTensor.empty(N, M)
+    fkw = dict(rht_signs=RHT_SIGNS, out=y, xq_row=xr, xq_col=xc)
+    dkw = dict(seed=SR_SEED, rht_signs=RHT_SIGNS, out=dx, dyq_row=dr, dyq_col=dc)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    res = {
+        "fwd_plain_ms": timed(lambda: api.linear_fwd(x, wq_row, **fkw)),
+        "fwd_lora_ms": timed(lambda: api.lora_linear_fwd(x, wq_row, l, r, u=u, **fkw)),
+        "dgrad_plain_ms": timed(lambda: api.linear_dgrad(dy, wq_col, **dkw)),
+        "dgrad_lora_ms": timed(lambda: api.lora_linear_dgrad(dy, wq_col, l, r, u=u, **dkw)),
+        "residual_ms": timed(lambda: api.lora_residual(w, l, r, out=w_res)),
+        "project_ms": timed(lambda: api.lowrank_project(x, r, out=u)),
+        "expand_ms": timed(lambda: api.lowrank_expand_add(y, u, l)),
+    }
+    api.get_status()
+    res["project_gbs"] = (2.0 * M * K + 2.0 * M * rank) / res["project_ms"] / 1e6
+    res["expand_gbs"] = 4.0 * M * N / res["expand_ms"] / 1e6
+    res["residual_gbs"] = 4.0 * N * K / res["residual_ms"] / 1e6
+    res["fwd_overhead"] = res["fwd_lora_ms"] / res["fwd_plain_ms"] - 1.0
+    res["dgrad_overhead"] = res["dgrad_lora_ms"] / res["dgrad_plain_ms"] - 1.0
+    print(json.dumps({"kernel": "lora", "shape": dims, "rank": rank, **res, "steps": args.steps,
+                      "l2": "flushed (256 MB write)"}), flush=True)
+    return 0
+
+
 def run_layer(args):
     """The four linears of a 3B-class decoder layer at 32768 tokens (QKV 3072->9216, O
     3072->3072, gate-up 3072->16384, down 8192->3072): forward through the layer, then
@@ -741,12 +800,15 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["step", "gemm", "quantize", "chain", "ns", "layer"], default="step",
+    ap.add_argument("--kernel", choices=["step", "gemm", "quantize", "chain", "ns", "layer", "lora"],
+                    default="step",
                     help="step: the contract benchmark; gemm/quantize: one kernel on --shape; chain: GEMM then "
                          "quantise its output, plain against epilogue-fused amax (--shape M,N,K); ns: NVFP4 "
                          "Newton-Schulz on a Gaussian --shape m,n for --iters steps; layer: the four linears of a "
-                         "3B decoder layer at 32768 tokens, in order and with wgrad on a side stream")
+                         "3B decoder layer at 32768 tokens, in order and with wgrad on a side stream; lora: the LoRA-SVD "
+                         "linear against the plain one (--shape M,N,K, --rank)")
     ap.add_argument("--iters", type=int, default=16, help="--kernel ns: Newton-Schulz steps per call")
+    ap.add_argument("--rank", type=int, default=32, help="--kernel lora: rank of the BF16 branch")
     ap.add_argument("--shape", default="16384,16384,16384")
     ap.add_argument("--mode", choices=sorted(QUANT_MODES), default="grad")
     ap.add_argument("--amax-in", action="store_true",

@@ -249,6 +249,59 @@ nvfp4_status nvfp4_newton_schulz(const void* G, int64_t m, int64_t n, int64_t ld
                                  int32_t iters, int32_t normalize, float* norm_out, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/* ---- LoRA-SVD linear.  "Full-Stack FP4: Preentrenamiento Estable de LLM" (linear-
+ * projection passage) splits each projection's weight with a light LoRA-SVD
+ * decomposition, W = W_res + L R, so that 4-bit quantisation noise falls on the
+ * residual; the page gives neither the rank nor the refresh of the factors, so
+ * L [N x r] and R [r x K] (BF16, e.g. the top-r singular triplets of W) are the
+ * caller's.  The residual takes the NVFP4 path (2D weight blocks); the rank-r part
+ * stays in BF16 on the tensor cores (warp-level m16n8k16 MMA, FP32 accumulation).
+ * Every call here takes r in {16, 32, 48, 64}. */
+
+/* W_res = BF16(fl32(W - s)), s = sum_j L[n][j] R[j][k] accumulated in FP32 in
+ * increasing j (each product of BF16 values is exact in FP32 barring underflow).
+ * W, W_res [N x K], L [N x r], R [r x K]: BF16 device matrices with row strides
+ * ldw, ldo, ldl, ldr (elements).  Requires K % 8 == 0, W, R, W_res 16-byte aligned
+ * with ldw, ldr, ldo multiples of 8.  Quantise W_res with 2D blocks for the
+ * linear calls below. */
+nvfp4_status nvfp4_lora_residual(const void* W, int64_t N, int64_t K, int64_t ldw, const void* L, int64_t ldl,
+                                 const void* R, int64_t ldr, int32_t rank, void* W_res, int64_t ldo,
+                                 void* stream);
+
+/* U = BF16(A B^T): A [M x K] BF16 (row stride lda); B [r x K] (b_trans == 0, row
+ * stride ldb) or given as its transpose [K x r] (b_trans != 0, row stride ldb);
+ * U [M x r] BF16 (row stride ldu).  FP32 accumulation, one rounding to BF16.
+ * Requires M % 64 == 0, K a positive multiple of 64, 16-byte aligned rows. */
+nvfp4_status nvfp4_lowrank_project(const void* A, int64_t M, int64_t K, int64_t lda, const void* B, int64_t ldb,
+                                   int32_t b_trans, int32_t rank, void* U, int64_t ldu, void* stream);
+
+/* Y <- BF16(fl32(Y + U C^T)) in place: Y [M x N] BF16 (row stride ldy); U [M x r];
+ * C [N x r] (c_trans == 0, row stride ldc) or given as its transpose [r x N]
+ * (c_trans != 0).  FP32 accumulation of the product.  Requires M % 128 == 0,
+ * N % 128 == 0, 16-byte aligned rows. */
+nvfp4_status nvfp4_lowrank_expand_add(void* Y, int64_t M, int64_t N, int64_t ldy, const void* U, int64_t ldu,
+                                      const void* C, int64_t ldc, int32_t c_trans, int32_t rank, void* stream);
+
+/* LoRA-SVD fprop: Y = BF16(fl32(Y4 + U L^T)) with Y4 = nvfp4_linear_fwd(X, Wq_res_row)
+ * (BF16) and U = BF16(X R^T).  Arguments as nvfp4_linear_fwd, plus L [N x r] and
+ * R [r x K] contiguous BF16 device matrices and U, caller scratch of M * r BF16
+ * (16-byte aligned).  Y is BF16.  Work: the NVFP4 fprop, then one pass over X for U
+ * and one read-modify-write pass over Y. */
+nvfp4_status nvfp4_lora_linear_fwd(const void* X, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* Wq_res_row,
+                                   const void* L, const void* R, int32_t rank, void* Y, int64_t ldy,
+                                   nvfp4_tensor* Xq_row, nvfp4_tensor* Xq_col, uint32_t rht_signs, void* U,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* LoRA-SVD dgrad: dX = BF16(fl32(dX4 + U R)) with dX4 = nvfp4_linear_dgrad(dY,
+ * Wq_res_col) (BF16) and U = BF16(dY L).  Arguments as nvfp4_linear_dgrad, plus L,
+ * R and U as for nvfp4_lora_linear_fwd.  The weight gradient is that of W itself:
+ * nvfp4_linear_wgrad, unchanged. */
+nvfp4_status nvfp4_lora_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ldy, const nvfp4_tensor* Wq_res_col,
+                                     const void* L, const void* R, int32_t rank, void* dX, int64_t ldx,
+                                     nvfp4_tensor* dYq_row, nvfp4_tensor* dYq_col, uint64_t seed, uint64_t offset,
+                                     uint32_t rht_signs, void* U, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
 /* nvfp4_quantize without a workspace argument, for callers that cannot
  * allocate device memory at the point of the call -- for example a host thread
  * that must not take the allocator's device-wide locks or trigger its implicit

@@ -83,6 +83,18 @@ SIGNATURES = {
     "nvfp4_newton_schulz_workspace_size": (c_size_t, [c_int64, c_int64]),
     "nvfp4_newton_schulz": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_int32, c_int32,
                                       c_void_p, c_void_p, c_size_t, c_void_p]),
+    "nvfp4_lora_residual": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_void_p, c_int64,
+                                      c_int32, c_void_p, c_int64, c_void_p]),
+    "nvfp4_lowrank_project": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_int32, c_int32,
+                                        c_void_p, c_int64, c_void_p]),
+    "nvfp4_lowrank_expand_add": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_void_p, c_int64,
+                                           c_int32, c_int32, c_void_p]),
+    "nvfp4_lora_linear_fwd": (c_int32, [c_void_p, c_int64, c_int64, c_int64, T_P, c_void_p, c_void_p, c_int32,
+                                        c_void_p, c_int64, T_P, T_P, c_uint32, c_void_p, c_void_p, c_size_t,
+                                        c_void_p]),
+    "nvfp4_lora_linear_dgrad": (c_int32, [c_void_p, c_int64, c_int64, c_int64, T_P, c_void_p, c_void_p, c_int32,
+                                          c_void_p, c_int64, T_P, T_P, c_uint64, c_uint64, c_uint32, c_void_p,
+                                          c_void_p, c_size_t, c_void_p]),
     "nvfp4_quantize_noalloc": (c_int32, [c_void_p, c_int64, c_int64, c_int64, O_P, T_P, T_P, c_void_p]),
     "nvfp4_check_conversions": (c_int32, [c_void_p, c_uint64, c_void_p]),
     "nvfp4_get_status": (c_int32, [c_void_p]),

@@ -208,6 +208,102 @@ def newton_schulz(g: torch.Tensor, iters=5, *, normalize=True, out: Optional[tor
     return out, (norm if normalize else None)
 
 
+def _bf16_matrix(t, name):
+    if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("%s must be a 2-D BF16 CUDA tensor with a contiguous last dimension" % name)
+
+
+def lora_residual(w: torch.Tensor, l: torch.Tensor, r: torch.Tensor, out: Optional[torch.Tensor] = None,
+                  stream=None):
+    """nvfp4_lora_residual: W_res = BF16(W - L R) (FP32 accumulation over the rank, in order)."""
+    lib = _lib.load()
+    for t, nm in ((w, "w"), (l, "l"), (r, "r")):
+        _bf16_matrix(t, nm)
+    N, K = w.shape
+    rank = l.shape[1]
+    if out is None:
+        out = torch.empty_like(w)
+    _lib.check(lib.nvfp4_lora_residual(w.data_ptr(), N, K, w.stride(0), l.data_ptr(), l.stride(0), r.data_ptr(),
+                                       r.stride(0), rank, out.data_ptr(), out.stride(0), _stream_ptr(stream)))
+    return out
+
+
+def lowrank_project(a: torch.Tensor, b: torch.Tensor, *, b_trans=False, out: Optional[torch.Tensor] = None,
+                    stream=None):
+    """nvfp4_lowrank_project: U = BF16(A B^T), B [r, K] (or its transpose [K, r] with b_trans)."""
+    lib = _lib.load()
+    _bf16_matrix(a, "a")
+    _bf16_matrix(b, "b")
+    M, K = a.shape
+    rank = b.shape[1] if b_trans else b.shape[0]
+    if out is None:
+        out = torch.empty((M, rank), dtype=torch.bfloat16, device=a.device)
+    _lib.check(lib.nvfp4_lowrank_project(a.data_ptr(), M, K, a.stride(0), b.data_ptr(), b.stride(0), int(b_trans),
+                                         rank, out.data_ptr(), out.stride(0), _stream_ptr(stream)))
+    return out
+
+
+def lowrank_expand_add(y: torch.Tensor, u: torch.Tensor, c: torch.Tensor, *, c_trans=False, stream=None):
+    """nvfp4_lowrank_expand_add: Y <- BF16(Y + U C^T) in place, C [N, r] (or [r, N] with c_trans)."""
+    lib = _lib.load()
+    for t, nm in ((y, "y"), (u, "u"), (c, "c")):
+        _bf16_matrix(t, nm)
+    M, N = y.shape
+    rank = u.shape[1]
+    _lib.check(lib.nvfp4_lowrank_expand_add(y.data_ptr(), M, N, y.stride(0), u.data_ptr(), u.stride(0), c.data_ptr(),
+                                            c.stride(0), int(c_trans), rank, _stream_ptr(stream)))
+    return y
+
+
+def lora_linear_fwd(x: torch.Tensor, wq_res_row: QTensor, l: torch.Tensor, r: torch.Tensor, *, save_col=True,
+                    rht_signs=0, out=None, u=None, xq_row=None, xq_col=None, stream=None):
+    """nvfp4_lora_linear_fwd: Y = BF16(Q(X) Q(W_res)^T + BF16(X R^T) L^T); returns
+    (Y, Xq_row, Xq_col or None).  l [N, r] and r [r, K] contiguous."""
+    lib = _lib.load()
+    M, K = x.shape
+    N = wq_res_row.rows
+    rank = l.shape[1]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if u is None:
+        u = torch.empty((M, rank), dtype=torch.bfloat16, device=x.device)
+    if xq_row is None:
+        xq_row = QTensor.empty(M, K, SCALE_MMA, x.device)
+    if save_col and xq_col is None:
+        xq_col = QTensor.empty(K, M, SCALE_MMA, x.device)
+    ws = workspace(x.device, stream)
+    xc = xq_col.struct() if save_col else None
+    _lib.check(lib.nvfp4_lora_linear_fwd(x.data_ptr(), M, K, x.stride(0), wq_res_row.struct(), l.data_ptr(),
+                                         r.data_ptr(), rank, out.data_ptr(), out.stride(0), xq_row.struct(), xc,
+                                         rht_signs, u.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
+    return out, xq_row, (xq_col if save_col else None)
+
+
+def lora_linear_dgrad(dy: torch.Tensor, wq_res_col: QTensor, l: torch.Tensor, r: torch.Tensor, *, seed, offset=0,
+                      save_col=True, rht_signs=0, out=None, u=None, dyq_row=None, dyq_col=None, stream=None):
+    """nvfp4_lora_linear_dgrad: dX = BF16(Q_sr(dY) Q(W_res) + BF16(dY L) R); returns
+    (dX, dYq_row, dYq_col or None)."""
+    lib = _lib.load()
+    M, N = dy.shape
+    K = wq_res_col.rows
+    rank = l.shape[1]
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.bfloat16, device=dy.device)
+    if u is None:
+        u = torch.empty((M, rank), dtype=torch.bfloat16, device=dy.device)
+    if dyq_row is None:
+        dyq_row = QTensor.empty(M, N, SCALE_MMA, dy.device)
+    if save_col and dyq_col is None:
+        dyq_col = QTensor.empty(N, M, SCALE_MMA, dy.device)
+    ws = workspace(dy.device, stream)
+    dc = dyq_col.struct() if save_col else None
+    _lib.check(lib.nvfp4_lora_linear_dgrad(dy.data_ptr(), M, N, dy.stride(0), wq_res_col.struct(), l.data_ptr(),
+                                           r.data_ptr(), rank, out.data_ptr(), out.stride(0), dyq_row.struct(), dc,
+                                           seed, offset, rht_signs, u.data_ptr(), ws.data_ptr(), ws.numel(),
+                                           _stream_ptr(stream)))
+    return out, dyq_row, (dyq_col if save_col else None)
+
+
 def check_conversions(n_sr=1 << 26, stream=None):
     """nvfp4_check_conversions: mismatch counts (E2M1 RNE, E4M3, E2M1 SR) of the hardware
     conversions against their definitions on the current device; all 0 when conforming."""

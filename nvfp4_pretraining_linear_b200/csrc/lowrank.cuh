@@ -1,0 +1,303 @@
+// Kernels of the LoRA-SVD linear (nvfp4_lora_*): the weight is split as
+// W = W_res + L R so that NVFP4 quantisation noise falls on the residual, and the
+// rank-r part runs in BF16 ("Full-Stack FP4: Preentrenamiento Estable de LLM",
+// linear-projection passage: a light LoRA-SVD decomposition that lowers the
+// quantisation error of direct 4-bit quantisation).
+//
+//   lora_residual_kernel   W_res = BF16(fl32(W - s)), s = sum_j L[n][j] R[j][k]
+//                          accumulated in FP32 in increasing j (each product of two
+//                          BF16 values is exact in FP32, so a fused multiply-add
+//                          rounds exactly as the separate product and sum would).
+//   lowrank_project_kernel U = BF16(A B^T), A [M x K] BF16, B [r x K] (or given as
+//                          [K x r]); HBM-bound on A.
+//   lowrank_expand_kernel  Y = BF16(fl32(Y + U C^T)), U [M x r], C [N x r] (or given
+//                          as [r x N]); HBM-bound on the read-modify-write of Y.
+//
+// The two products are dense contractions with a short side (r <= 64), so they run
+// on the warp-level BF16 tensor-core MMA (m16n8k16, FP32 accumulation) from shared
+// memory; the tiles are small and the work is bound by streaming A or Y, not by the
+// MMA rate.
+#pragma once
+
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace lowrank {
+
+constexpr int kMaxRank = 64;
+constexpr int kResidualThreads = 256;
+constexpr int kResRows = 4;            // rows of W per residual thread
+constexpr int kProjRows = 64;          // rows of A per CTA (4 warps x 16)
+constexpr int kProjThreads = 128;
+constexpr int kProjKc = 64;            // K per pipeline stage
+constexpr int kProjStages = 4;
+constexpr int kPad = 72;               // shared row stride in BF16 elements (144 B, conflict-free)
+constexpr int kProjSmemBytes = kProjStages * (kProjRows + kMaxRank) * kPad * 2;
+constexpr int kExpTile = 128;          // Y tile 128 x 128 per CTA
+constexpr int kExpThreads = 256;
+constexpr int kAccStride = 132;        // FP32 row stride of the staged accumulator tile
+constexpr int kExpSmemBytes = 2 * kExpTile * kPad * 2 + kExpTile * kAccStride * 4;
+
+// One warp-level BF16 MMA: d += a(16x16, row) * b(16x8, col), FP32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_pending() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// ------------------------------------------------------------------ residual
+
+// A thread computes 8 consecutive columns k of kResRows consecutive rows n, so each
+// 16-byte load of R serves kResRows rows (row groups grid-stride over blockIdx.y).
+// The products are exact barring FP32 underflow (BF16 factors below about 1e-19).
+__global__ void __launch_bounds__(kResidualThreads) lora_residual_kernel(
+    const uint16_t* __restrict__ w, int64_t ldw, const uint16_t* __restrict__ l, int64_t ldl,
+    const uint16_t* __restrict__ r, int64_t ldr, uint16_t* __restrict__ out, int64_t ldo, int64_t N, int64_t K,
+    int rank) {
+  const int64_t k0 = ((int64_t)blockIdx.x * kResidualThreads + threadIdx.x) * 8;
+  if (k0 >= K) return;
+  for (int64_t n0 = (int64_t)blockIdx.y * kResRows; n0 < N; n0 += (int64_t)gridDim.y * kResRows) {
+    float s[kResRows][8];
+#pragma unroll
+    for (int i = 0; i < kResRows; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s[i][e] = 0.f;
+    for (int j = 0; j < rank; ++j) {
+      const uint4 rv = *reinterpret_cast<const uint4*>(r + (int64_t)j * ldr + k0);
+      const float rf[8] = {bf16_lo(rv.x), bf16_hi(rv.x), bf16_lo(rv.y), bf16_hi(rv.y),
+                           bf16_lo(rv.z), bf16_hi(rv.z), bf16_lo(rv.w), bf16_hi(rv.w)};
+#pragma unroll
+      for (int i = 0; i < kResRows; ++i) {
+        const int64_t n = min(n0 + i, N - 1);           // rows past N compute row N-1 and are not stored
+        const float lj = __uint_as_float((uint32_t)l[n * ldl + j] << 16);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s[i][e] = __fmaf_rn(lj, rf[e], s[i][e]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kResRows; ++i) {
+      const int64_t n = n0 + i;
+      if (n >= N) break;
+      const uint4 wv = *reinterpret_cast<const uint4*>(w + n * ldw + k0);
+      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        o[e] = f32_to_bf16_bits(__fsub_rn(bf16_lo(ww[e]), s[i][2 * e])) |
+               (f32_to_bf16_bits(__fsub_rn(bf16_hi(ww[e]), s[i][2 * e + 1])) << 16);
+      *reinterpret_cast<uint4*>(out + n * ldo + k0) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ U = BF16(A B^T)
+
+// RT = rank / 8 (n8 tiles).  CTA: 64 rows of A; warp w owns rows 16w..16w+15 and all
+// rank columns.  K streams through a kProjStages-deep cp.async ring of 64-column
+// chunks (dynamic shared memory, kProjSmemBytes), so about 24 KB of A is in flight per
+// CTA; B given transposed ([K x r]) is transposed while it is stored.
+template <int RT>
+__global__ void __launch_bounds__(kProjThreads) lowrank_project_kernel(const uint16_t* __restrict__ a, int64_t lda,
+                                                                       const uint16_t* __restrict__ b, int64_t ldb,
+                                                                       int b_trans, int64_t K,
+                                                                       uint16_t* __restrict__ u, int64_t ldu) {
+  constexpr int R = RT * 8;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint16_t (*As)[kProjRows][kPad] = reinterpret_cast<uint16_t (*)[kProjRows][kPad]>(smem_raw);
+  uint16_t (*Bs)[kMaxRank][kPad] =
+      reinterpret_cast<uint16_t (*)[kMaxRank][kPad]>(smem_raw + kProjStages * kProjRows * kPad * 2);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int64_t m0 = (int64_t)blockIdx.x * kProjRows;
+  const int chunks = (int)(K / kProjKc);
+
+  auto load = [&](int c, int buf) {
+    const int64_t k0 = (int64_t)c * kProjKc;
+#pragma unroll
+    for (int i = 0; i < (kProjRows * 8) / kProjThreads; ++i) {
+      const int idx = tid + i * kProjThreads, row = idx >> 3, ch = idx & 7;
+      cp_async16(&As[buf][row][ch * 8], a + (m0 + row) * lda + k0 + ch * 8);
+    }
+    if (!b_trans) {
+      for (int idx = tid; idx < R * 8; idx += kProjThreads) {
+        const int j = idx >> 3, ch = idx & 7;
+        cp_async16(&Bs[buf][j][ch * 8], b + (int64_t)j * ldb + k0 + ch * 8);
+      }
+    } else {
+      for (int idx = tid; idx < kProjKc * RT; idx += kProjThreads) {
+        const int kr = idx / RT, jc = idx - kr * RT;
+        const uint4 v = *reinterpret_cast<const uint4*>(b + (k0 + kr) * ldb + jc * 8);
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          Bs[buf][jc * 8 + 2 * e][kr] = (uint16_t)(vw[e] & 0xFFFFu);
+          Bs[buf][jc * 8 + 2 * e + 1][kr] = (uint16_t)(vw[e] >> 16);
+        }
+      }
+    }
+  };
+
+  float acc[RT][4];
+#pragma unroll
+  for (int nt = 0; nt < RT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+
+  // prologue: chunks 0 .. S-2, one commit group each (empty past the end)
+#pragma unroll
+  for (int c = 0; c < kProjStages - 1; ++c) {
+    if (c < chunks) load(c, c);
+    cp_async_commit();
+  }
+  for (int c = 0; c < chunks; ++c) {
+    cp_async_wait_pending<kProjStages - 2>();         // chunk c has landed (this thread's copies)
+    __syncthreads();                                  // ... everyone's; chunk c-1's buffer is free
+    const int nc = c + kProjStages - 1;
+    if (nc < chunks) load(nc, nc % kProjStages);
+    cp_async_commit();
+    const int buf = c % kProjStages;
+    const int r0 = warp * 16 + g;
+#pragma unroll
+    for (int kk = 0; kk < kProjKc / 16; ++kk) {
+      const int kc = kk * 16 + 2 * t;
+      uint32_t af[4];
+      af[0] = *reinterpret_cast<const uint32_t*>(&As[buf][r0][kc]);
+      af[1] = *reinterpret_cast<const uint32_t*>(&As[buf][r0 + 8][kc]);
+      af[2] = *reinterpret_cast<const uint32_t*>(&As[buf][r0][kc + 8]);
+      af[3] = *reinterpret_cast<const uint32_t*>(&As[buf][r0 + 8][kc + 8]);
+#pragma unroll
+      for (int nt = 0; nt < RT; ++nt) {
+        uint32_t bfr[2];
+        bfr[0] = *reinterpret_cast<const uint32_t*>(&Bs[buf][nt * 8 + g][kc]);
+        bfr[1] = *reinterpret_cast<const uint32_t*>(&Bs[buf][nt * 8 + g][kc + 8]);
+        mma_bf16_16816(acc[nt], af, bfr);
+      }
+    }
+  }
+  cp_async_wait_pending<0>();
+  const int64_t row = m0 + warp * 16 + g;
+#pragma unroll
+  for (int nt = 0; nt < RT; ++nt) {
+    const int col = nt * 8 + 2 * t;
+    *reinterpret_cast<uint32_t*>(u + row * ldu + col) =
+        f32_to_bf16_bits(acc[nt][0]) | (f32_to_bf16_bits(acc[nt][1]) << 16);
+    *reinterpret_cast<uint32_t*>(u + (row + 8) * ldu + col) =
+        f32_to_bf16_bits(acc[nt][2]) | (f32_to_bf16_bits(acc[nt][3]) << 16);
+  }
+}
+
+// ------------------------------------------------------------------ Y = BF16(Y + U C^T)
+
+// KS = rank / 16 (k16 steps).  CTA: a 128 x 128 tile of Y (blockIdx.x over N tiles,
+// blockIdx.y over M tiles); warp w computes rows 32(w/2).. and columns 64(w%2)..,
+// stages its FP32 results in shared memory, then every thread adds them to the 8
+// 16-byte chunks of Y it read at the start and writes them back.
+template <int KS>
+__global__ void __launch_bounds__(kExpThreads, 2) lowrank_expand_kernel(uint16_t* __restrict__ y, int64_t ldy,
+                                                                     const uint16_t* __restrict__ u, int64_t ldu,
+                                                                     const uint16_t* __restrict__ c, int64_t ldc,
+                                                                     int c_trans) {
+  constexpr int R = KS * 16;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint16_t (*Us)[kPad] = reinterpret_cast<uint16_t (*)[kPad]>(smem_raw);
+  uint16_t (*Cs)[kPad] = reinterpret_cast<uint16_t (*)[kPad]>(smem_raw + kExpTile * kPad * 2);
+  float (*Acc)[kAccStride] = reinterpret_cast<float (*)[kAccStride]>(smem_raw + 2 * kExpTile * kPad * 2);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int64_t n0 = (int64_t)blockIdx.x * kExpTile, m0 = (int64_t)blockIdx.y * kExpTile;
+
+  // This thread's 8 chunks of the Y tile (16 bytes each), read first so that their
+  // latency overlaps the loads and MMAs below; streaming hints keep Y out of the way.
+  constexpr int kChunks = (kExpTile * kExpTile / 8) / kExpThreads;
+  uint4 yold[kChunks];
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    const int idx = tid + i * kExpThreads, row = idx >> 4, ch = idx & 15;
+    yold[i] = __ldcs(reinterpret_cast<const uint4*>(y + (m0 + row) * ldy + n0 + ch * 8));
+  }
+
+  for (int idx = tid; idx < kExpTile * (R / 8); idx += kExpThreads) {
+    const int row = idx / (R / 8), ch = idx - row * (R / 8);
+    *reinterpret_cast<uint4*>(&Us[row][ch * 8]) = *reinterpret_cast<const uint4*>(u + (m0 + row) * ldu + ch * 8);
+  }
+  if (!c_trans) {
+    for (int idx = tid; idx < kExpTile * (R / 8); idx += kExpThreads) {
+      const int row = idx / (R / 8), ch = idx - row * (R / 8);
+      *reinterpret_cast<uint4*>(&Cs[row][ch * 8]) = *reinterpret_cast<const uint4*>(c + (n0 + row) * ldc + ch * 8);
+    }
+  } else {
+    for (int idx = tid; idx < R * (kExpTile / 8); idx += kExpThreads) {
+      const int j = idx / (kExpTile / 8), ch = idx - j * (kExpTile / 8);
+      const uint4 v = *reinterpret_cast<const uint4*>(c + (int64_t)j * ldc + n0 + ch * 8);
+      const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        Cs[ch * 8 + 2 * e][j] = (uint16_t)(vw[e] & 0xFFFFu);
+        Cs[ch * 8 + 2 * e + 1][j] = (uint16_t)(vw[e] >> 16);
+      }
+    }
+  }
+  __syncthreads();
+
+  const int wm = (warp >> 1) * 32, wn = (warp & 1) * 64;
+  float acc[2][8][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
+#pragma unroll 1
+  for (int ks = 0; ks < KS; ++ks) {
+    const int kc = ks * 16 + 2 * t;
+    uint32_t af[2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      const int r0 = wm + mt * 16 + g;
+      af[mt][0] = *reinterpret_cast<const uint32_t*>(&Us[r0][kc]);
+      af[mt][1] = *reinterpret_cast<const uint32_t*>(&Us[r0 + 8][kc]);
+      af[mt][2] = *reinterpret_cast<const uint32_t*>(&Us[r0][kc + 8]);
+      af[mt][3] = *reinterpret_cast<const uint32_t*>(&Us[r0 + 8][kc + 8]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      uint32_t bfr[2];
+      bfr[0] = *reinterpret_cast<const uint32_t*>(&Cs[wn + nt * 8 + g][kc]);
+      bfr[1] = *reinterpret_cast<const uint32_t*>(&Cs[wn + nt * 8 + g][kc + 8]);
+      mma_bf16_16816(acc[0][nt], af[0], bfr);
+      mma_bf16_16816(acc[1][nt], af[1], bfr);
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const int r0 = wm + mt * 16 + g, c0 = wn + nt * 8 + 2 * t;
+      *reinterpret_cast<float2*>(&Acc[r0][c0]) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+      *reinterpret_cast<float2*>(&Acc[r0 + 8][c0]) = make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+    }
+  __syncthreads();
+
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    const int idx = tid + i * kExpThreads, row = idx >> 4, ch = idx & 15;
+    const float4 v0 = *reinterpret_cast<const float4*>(&Acc[row][ch * 8]);
+    const float4 v1 = *reinterpret_cast<const float4*>(&Acc[row][ch * 8 + 4]);
+    const uint32_t ow[4] = {yold[i].x, yold[i].y, yold[i].z, yold[i].w};
+    const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      o[e] = f32_to_bf16_bits(__fadd_rn(bf16_lo(ow[e]), vv[2 * e])) |
+             (f32_to_bf16_bits(__fadd_rn(bf16_hi(ow[e]), vv[2 * e + 1])) << 16);
+    __stcs(reinterpret_cast<uint4*>(y + (m0 + row) * ldy + n0 + ch * 8), make_uint4(o[0], o[1], o[2], o[3]));
+  }
+}
+
+}  // namespace lowrank
+}  // namespace nvfp4

@@ -2,8 +2,8 @@
 //
 // Host side only: argument validation, tensor-map construction for the GEMM's
 // TMA loads, and kernel launches on the caller's stream.  One translation unit
-// holds every kernel (quantize.cuh, gemm.cuh, ns.cuh) so that the module-scope
-// device error word is shared by all of them.
+// holds every kernel (quantize.cuh, gemm.cuh, ns.cuh, lowrank.cuh) so that the
+// module-scope device error word is shared by all of them.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -17,6 +17,7 @@
 #include "nvfp4.h"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "lowrank.cuh"
 #include "ns.cuh"
 #include "quantize.cuh"
 #include "selfcheck.cuh"
@@ -694,6 +695,144 @@ nvfp4_status nvfp4_newton_schulz(const void* G, int64_t m, int64_t n, int64_t ld
     if ((st = gemm_impl(&rr, &xc, X, ldx, NVFP4_OUT_BF16, 0.5f, 1, nullptr, 0u, stream)) != NVFP4_OK) return st;
   }
   return NVFP4_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+bool rank_ok(int32_t rank) { return rank >= 16 && rank <= nvfp4::lowrank::kMaxRank && rank % 16 == 0; }
+
+template <int RT>
+cudaError_t launch_project(const uint16_t* a, int64_t lda, const uint16_t* b, int64_t ldb, int b_trans, int64_t M,
+                           int64_t K, uint16_t* u, int64_t ldu, cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  static std::mutex m;
+  auto kernel = nvfp4::lowrank::lowrank_project_kernel<RT>;
+  cudaError_t e = ensure_smem(kernel, nvfp4::lowrank::kProjSmemBytes, done, m);
+  if (e != cudaSuccess) return e;
+  kernel<<<(unsigned)(M / nvfp4::lowrank::kProjRows), nvfp4::lowrank::kProjThreads, nvfp4::lowrank::kProjSmemBytes,
+           s>>>(a, lda, b, ldb, b_trans, K, u, ldu);
+  return cudaGetLastError();
+}
+
+template <int KS>
+cudaError_t launch_expand(uint16_t* y, int64_t ldy, const uint16_t* u, int64_t ldu, const uint16_t* c, int64_t ldc,
+                          int c_trans, int64_t M, int64_t N, cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  static std::mutex m;
+  auto kernel = nvfp4::lowrank::lowrank_expand_kernel<KS>;
+  cudaError_t e = ensure_smem(kernel, nvfp4::lowrank::kExpSmemBytes, done, m);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)(N / nvfp4::lowrank::kExpTile), (unsigned)(M / nvfp4::lowrank::kExpTile));
+  kernel<<<grid, nvfp4::lowrank::kExpThreads, nvfp4::lowrank::kExpSmemBytes, s>>>(y, ldy, u, ldu, c, ldc, c_trans);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_lora_residual(const void* W, int64_t N, int64_t K, int64_t ldw, const void* L, int64_t ldl,
+                                 const void* R, int64_t ldr, int32_t rank, void* W_res, int64_t ldo, void* stream) {
+  if (!rank_ok(rank)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
+  if (N < 0 || K < 0) return fail(NVFP4_ERR_INVALID_ARG, "negative extent");
+  if (K % 8) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K %lld is not a multiple of 8", (long long)K);
+  if (N == 0 || K == 0) return NVFP4_OK;
+  if (!W || !L || !R || !W_res) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
+  if (ldw < K || ldr < K || ldo < K || ldl < rank) return fail(NVFP4_ERR_INVALID_ARG, "leading dimension too small");
+  if (!aligned16(W) || !aligned16(R) || !aligned16(W_res) || ldw % 8 || ldr % 8 || ldo % 8 ||
+      reinterpret_cast<uintptr_t>(L) % 2)
+    return fail(NVFP4_ERR_MISALIGNED, "W, R and W_res rows must be 16-byte aligned");
+  const int64_t per_row = ceil_div(K / 8, nvfp4::lowrank::kResidualThreads);
+  const dim3 grid((unsigned)per_row, (unsigned)std::min<int64_t>(ceil_div(N, nvfp4::lowrank::kResRows), 65535));
+  nvfp4::lowrank::lora_residual_kernel<<<grid, nvfp4::lowrank::kResidualThreads, 0,
+                                         static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(W), ldw, static_cast<const uint16_t*>(L), ldl, static_cast<const uint16_t*>(R),
+      ldr, static_cast<uint16_t*>(W_res), ldo, N, K, rank);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "lora residual launch");
+}
+
+nvfp4_status nvfp4_lowrank_project(const void* A, int64_t M, int64_t K, int64_t lda, const void* B, int64_t ldb,
+                                   int32_t b_trans, int32_t rank, void* U, int64_t ldu, void* stream) {
+  if (!rank_ok(rank)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
+  if (M < 0 || K < 0) return fail(NVFP4_ERR_INVALID_ARG, "negative extent");
+  if (M % nvfp4::lowrank::kProjRows || K % nvfp4::lowrank::kProjKc || K == 0)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "projection needs M %% 64 == 0 and K a positive multiple of 64");
+  if (M == 0) return NVFP4_OK;
+  if (!A || !B || !U) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
+  if (lda < K || ldu < rank || ldb < (b_trans ? (int64_t)rank : K))
+    return fail(NVFP4_ERR_INVALID_ARG, "leading dimension too small");
+  if (!aligned16(A) || !aligned16(B) || !aligned16(U) || lda % 8 || ldb % 8 || ldu % 8)
+    return fail(NVFP4_ERR_MISALIGNED, "A, B and U rows must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t* a = static_cast<const uint16_t*>(A);
+  const uint16_t* b = static_cast<const uint16_t*>(B);
+  uint16_t* u = static_cast<uint16_t*>(U);
+  const int bt = b_trans ? 1 : 0;
+  cudaError_t e;
+  switch (rank / 8) {
+    case 2: e = launch_project<2>(a, lda, b, ldb, bt, M, K, u, ldu, s); break;
+    case 4: e = launch_project<4>(a, lda, b, ldb, bt, M, K, u, ldu, s); break;
+    case 6: e = launch_project<6>(a, lda, b, ldb, bt, M, K, u, ldu, s); break;
+    default: e = launch_project<8>(a, lda, b, ldb, bt, M, K, u, ldu, s); break;
+  }
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "low-rank projection launch");
+}
+
+nvfp4_status nvfp4_lowrank_expand_add(void* Y, int64_t M, int64_t N, int64_t ldy, const void* U, int64_t ldu,
+                                      const void* C, int64_t ldc, int32_t c_trans, int32_t rank, void* stream) {
+  if (!rank_ok(rank)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
+  if (M < 0 || N < 0) return fail(NVFP4_ERR_INVALID_ARG, "negative extent");
+  if (M % nvfp4::lowrank::kExpTile || N % nvfp4::lowrank::kExpTile)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "expansion needs M %% 128 == 0 and N %% 128 == 0");
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (!Y || !U || !C) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
+  if (ldy < N || ldu < rank || ldc < (c_trans ? N : (int64_t)rank))
+    return fail(NVFP4_ERR_INVALID_ARG, "leading dimension too small");
+  if (!aligned16(Y) || !aligned16(U) || !aligned16(C) || ldy % 8 || ldu % 8 || ldc % 8)
+    return fail(NVFP4_ERR_MISALIGNED, "Y, U and C rows must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* y = static_cast<uint16_t*>(Y);
+  const uint16_t* u = static_cast<const uint16_t*>(U);
+  const uint16_t* c = static_cast<const uint16_t*>(C);
+  const int ct = c_trans ? 1 : 0;
+  cudaError_t e;
+  switch (rank / 16) {
+    case 1: e = launch_expand<1>(y, ldy, u, ldu, c, ldc, ct, M, N, s); break;
+    case 2: e = launch_expand<2>(y, ldy, u, ldu, c, ldc, ct, M, N, s); break;
+    case 3: e = launch_expand<3>(y, ldy, u, ldu, c, ldc, ct, M, N, s); break;
+    default: e = launch_expand<4>(y, ldy, u, ldu, c, ldc, ct, M, N, s); break;
+  }
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "low-rank expansion launch");
+}
+
+nvfp4_status nvfp4_lora_linear_fwd(const void* X, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* Wq_res_row,
+                                   const void* L, const void* R, int32_t rank, void* Y, int64_t ldy,
+                                   nvfp4_tensor* Xq_row, nvfp4_tensor* Xq_col, uint32_t rht_signs, void* U,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (!rank_ok(rank)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
+  nvfp4_status st = nvfp4_linear_fwd(X, M, K, ldx, Wq_res_row, Y, ldy, NVFP4_OUT_BF16, Xq_row, Xq_col, rht_signs,
+                                     workspace, workspace_bytes, stream);
+  if (st != NVFP4_OK) return st;
+  const int64_t N = Wq_res_row->rows;
+  if ((st = nvfp4_lowrank_project(X, M, K, ldx, R, K, 0, rank, U, rank, stream)) != NVFP4_OK) return st;
+  return nvfp4_lowrank_expand_add(Y, M, N, ldy, U, rank, L, rank, 0, rank, stream);
+}
+
+nvfp4_status nvfp4_lora_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ldy, const nvfp4_tensor* Wq_res_col,
+                                     const void* L, const void* R, int32_t rank, void* dX, int64_t ldx,
+                                     nvfp4_tensor* dYq_row, nvfp4_tensor* dYq_col, uint64_t seed, uint64_t offset,
+                                     uint32_t rht_signs, void* U, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (!rank_ok(rank)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
+  nvfp4_status st = nvfp4_linear_dgrad(dY, M, N, ldy, Wq_res_col, dX, ldx, NVFP4_OUT_BF16, dYq_row, dYq_col, seed,
+                                       offset, rht_signs, workspace, workspace_bytes, stream);
+  if (st != NVFP4_OK) return st;
+  const int64_t K = Wq_res_col->rows;
+  if ((st = nvfp4_lowrank_project(dY, M, N, ldy, L, rank, 1, rank, U, rank, stream)) != NVFP4_OK) return st;
+  return nvfp4_lowrank_expand_add(dX, M, K, ldx, U, rank, R, K, 1, rank, stream);
 }
 
 nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,

@@ -130,3 +130,21 @@ def test_newton_schulz_workspace_and_argument_errors(lib):
     assert call(wsb=need - 1) == 6
     assert call(ws=0x300010) == 3               # workspace not 256-byte aligned
     assert "workspace" in lib.nvfp4_last_error_string().decode()
+
+
+def test_lowrank_argument_errors(lib):
+    a, b, u, y = 0x100000, 0x200000, 0x300000, 0x400000
+    assert lib.nvfp4_lowrank_project(a, 128, 256, 256, b, 256, 0, 24, u, 24, None) == 2       # rank not 16k
+    assert lib.nvfp4_lowrank_project(a, 128, 256, 256, b, 256, 0, 80, u, 80, None) == 2       # rank above 64
+    assert lib.nvfp4_lowrank_project(a, 96, 256, 256, b, 256, 0, 32, u, 32, None) == 2        # M % 64
+    assert lib.nvfp4_lowrank_project(a, 128, 200, 200, b, 200, 0, 32, u, 32, None) == 2       # K % 64
+    assert lib.nvfp4_lowrank_project(a, 128, 256, 256, b, 16, 1, 32, u, 32, None) == 1        # ldb < rank (transposed)
+    assert lib.nvfp4_lowrank_project(a + 8, 128, 256, 256, b, 256, 0, 32, u, 32, None) == 3
+    assert lib.nvfp4_lowrank_project(None, 128, 256, 256, b, 256, 0, 32, u, 32, None) == 1
+    assert lib.nvfp4_lowrank_expand_add(y, 128, 192, 192, u, 32, b, 32, 0, 32, None) == 2     # N % 128
+    assert lib.nvfp4_lowrank_expand_add(y, 128, 256, 256, u, 32, b, 128, 1, 32, None) == 1    # ldc < N (transposed)
+    assert lib.nvfp4_lowrank_expand_add(y, 128, 256, 260, u, 32, b, 32, 0, 32, None) == 3     # ldy % 8
+    assert lib.nvfp4_lora_residual(y, 64, 100, 100, b, 32, a, 100, 32, u, 100, None) == 2     # K % 8
+    assert lib.nvfp4_lora_residual(y, 64, 128, 128, b, 16, a, 128, 32, u, 128, None) == 1     # ldl < rank
+    assert lib.nvfp4_lora_residual(y + 4, 64, 128, 128, b, 32, a, 128, 32, u, 128, None) == 3
+    assert lib.nvfp4_lora_residual(y, 64, 128, 128, b, 32, a, 128, 8, u, 128, None) == 2       # rank 8
