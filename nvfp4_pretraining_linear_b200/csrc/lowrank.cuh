@@ -11,7 +11,8 @@
 //   lowrank_project_kernel U = BF16(A B^T), A [M x K] BF16, B [r x K] (or given as
 //                          [K x r]); HBM-bound on A.
 //   lowrank_expand_kernel  Y = BF16(fl32(Y + U C^T)), U [M x r], C [N x r] (or given
-//                          as [r x N]); HBM-bound on the read-modify-write of Y.
+//                          as [r x N]); HBM-bound on the read-modify-write of Y,
+//                          persistent, with a ring of Y tiles in flight.
 //
 // The two products are dense contractions with a short side (r <= 64), so they run
 // on the warp-level BF16 tensor-core MMA (m16n8k16, FP32 accumulation) from shared
@@ -35,10 +36,8 @@ constexpr int kProjKc = 64;            // K per pipeline stage
 constexpr int kProjStages = 4;
 constexpr int kPad = 72;               // shared row stride in BF16 elements (144 B, conflict-free)
 constexpr int kProjSmemBytes = kProjStages * (kProjRows + kMaxRank) * kPad * 2;
-constexpr int kExpTile = 128;          // Y tile 128 x 128 per CTA
+constexpr int kExpTile = 128;          // Y tile 128 x 128
 constexpr int kExpThreads = 256;
-constexpr int kAccStride = 132;        // FP32 row stride of the staged accumulator tile
-constexpr int kExpSmemBytes = 2 * kExpTile * kPad * 2 + kExpTile * kAccStride * 4;
 
 // One warp-level BF16 MMA: d += a(16x16, row) * b(16x8, col), FP32 accumulators.
 __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, const uint32_t* b) {
@@ -196,107 +195,141 @@ __global__ void __launch_bounds__(kProjThreads) lowrank_project_kernel(const uin
 
 // ------------------------------------------------------------------ Y = BF16(Y + U C^T)
 
-// KS = rank / 16 (k16 steps).  CTA: a 128 x 128 tile of Y (blockIdx.x over N tiles,
-// blockIdx.y over M tiles); warp w computes rows 32(w/2).. and columns 64(w%2)..,
-// stages its FP32 results in shared memory, then every thread adds them to the 8
-// 16-byte chunks of Y it read at the start and writes them back.
+// Ring depth of the expansion and its shared-memory bytes per stage: the staged Y tile
+// (128 x 136 BF16), the U tile and the C tile (128 x (r + 8) BF16 each).
 template <int KS>
-__global__ void __launch_bounds__(kExpThreads, 2) lowrank_expand_kernel(uint16_t* __restrict__ y, int64_t ldy,
+__host__ __device__ constexpr int exp_stages() { return KS <= 2 ? 4 : 3; }
+constexpr int kYStride = kExpTile + 8;
+template <int KS>
+__host__ __device__ constexpr int exp_stage_bytes() { return kExpTile * kYStride * 2 + 2 * kExpTile * (KS * 16 + 8) * 2; }
+template <int KS>
+__host__ __device__ constexpr int exp_smem_bytes() { return exp_stages<KS>() * exp_stage_bytes<KS>(); }
+
+// KS = rank / 16 (k16 steps).  Persistent: CTA b takes the 128 x 128 tiles b, b + G,
+// ... of Y (G = gridDim.x, N tiles fastest) through a ring of exp_stages() stages, so
+// the Y tiles of the next stages stream in (cp.async) while one is computed.  Per
+// tile: warp w multiplies rows 32(w/2).. by columns 64(w%2).. (r/16 MMAs of m16n8k16
+// per 16 x 8 block), adds its FP32 results into the staged BF16 Y in place (each
+// element belongs to one lane), and the CTA writes the tile back in 16-byte chunks.
+// C given as [r x N] (c_trans) is transposed while it is stored.
+template <int KS>
+__global__ void __launch_bounds__(kExpThreads) lowrank_expand_kernel(uint16_t* __restrict__ y, int64_t ldy,
                                                                      const uint16_t* __restrict__ u, int64_t ldu,
                                                                      const uint16_t* __restrict__ c, int64_t ldc,
-                                                                     int c_trans) {
-  constexpr int R = KS * 16;
+                                                                     int c_trans, int32_t tiles_n, int32_t tiles) {
+  constexpr int R = KS * 16, RS = R + 8, S = exp_stages<KS>();
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  uint16_t (*Us)[kPad] = reinterpret_cast<uint16_t (*)[kPad]>(smem_raw);
-  uint16_t (*Cs)[kPad] = reinterpret_cast<uint16_t (*)[kPad]>(smem_raw + kExpTile * kPad * 2);
-  float (*Acc)[kAccStride] = reinterpret_cast<float (*)[kAccStride]>(smem_raw + 2 * kExpTile * kPad * 2);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int64_t n0 = (int64_t)blockIdx.x * kExpTile, m0 = (int64_t)blockIdx.y * kExpTile;
+  const int wm = (warp >> 1) * 32, wn = (warp & 1) * 64;
+  auto Ys = [&](int st) { return reinterpret_cast<uint16_t (*)[kYStride]>(smem_raw + st * exp_stage_bytes<KS>()); };
+  auto Us = [&](int st) {
+    return reinterpret_cast<uint16_t (*)[RS]>(smem_raw + st * exp_stage_bytes<KS>() + kExpTile * kYStride * 2);
+  };
+  auto Cs = [&](int st) {
+    return reinterpret_cast<uint16_t (*)[RS]>(smem_raw + st * exp_stage_bytes<KS>() + kExpTile * kYStride * 2 +
+                                              kExpTile * RS * 2);
+  };
 
-  // This thread's 8 chunks of the Y tile (16 bytes each), read first so that their
-  // latency overlaps the loads and MMAs below; streaming hints keep Y out of the way.
-  constexpr int kChunks = (kExpTile * kExpTile / 8) / kExpThreads;
-  uint4 yold[kChunks];
+  auto load = [&](int tile, int st) {
+    const int64_t m0 = (int64_t)(tile / tiles_n) * kExpTile, n0 = (int64_t)(tile % tiles_n) * kExpTile;
+    uint16_t (*ys)[kYStride] = Ys(st);
+    uint16_t (*us)[RS] = Us(st);
+    uint16_t (*cs)[RS] = Cs(st);
 #pragma unroll
-  for (int i = 0; i < kChunks; ++i) {
-    const int idx = tid + i * kExpThreads, row = idx >> 4, ch = idx & 15;
-    yold[i] = __ldcs(reinterpret_cast<const uint4*>(y + (m0 + row) * ldy + n0 + ch * 8));
-  }
-
-  for (int idx = tid; idx < kExpTile * (R / 8); idx += kExpThreads) {
-    const int row = idx / (R / 8), ch = idx - row * (R / 8);
-    *reinterpret_cast<uint4*>(&Us[row][ch * 8]) = *reinterpret_cast<const uint4*>(u + (m0 + row) * ldu + ch * 8);
-  }
-  if (!c_trans) {
+    for (int i = 0; i < (kExpTile * kExpTile / 8) / kExpThreads; ++i) {
+      const int idx = tid + i * kExpThreads, row = idx >> 4, ch = idx & 15;
+      cp_async16(&ys[row][ch * 8], y + (m0 + row) * ldy + n0 + ch * 8);
+    }
     for (int idx = tid; idx < kExpTile * (R / 8); idx += kExpThreads) {
       const int row = idx / (R / 8), ch = idx - row * (R / 8);
-      *reinterpret_cast<uint4*>(&Cs[row][ch * 8]) = *reinterpret_cast<const uint4*>(c + (n0 + row) * ldc + ch * 8);
+      cp_async16(&us[row][ch * 8], u + (m0 + row) * ldu + ch * 8);
     }
-  } else {
-    for (int idx = tid; idx < R * (kExpTile / 8); idx += kExpThreads) {
-      const int j = idx / (kExpTile / 8), ch = idx - j * (kExpTile / 8);
-      const uint4 v = *reinterpret_cast<const uint4*>(c + (int64_t)j * ldc + n0 + ch * 8);
-      const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+    if (!c_trans) {
+      for (int idx = tid; idx < kExpTile * (R / 8); idx += kExpThreads) {
+        const int row = idx / (R / 8), ch = idx - row * (R / 8);
+        cp_async16(&cs[row][ch * 8], c + (n0 + row) * ldc + ch * 8);
+      }
+    } else {
+      for (int idx = tid; idx < R * (kExpTile / 8); idx += kExpThreads) {
+        const int j = idx / (kExpTile / 8), ch = idx - j * (kExpTile / 8);
+        const uint4 v = *reinterpret_cast<const uint4*>(c + (int64_t)j * ldc + n0 + ch * 8);
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        Cs[ch * 8 + 2 * e][j] = (uint16_t)(vw[e] & 0xFFFFu);
-        Cs[ch * 8 + 2 * e + 1][j] = (uint16_t)(vw[e] >> 16);
+        for (int e = 0; e < 4; ++e) {
+          cs[ch * 8 + 2 * e][j] = (uint16_t)(vw[e] & 0xFFFFu);
+          cs[ch * 8 + 2 * e + 1][j] = (uint16_t)(vw[e] >> 16);
+        }
       }
     }
-  }
-  __syncthreads();
+  };
 
-  const int wm = (warp >> 1) * 32, wn = (warp & 1) * 64;
-  float acc[2][8][4];
+  const int first = blockIdx.x, step = gridDim.x;
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
+  for (int k = 0; k < S - 1; ++k) {
+    const int tile = first + k * step;
+    if (tile < tiles) load(tile, k);
+    cp_async_commit();
+  }
+  for (int k = 0;; ++k) {
+    const int tile = first + k * step;
+    if (tile >= tiles) break;
+    const int st = k % S;
+    cp_async_wait_pending<S - 2>();                   // tile k has landed (this thread's copies)
+    __syncthreads();                                  // ... everyone's; the stage of tile k-1 is free
+    const int ahead = first + (k + S - 1) * step;
+    if (ahead < tiles) load(ahead, (k + S - 1) % S);
+    cp_async_commit();
+
+    uint16_t (*ys)[kYStride] = Ys(st);
+    uint16_t (*us)[RS] = Us(st);
+    uint16_t (*cs)[RS] = Cs(st);
+    float acc[2][8][4];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
 #pragma unroll 1
-  for (int ks = 0; ks < KS; ++ks) {
-    const int kc = ks * 16 + 2 * t;
-    uint32_t af[2][4];
+    for (int ks = 0; ks < KS; ++ks) {
+      const int kc = ks * 16 + 2 * t;
+      uint32_t af[2][4];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      const int r0 = wm + mt * 16 + g;
-      af[mt][0] = *reinterpret_cast<const uint32_t*>(&Us[r0][kc]);
-      af[mt][1] = *reinterpret_cast<const uint32_t*>(&Us[r0 + 8][kc]);
-      af[mt][2] = *reinterpret_cast<const uint32_t*>(&Us[r0][kc + 8]);
-      af[mt][3] = *reinterpret_cast<const uint32_t*>(&Us[r0 + 8][kc + 8]);
+      for (int mt = 0; mt < 2; ++mt) {
+        const int r0 = wm + mt * 16 + g;
+        af[mt][0] = *reinterpret_cast<const uint32_t*>(&us[r0][kc]);
+        af[mt][1] = *reinterpret_cast<const uint32_t*>(&us[r0 + 8][kc]);
+        af[mt][2] = *reinterpret_cast<const uint32_t*>(&us[r0][kc + 8]);
+        af[mt][3] = *reinterpret_cast<const uint32_t*>(&us[r0 + 8][kc + 8]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        uint32_t bfr[2];
+        bfr[0] = *reinterpret_cast<const uint32_t*>(&cs[wn + nt * 8 + g][kc]);
+        bfr[1] = *reinterpret_cast<const uint32_t*>(&cs[wn + nt * 8 + g][kc + 8]);
+        mma_bf16_16816(acc[0][nt], af[0], bfr);
+        mma_bf16_16816(acc[1][nt], af[1], bfr);
+      }
     }
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      uint32_t bfr[2];
-      bfr[0] = *reinterpret_cast<const uint32_t*>(&Cs[wn + nt * 8 + g][kc]);
-      bfr[1] = *reinterpret_cast<const uint32_t*>(&Cs[wn + nt * 8 + g][kc + 8]);
-      mma_bf16_16816(acc[0][nt], af[0], bfr);
-      mma_bf16_16816(acc[1][nt], af[1], bfr);
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t* p = reinterpret_cast<uint32_t*>(&ys[wm + mt * 16 + g + 8 * h][wn + nt * 8 + 2 * t]);
+          const uint32_t old = *p;
+          *p = f32_to_bf16_bits(__fadd_rn(bf16_lo(old), acc[mt][nt][2 * h])) |
+               (f32_to_bf16_bits(__fadd_rn(bf16_hi(old), acc[mt][nt][2 * h + 1])) << 16);
+        }
+    __syncthreads();
+    const int64_t m0 = (int64_t)(tile / tiles_n) * kExpTile, n0 = (int64_t)(tile % tiles_n) * kExpTile;
+#pragma unroll
+    for (int i = 0; i < (kExpTile * kExpTile / 8) / kExpThreads; ++i) {
+      const int idx = tid + i * kExpThreads, row = idx >> 4, ch = idx & 15;
+      __stcs(reinterpret_cast<uint4*>(y + (m0 + row) * ldy + n0 + ch * 8),
+             *reinterpret_cast<const uint4*>(&ys[row][ch * 8]));
     }
   }
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int r0 = wm + mt * 16 + g, c0 = wn + nt * 8 + 2 * t;
-      *reinterpret_cast<float2*>(&Acc[r0][c0]) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
-      *reinterpret_cast<float2*>(&Acc[r0 + 8][c0]) = make_float2(acc[mt][nt][2], acc[mt][nt][3]);
-    }
-  __syncthreads();
-
-#pragma unroll
-  for (int i = 0; i < kChunks; ++i) {
-    const int idx = tid + i * kExpThreads, row = idx >> 4, ch = idx & 15;
-    const float4 v0 = *reinterpret_cast<const float4*>(&Acc[row][ch * 8]);
-    const float4 v1 = *reinterpret_cast<const float4*>(&Acc[row][ch * 8 + 4]);
-    const uint32_t ow[4] = {yold[i].x, yold[i].y, yold[i].z, yold[i].w};
-    const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      o[e] = f32_to_bf16_bits(__fadd_rn(bf16_lo(ow[e]), vv[2 * e])) |
-             (f32_to_bf16_bits(__fadd_rn(bf16_hi(ow[e]), vv[2 * e + 1])) << 16);
-    __stcs(reinterpret_cast<uint4*>(y + (m0 + row) * ldy + n0 + ch * 8), make_uint4(o[0], o[1], o[2], o[3]));
-  }
+  cp_async_wait_pending<0>();
 }
 
 }  // namespace lowrank

@@ -718,14 +718,18 @@ cudaError_t launch_project(const uint16_t* a, int64_t lda, const uint16_t* b, in
 
 template <int KS>
 cudaError_t launch_expand(uint16_t* y, int64_t ldy, const uint16_t* u, int64_t ldu, const uint16_t* c, int64_t ldc,
-                          int c_trans, int64_t M, int64_t N, cudaStream_t s) {
+                          int c_trans, int64_t M, int64_t N, int sm_count, cudaStream_t s) {
   static bool done[kMaxDevices] = {};
   static std::mutex m;
   auto kernel = nvfp4::lowrank::lowrank_expand_kernel<KS>;
-  cudaError_t e = ensure_smem(kernel, nvfp4::lowrank::kExpSmemBytes, done, m);
+  constexpr int smem = nvfp4::lowrank::exp_smem_bytes<KS>();
+  cudaError_t e = ensure_smem(kernel, smem, done, m);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)(N / nvfp4::lowrank::kExpTile), (unsigned)(M / nvfp4::lowrank::kExpTile));
-  kernel<<<grid, nvfp4::lowrank::kExpThreads, nvfp4::lowrank::kExpSmemBytes, s>>>(y, ldy, u, ldu, c, ldc, c_trans);
+  const int64_t tiles_n = N / nvfp4::lowrank::kExpTile;
+  const int64_t tiles = (M / nvfp4::lowrank::kExpTile) * tiles_n;
+  const int grid = (int)std::min<int64_t>(tiles, sm_count);
+  kernel<<<grid, nvfp4::lowrank::kExpThreads, smem, s>>>(y, ldy, u, ldu, c, ldc, c_trans, (int32_t)tiles_n,
+                                                         (int32_t)tiles);
   return cudaGetLastError();
 }
 
@@ -793,17 +797,23 @@ nvfp4_status nvfp4_lowrank_expand_add(void* Y, int64_t M, int64_t N, int64_t ldy
     return fail(NVFP4_ERR_INVALID_ARG, "leading dimension too small");
   if (!aligned16(Y) || !aligned16(U) || !aligned16(C) || ldy % 8 || ldu % 8 || ldc % 8)
     return fail(NVFP4_ERR_MISALIGNED, "Y, U and C rows must be 16-byte aligned");
+  if ((M / nvfp4::lowrank::kExpTile) * (N / nvfp4::lowrank::kExpTile) > INT32_MAX)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "expansion has more than 2^31 tiles");
+  DeviceInfo* dev;
+  nvfp4_status st = device_info(&dev);
+  if (st != NVFP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint16_t* y = static_cast<uint16_t*>(Y);
   const uint16_t* u = static_cast<const uint16_t*>(U);
   const uint16_t* c = static_cast<const uint16_t*>(C);
   const int ct = c_trans ? 1 : 0;
+  const int sms = dev->sm_count;
   cudaError_t e;
   switch (rank / 16) {
-    case 1: e = launch_expand<1>(y, ldy, u, ldu, c, ldc, ct, M, N, s); break;
-    case 2: e = launch_expand<2>(y, ldy, u, ldu, c, ldc, ct, M, N, s); break;
-    case 3: e = launch_expand<3>(y, ldy, u, ldu, c, ldc, ct, M, N, s); break;
-    default: e = launch_expand<4>(y, ldy, u, ldu, c, ldc, ct, M, N, s); break;
+    case 1: e = launch_expand<1>(y, ldy, u, ldu, c, ldc, ct, M, N, sms, s); break;
+    case 2: e = launch_expand<2>(y, ldy, u, ldu, c, ldc, ct, M, N, sms, s); break;
+    case 3: e = launch_expand<3>(y, ldy, u, ldu, c, ldc, ct, M, N, sms, s); break;
+    default: e = launch_expand<4>(y, ldy, u, ldu, c, ldc, ct, M, N, sms, s); break;
   }
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "low-rank expansion launch");
 }
