@@ -102,16 +102,24 @@ __global__ void __launch_bounds__(kResidualThreads) lora_residual_kernel(
 
 // ------------------------------------------------------------------ U = BF16(A B^T)
 
+// Two BF16 values from shared memory packed as one MMA operand register, the first in
+// the low half (the operand element with the lower K index).
+__device__ __forceinline__ uint32_t pack_bf16_pair(const uint16_t* lo, const uint16_t* hi) {
+  return (uint32_t)*lo | ((uint32_t)*hi << 16);
+}
+
 // RT = rank / 8 (n8 tiles).  CTA: 64 rows of A; warp w owns rows 16w..16w+15 and all
 // rank columns.  K streams through a kProjStages-deep cp.async ring of 64-column
 // chunks (dynamic shared memory, kProjSmemBytes), so about 24 KB of A is in flight per
-// CTA; B given transposed ([K x r]) is transposed while it is stored.
-template <int RT>
+// CTA.  B is staged as given: [r x K] rows (BT false) give each MMA operand register
+// as one 32-bit load; [K x r] rows (BT true, e.g. L in dgrad) are staged unchanged and
+// each register is packed from two 16-bit loads.
+template <int RT, bool BT>
 __global__ void __launch_bounds__(kProjThreads) lowrank_project_kernel(const uint16_t* __restrict__ a, int64_t lda,
                                                                        const uint16_t* __restrict__ b, int64_t ldb,
-                                                                       int b_trans, int64_t K,
-                                                                       uint16_t* __restrict__ u, int64_t ldu) {
-  constexpr int R = RT * 8;
+                                                                       int64_t K, uint16_t* __restrict__ u,
+                                                                       int64_t ldu) {
+  constexpr int R = RT * 8, RSn = R + 8;          // RSn: row stride of a staged [K x r] chunk
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint16_t (*As)[kProjRows][kPad] = reinterpret_cast<uint16_t (*)[kProjRows][kPad]>(smem_raw);
   uint16_t (*Bs)[kMaxRank][kPad] =
@@ -127,21 +135,16 @@ __global__ void __launch_bounds__(kProjThreads) lowrank_project_kernel(const uin
       const int idx = tid + i * kProjThreads, row = idx >> 3, ch = idx & 7;
       cp_async16(&As[buf][row][ch * 8], a + (m0 + row) * lda + k0 + ch * 8);
     }
-    if (!b_trans) {
+    if constexpr (!BT) {
       for (int idx = tid; idx < R * 8; idx += kProjThreads) {
         const int j = idx >> 3, ch = idx & 7;
         cp_async16(&Bs[buf][j][ch * 8], b + (int64_t)j * ldb + k0 + ch * 8);
       }
     } else {
+      uint16_t* bn = &Bs[buf][0][0];                 // [kProjKc][RSn] within the same stage buffer
       for (int idx = tid; idx < kProjKc * RT; idx += kProjThreads) {
         const int kr = idx / RT, jc = idx - kr * RT;
-        const uint4 v = *reinterpret_cast<const uint4*>(b + (k0 + kr) * ldb + jc * 8);
-        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          Bs[buf][jc * 8 + 2 * e][kr] = (uint16_t)(vw[e] & 0xFFFFu);
-          Bs[buf][jc * 8 + 2 * e + 1][kr] = (uint16_t)(vw[e] >> 16);
-        }
+        cp_async16(bn + kr * RSn + jc * 8, b + (k0 + kr) * ldb + jc * 8);
       }
     }
   };
@@ -175,8 +178,14 @@ __global__ void __launch_bounds__(kProjThreads) lowrank_project_kernel(const uin
 #pragma unroll
       for (int nt = 0; nt < RT; ++nt) {
         uint32_t bfr[2];
-        bfr[0] = *reinterpret_cast<const uint32_t*>(&Bs[buf][nt * 8 + g][kc]);
-        bfr[1] = *reinterpret_cast<const uint32_t*>(&Bs[buf][nt * 8 + g][kc + 8]);
+        if constexpr (!BT) {
+          bfr[0] = *reinterpret_cast<const uint32_t*>(&Bs[buf][nt * 8 + g][kc]);
+          bfr[1] = *reinterpret_cast<const uint32_t*>(&Bs[buf][nt * 8 + g][kc + 8]);
+        } else {
+          const uint16_t* bn = &Bs[buf][0][0] + nt * 8 + g;
+          bfr[0] = pack_bf16_pair(bn + kc * RSn, bn + (kc + 1) * RSn);
+          bfr[1] = pack_bf16_pair(bn + (kc + 8) * RSn, bn + (kc + 9) * RSn);
+        }
         mma_bf16_16816(acc[nt], af, bfr);
       }
     }
@@ -196,7 +205,8 @@ __global__ void __launch_bounds__(kProjThreads) lowrank_project_kernel(const uin
 // ------------------------------------------------------------------ Y = BF16(Y + U C^T)
 
 // Ring depth of the expansion and its shared-memory bytes per stage: the staged Y tile
-// (128 x 136 BF16), the U tile and the C tile (128 x (r + 8) BF16 each).
+// (128 x 136 BF16), the U tile and the C tile (128 x (r + 8) BF16 each; a C given as
+// [r x N] takes r x 136 of that space).
 template <int KS>
 __host__ __device__ constexpr int exp_stages() { return KS <= 2 ? 4 : 3; }
 constexpr int kYStride = kExpTile + 8;
@@ -211,12 +221,13 @@ __host__ __device__ constexpr int exp_smem_bytes() { return exp_stages<KS>() * e
 // tile: warp w multiplies rows 32(w/2).. by columns 64(w%2).. (r/16 MMAs of m16n8k16
 // per 16 x 8 block), adds its FP32 results into the staged BF16 Y in place (each
 // element belongs to one lane), and the CTA writes the tile back in 16-byte chunks.
-// C given as [r x N] (c_trans) is transposed while it is stored.
-template <int KS>
+// C is staged as given: [N x r] rows (CT false) or [r x N] rows (CT true, e.g. R^T in
+// dgrad), whose MMA operand registers are packed from two 16-bit loads.
+template <int KS, bool CT>
 __global__ void __launch_bounds__(kExpThreads) lowrank_expand_kernel(uint16_t* __restrict__ y, int64_t ldy,
                                                                      const uint16_t* __restrict__ u, int64_t ldu,
                                                                      const uint16_t* __restrict__ c, int64_t ldc,
-                                                                     int c_trans, int32_t tiles_n, int32_t tiles) {
+                                                                     int32_t tiles_n, int32_t tiles) {
   constexpr int R = KS * 16, RS = R + 8, S = exp_stages<KS>();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
@@ -244,21 +255,16 @@ __global__ void __launch_bounds__(kExpThreads) lowrank_expand_kernel(uint16_t* _
       const int row = idx / (R / 8), ch = idx - row * (R / 8);
       cp_async16(&us[row][ch * 8], u + (m0 + row) * ldu + ch * 8);
     }
-    if (!c_trans) {
+    if constexpr (!CT) {
       for (int idx = tid; idx < kExpTile * (R / 8); idx += kExpThreads) {
         const int row = idx / (R / 8), ch = idx - row * (R / 8);
         cp_async16(&cs[row][ch * 8], c + (n0 + row) * ldc + ch * 8);
       }
     } else {
+      uint16_t* cn = &cs[0][0];                      // [R][kYStride] within the same stage buffer
       for (int idx = tid; idx < R * (kExpTile / 8); idx += kExpThreads) {
         const int j = idx / (kExpTile / 8), ch = idx - j * (kExpTile / 8);
-        const uint4 v = *reinterpret_cast<const uint4*>(c + (int64_t)j * ldc + n0 + ch * 8);
-        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          cs[ch * 8 + 2 * e][j] = (uint16_t)(vw[e] & 0xFFFFu);
-          cs[ch * 8 + 2 * e + 1][j] = (uint16_t)(vw[e] >> 16);
-        }
+        cp_async16(cn + j * kYStride + ch * 8, c + (int64_t)j * ldc + n0 + ch * 8);
       }
     }
   };
@@ -303,8 +309,14 @@ __global__ void __launch_bounds__(kExpThreads) lowrank_expand_kernel(uint16_t* _
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         uint32_t bfr[2];
-        bfr[0] = *reinterpret_cast<const uint32_t*>(&cs[wn + nt * 8 + g][kc]);
-        bfr[1] = *reinterpret_cast<const uint32_t*>(&cs[wn + nt * 8 + g][kc + 8]);
+        if constexpr (!CT) {
+          bfr[0] = *reinterpret_cast<const uint32_t*>(&cs[wn + nt * 8 + g][kc]);
+          bfr[1] = *reinterpret_cast<const uint32_t*>(&cs[wn + nt * 8 + g][kc + 8]);
+        } else {
+          const uint16_t* cn = &cs[0][0] + wn + nt * 8 + g;
+          bfr[0] = pack_bf16_pair(cn + kc * kYStride, cn + (kc + 1) * kYStride);
+          bfr[1] = pack_bf16_pair(cn + (kc + 8) * kYStride, cn + (kc + 9) * kYStride);
+        }
         mma_bf16_16816(acc[0][nt], af[0], bfr);
         mma_bf16_16816(acc[1][nt], af[1], bfr);
       }

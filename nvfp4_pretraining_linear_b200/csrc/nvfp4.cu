@@ -703,34 +703,47 @@ namespace {
 
 bool rank_ok(int32_t rank) { return rank >= 16 && rank <= nvfp4::lowrank::kMaxRank && rank % 16 == 0; }
 
-template <int RT>
-cudaError_t launch_project(const uint16_t* a, int64_t lda, const uint16_t* b, int64_t ldb, int b_trans, int64_t M,
-                           int64_t K, uint16_t* u, int64_t ldu, cudaStream_t s) {
+template <int RT, bool BT>
+cudaError_t launch_project(const uint16_t* a, int64_t lda, const uint16_t* b, int64_t ldb, int64_t M, int64_t K,
+                           uint16_t* u, int64_t ldu, cudaStream_t s) {
   static bool done[kMaxDevices] = {};
   static std::mutex m;
-  auto kernel = nvfp4::lowrank::lowrank_project_kernel<RT>;
+  auto kernel = nvfp4::lowrank::lowrank_project_kernel<RT, BT>;
   cudaError_t e = ensure_smem(kernel, nvfp4::lowrank::kProjSmemBytes, done, m);
   if (e != cudaSuccess) return e;
   kernel<<<(unsigned)(M / nvfp4::lowrank::kProjRows), nvfp4::lowrank::kProjThreads, nvfp4::lowrank::kProjSmemBytes,
-           s>>>(a, lda, b, ldb, b_trans, K, u, ldu);
+           s>>>(a, lda, b, ldb, K, u, ldu);
   return cudaGetLastError();
 }
 
-template <int KS>
+template <int RT>
+cudaError_t dispatch_project(bool bt, const uint16_t* a, int64_t lda, const uint16_t* b, int64_t ldb, int64_t M,
+                             int64_t K, uint16_t* u, int64_t ldu, cudaStream_t s) {
+  return bt ? launch_project<RT, true>(a, lda, b, ldb, M, K, u, ldu, s)
+            : launch_project<RT, false>(a, lda, b, ldb, M, K, u, ldu, s);
+}
+
+template <int KS, bool CT>
 cudaError_t launch_expand(uint16_t* y, int64_t ldy, const uint16_t* u, int64_t ldu, const uint16_t* c, int64_t ldc,
-                          int c_trans, int64_t M, int64_t N, int sm_count, cudaStream_t s) {
+                          int64_t M, int64_t N, int sm_count, cudaStream_t s) {
   static bool done[kMaxDevices] = {};
   static std::mutex m;
-  auto kernel = nvfp4::lowrank::lowrank_expand_kernel<KS>;
+  auto kernel = nvfp4::lowrank::lowrank_expand_kernel<KS, CT>;
   constexpr int smem = nvfp4::lowrank::exp_smem_bytes<KS>();
   cudaError_t e = ensure_smem(kernel, smem, done, m);
   if (e != cudaSuccess) return e;
   const int64_t tiles_n = N / nvfp4::lowrank::kExpTile;
   const int64_t tiles = (M / nvfp4::lowrank::kExpTile) * tiles_n;
   const int grid = (int)std::min<int64_t>(tiles, sm_count);
-  kernel<<<grid, nvfp4::lowrank::kExpThreads, smem, s>>>(y, ldy, u, ldu, c, ldc, c_trans, (int32_t)tiles_n,
-                                                         (int32_t)tiles);
+  kernel<<<grid, nvfp4::lowrank::kExpThreads, smem, s>>>(y, ldy, u, ldu, c, ldc, (int32_t)tiles_n, (int32_t)tiles);
   return cudaGetLastError();
+}
+
+template <int KS>
+cudaError_t dispatch_expand(bool ct, uint16_t* y, int64_t ldy, const uint16_t* u, int64_t ldu, const uint16_t* c,
+                            int64_t ldc, int64_t M, int64_t N, int sm_count, cudaStream_t s) {
+  return ct ? launch_expand<KS, true>(y, ldy, u, ldu, c, ldc, M, N, sm_count, s)
+            : launch_expand<KS, false>(y, ldy, u, ldu, c, ldc, M, N, sm_count, s);
 }
 
 }  // namespace
@@ -774,13 +787,13 @@ nvfp4_status nvfp4_lowrank_project(const void* A, int64_t M, int64_t K, int64_t 
   const uint16_t* a = static_cast<const uint16_t*>(A);
   const uint16_t* b = static_cast<const uint16_t*>(B);
   uint16_t* u = static_cast<uint16_t*>(U);
-  const int bt = b_trans ? 1 : 0;
+  const bool bt = b_trans != 0;
   cudaError_t e;
   switch (rank / 8) {
-    case 2: e = launch_project<2>(a, lda, b, ldb, bt, M, K, u, ldu, s); break;
-    case 4: e = launch_project<4>(a, lda, b, ldb, bt, M, K, u, ldu, s); break;
-    case 6: e = launch_project<6>(a, lda, b, ldb, bt, M, K, u, ldu, s); break;
-    default: e = launch_project<8>(a, lda, b, ldb, bt, M, K, u, ldu, s); break;
+    case 2: e = dispatch_project<2>(bt, a, lda, b, ldb, M, K, u, ldu, s); break;
+    case 4: e = dispatch_project<4>(bt, a, lda, b, ldb, M, K, u, ldu, s); break;
+    case 6: e = dispatch_project<6>(bt, a, lda, b, ldb, M, K, u, ldu, s); break;
+    default: e = dispatch_project<8>(bt, a, lda, b, ldb, M, K, u, ldu, s); break;
   }
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "low-rank projection launch");
 }
@@ -806,14 +819,14 @@ nvfp4_status nvfp4_lowrank_expand_add(void* Y, int64_t M, int64_t N, int64_t ldy
   uint16_t* y = static_cast<uint16_t*>(Y);
   const uint16_t* u = static_cast<const uint16_t*>(U);
   const uint16_t* c = static_cast<const uint16_t*>(C);
-  const int ct = c_trans ? 1 : 0;
+  const bool ct = c_trans != 0;
   const int sms = dev->sm_count;
   cudaError_t e;
   switch (rank / 16) {
-    case 1: e = launch_expand<1>(y, ldy, u, ldu, c, ldc, ct, M, N, sms, s); break;
-    case 2: e = launch_expand<2>(y, ldy, u, ldu, c, ldc, ct, M, N, sms, s); break;
-    case 3: e = launch_expand<3>(y, ldy, u, ldu, c, ldc, ct, M, N, sms, s); break;
-    default: e = launch_expand<4>(y, ldy, u, ldu, c, ldc, ct, M, N, sms, s); break;
+    case 1: e = dispatch_expand<1>(ct, y, ldy, u, ldu, c, ldc, M, N, sms, s); break;
+    case 2: e = dispatch_expand<2>(ct, y, ldy, u, ldu, c, ldc, M, N, sms, s); break;
+    case 3: e = dispatch_expand<3>(ct, y, ldy, u, ldu, c, ldc, M, N, sms, s); break;
+    default: e = dispatch_expand<4>(ct, y, ldy, u, ldu, c, ldc, M, N, sms, s); break;
   }
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "low-rank expansion launch");
 }
