@@ -260,9 +260,13 @@ def lora_linear_fwd(x: torch.Tensor, wq_res_row: QTensor, l: torch.Tensor, r: to
     """nvfp4_lora_linear_fwd: Y = BF16(Q(X) Q(W_res)^T + BF16(X R^T) L^T); returns
     (Y, Xq_row, Xq_col or None).  l [N, r] and r [r, K] contiguous."""
     lib = _lib.load()
+    for t, nm in ((x, "x"), (l, "l"), (r, "r")):
+        _bf16_matrix(t, nm)
     M, K = x.shape
     N = wq_res_row.rows
     rank = l.shape[1]
+    if l.shape != (N, rank) or r.shape != (rank, K) or not (l.is_contiguous() and r.is_contiguous()):
+        raise ValueError("l must be a contiguous [N, r] and r a contiguous [r, K] BF16 matrix")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     if u is None:
@@ -284,9 +288,13 @@ def lora_linear_dgrad(dy: torch.Tensor, wq_res_col: QTensor, l: torch.Tensor, r:
     """nvfp4_lora_linear_dgrad: dX = BF16(Q_sr(dY) Q(W_res) + BF16(dY L) R); returns
     (dX, dYq_row, dYq_col or None)."""
     lib = _lib.load()
+    for t, nm in ((dy, "dy"), (l, "l"), (r, "r")):
+        _bf16_matrix(t, nm)
     M, N = dy.shape
     K = wq_res_col.rows
     rank = l.shape[1]
+    if l.shape != (N, rank) or r.shape != (rank, K) or not (l.is_contiguous() and r.is_contiguous()):
+        raise ValueError("l must be a contiguous [N, r] and r a contiguous [r, K] BF16 matrix")
     if out is None:
         out = torch.empty((M, K), dtype=torch.bfloat16, device=dy.device)
     if u is None:

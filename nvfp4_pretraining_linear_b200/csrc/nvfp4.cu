@@ -831,12 +831,37 @@ nvfp4_status nvfp4_lowrank_expand_add(void* Y, int64_t M, int64_t N, int64_t ldy
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "low-rank expansion launch");
 }
 
+}  // extern "C"
+
+namespace {
+
+// Arguments of the low-rank branch of a LoRA-SVD call, checked before the NVFP4 part
+// launches anything: rows x cols is the output (Y or dX), inner the projection's
+// contraction length (K or N).
+nvfp4_status lora_precheck(const nvfp4_tensor* Wq, const void* L, const void* R, int32_t rank, const void* U,
+                           int64_t rows, int64_t cols, int64_t inner, int64_t ld_in, int64_t ld_out) {
+  if (!rank_ok(rank)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
+  if (!Wq) return fail(NVFP4_ERR_INVALID_ARG, "the quantised residual weight is NULL");
+  if (!L || !R || !U) return fail(NVFP4_ERR_INVALID_ARG, "L, R or U is NULL");
+  if (!aligned16(L) || !aligned16(R) || !aligned16(U)) return fail(NVFP4_ERR_MISALIGNED, "L, R and U must be 16-byte aligned");
+  if (rows % nvfp4::lowrank::kExpTile || cols % nvfp4::lowrank::kExpTile || inner % nvfp4::lowrank::kProjKc ||
+      inner == 0)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "LoRA-SVD needs the output extents %% 128 and the inner extent %% 64");
+  if (ld_in % 8 || ld_out % 8) return fail(NVFP4_ERR_MISALIGNED, "input and output rows must be 16-byte aligned");
+  return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 nvfp4_status nvfp4_lora_linear_fwd(const void* X, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* Wq_res_row,
                                    const void* L, const void* R, int32_t rank, void* Y, int64_t ldy,
                                    nvfp4_tensor* Xq_row, nvfp4_tensor* Xq_col, uint32_t rht_signs, void* U,
                                    void* workspace, size_t workspace_bytes, void* stream) {
-  if (!rank_ok(rank)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
-  nvfp4_status st = nvfp4_linear_fwd(X, M, K, ldx, Wq_res_row, Y, ldy, NVFP4_OUT_BF16, Xq_row, Xq_col, rht_signs,
+  nvfp4_status st = lora_precheck(Wq_res_row, L, R, rank, U, M, Wq_res_row ? Wq_res_row->rows : 0, K, ldx, ldy);
+  if (st != NVFP4_OK) return st;
+  st = nvfp4_linear_fwd(X, M, K, ldx, Wq_res_row, Y, ldy, NVFP4_OUT_BF16, Xq_row, Xq_col, rht_signs,
                                      workspace, workspace_bytes, stream);
   if (st != NVFP4_OK) return st;
   const int64_t N = Wq_res_row->rows;
@@ -849,8 +874,9 @@ nvfp4_status nvfp4_lora_linear_dgrad(const void* dY, int64_t M, int64_t N, int64
                                      nvfp4_tensor* dYq_row, nvfp4_tensor* dYq_col, uint64_t seed, uint64_t offset,
                                      uint32_t rht_signs, void* U, void* workspace, size_t workspace_bytes,
                                      void* stream) {
-  if (!rank_ok(rank)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
-  nvfp4_status st = nvfp4_linear_dgrad(dY, M, N, ldy, Wq_res_col, dX, ldx, NVFP4_OUT_BF16, dYq_row, dYq_col, seed,
+  nvfp4_status st = lora_precheck(Wq_res_col, L, R, rank, U, M, Wq_res_col ? Wq_res_col->rows : 0, N, ldy, ldx);
+  if (st != NVFP4_OK) return st;
+  st = nvfp4_linear_dgrad(dY, M, N, ldy, Wq_res_col, dX, ldx, NVFP4_OUT_BF16, dYq_row, dYq_col, seed,
                                        offset, rht_signs, workspace, workspace_bytes, stream);
   if (st != NVFP4_OK) return st;
   const int64_t K = Wq_res_col->rows;

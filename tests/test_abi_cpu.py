@@ -148,3 +148,28 @@ def test_lowrank_argument_errors(lib):
     assert lib.nvfp4_lora_residual(y, 64, 128, 128, b, 16, a, 128, 32, u, 128, None) == 1     # ldl < rank
     assert lib.nvfp4_lora_residual(y + 4, 64, 128, 128, b, 32, a, 128, 32, u, 128, None) == 3
     assert lib.nvfp4_lora_residual(y, 64, 128, 128, b, 32, a, 128, 8, u, 128, None) == 2       # rank 8
+
+
+def test_lora_linear_checks_its_branch_before_launching(lib):
+    """Every argument error of the composed LoRA-SVD calls returns before the NVFP4 part
+    launches (no GPU here: reaching a launch would fail differently)."""
+    w = _tensor(256, 384)
+    x, l, r, u, y, ws = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000, 0x600000
+    xr = _tensor(256, 384)
+
+    def fwd(**kw):
+        a = dict(x=x, m=256, k=384, ldx=384, w=ctypes.byref(w), l=l, r=r, rank=32, y=y, ldy=256,
+                 xr=ctypes.byref(xr), u=u)
+        a.update(kw)
+        return lib.nvfp4_lora_linear_fwd(a["x"], a["m"], a["k"], a["ldx"], a["w"], a["l"], a["r"], a["rank"], a["y"],
+                                         a["ldy"], a["xr"], None, 0, a["u"], ws, 256, None)
+
+    assert fwd(rank=24) == 2
+    assert fwd(u=None) == 1
+    assert fwd(l=0x200008) == 3
+    assert fwd(m=192) == 2                      # output rows % 128
+    w352 = _tensor(256, 352)
+    assert fwd(k=352, ldx=352, w=ctypes.byref(w352)) == 2     # inner % 64
+    assert fwd(w=None) == 1
+    assert lib.nvfp4_lora_linear_dgrad(y, 256, 256, 256, ctypes.byref(_tensor(384, 256)), l, r, 32, x, 384,
+                                       ctypes.byref(_tensor(256, 256)), None, 1, 0, 0, None, ws, 256, None) == 1
