@@ -102,6 +102,14 @@ __global__ void __launch_bounds__(kResidualThreads) lora_residual_kernel(
 
 // ------------------------------------------------------------------ U = BF16(A B^T)
 
+// Two floats rounded to BF16 (nearest even, the hardware conversion) and packed, lo in
+// the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+  uint32_t out;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(hi), "f"(lo));
+  return out;
+}
+
 // Two BF16 values from shared memory packed as one MMA operand register, the first in
 // the low half (the operand element with the lower K index).
 __device__ __forceinline__ uint32_t pack_bf16_pair(const uint16_t* lo, const uint16_t* hi) {
@@ -195,10 +203,8 @@ __global__ void __launch_bounds__(kProjThreads) lowrank_project_kernel(const uin
 #pragma unroll
   for (int nt = 0; nt < RT; ++nt) {
     const int col = nt * 8 + 2 * t;
-    *reinterpret_cast<uint32_t*>(u + row * ldu + col) =
-        f32_to_bf16_bits(acc[nt][0]) | (f32_to_bf16_bits(acc[nt][1]) << 16);
-    *reinterpret_cast<uint32_t*>(u + (row + 8) * ldu + col) =
-        f32_to_bf16_bits(acc[nt][2]) | (f32_to_bf16_bits(acc[nt][3]) << 16);
+    *reinterpret_cast<uint32_t*>(u + row * ldu + col) = pack_bf16x2_rn(acc[nt][0], acc[nt][1]);
+    *reinterpret_cast<uint32_t*>(u + (row + 8) * ldu + col) = pack_bf16x2_rn(acc[nt][2], acc[nt][3]);
   }
 }
 
@@ -329,8 +335,8 @@ __global__ void __launch_bounds__(kExpThreads) lowrank_expand_kernel(uint16_t* _
         for (int h = 0; h < 2; ++h) {
           uint32_t* p = reinterpret_cast<uint32_t*>(&ys[wm + mt * 16 + g + 8 * h][wn + nt * 8 + 2 * t]);
           const uint32_t old = *p;
-          *p = f32_to_bf16_bits(__fadd_rn(bf16_lo(old), acc[mt][nt][2 * h])) |
-               (f32_to_bf16_bits(__fadd_rn(bf16_hi(old), acc[mt][nt][2 * h + 1])) << 16);
+          *p = pack_bf16x2_rn(__fadd_rn(bf16_lo(old), acc[mt][nt][2 * h]),
+                              __fadd_rn(bf16_hi(old), acc[mt][nt][2 * h + 1]));
         }
     __syncthreads();
     const int64_t m0 = (int64_t)(tile / tiles_n) * kExpTile, n0 = (int64_t)(tile % tiles_n) * kExpTile;
