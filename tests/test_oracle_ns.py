@@ -102,3 +102,15 @@ def test_converges_towards_polar_factor():
     assert np.linalg.norm(x - polar) / np.sqrt(m) < 0.16
     x0, _ = O.newton_schulz(g, 0)
     assert np.linalg.norm(x0 - polar) / np.sqrt(m) > 0.8                   # far before iterating
+
+
+def test_spectrum_generator_has_the_requested_singular_values():
+    """The seeded Newton-Schulz inputs: U diag(sigma) V^T with orthonormal factors, so the
+    singular values are the requested ones up to BF16 rounding of the entries."""
+    from nvfp4_pretraining_linear_b200 import synthetic
+    g = synthetic.spectrum(64, 160, 0.1, 1.0, seed=3).float().numpy().astype(np.float64)
+    sv = np.sort(np.linalg.svd(g, compute_uv=False))
+    want = np.linspace(0.1, 1.0, 64)
+    assert np.abs(sv - want).max() < 2e-3
+    again = synthetic.spectrum(64, 160, 0.1, 1.0, seed=3).float().numpy()
+    assert np.array_equal(again, g.astype(np.float32))                      # seeded
