@@ -188,10 +188,14 @@ def newton_schulz_workspace(m, n, device=None):
     return torch.empty(nbytes, dtype=torch.uint8, device=device if device is not None else "cuda")
 
 
-def newton_schulz(g: torch.Tensor, iters=5, *, normalize=True, out: Optional[torch.Tensor] = None,
+def newton_schulz(g: torch.Tensor, iters: int, *, normalize=True, out: Optional[torch.Tensor] = None,
                   norm: Optional[torch.Tensor] = None, workspace=None, stream=None):
     """nvfp4_newton_schulz on a BF16 [m, n] CUDA tensor: returns (X, ||G||_F as a 1-float
-    device tensor, or None without normalisation).  out may be g itself (in place)."""
+    device tensor, or None without normalisation).  out may be g itself (in place).
+
+    The cubic iteration multiplies a small singular value by about 1.5 per step, and
+    after the Frobenius normalisation the smallest ones start near 1/sqrt(m) of the
+    largest or below, so a few-thousand-row matrix takes about 12-16 steps."""
     lib = _lib.load()
     if g.dtype != torch.bfloat16 or not g.is_cuda or g.dim() != 2 or g.stride(1) != 1:
         raise ValueError("g must be a 2-D BF16 CUDA tensor with a contiguous last dimension")
