@@ -7,7 +7,7 @@ up-projection W[20480 x 5120] and the down-projection W[5120 x 20480]):
   quantise W (16x16 blocks, row + col layouts)
   fprop:  quantise X (row, RNE; col with 16x16 RHT, RNE)   + GEMM  Y  = X W^T
   dgrad:  quantise dY (row, SR; col with RHT + SR)          + GEMM  dX = dY W
-  wgrad:                                                      GEMM  dW = dY^T X
+  wgrad:                                                      GEMM  dW = dY^T X (FP32)
 Inputs are seeded synthetic BF16 tensors resident in HBM (each larger than the
 126 MB L2, so no flush is needed between steps).
 
@@ -17,9 +17,14 @@ Prints one JSON line (rank 0).  `value` is the step's NVFP4 GEMM work (6 GEMMs,
 activations and gradients copied from pinned host memory and the weight
 gradients read back, inside the timed region.  `roofline` covers the dominant
 kernel (the GEMM) against the FP4 tensor peak; `quantizer` the HBM side.
+`targets` times the two single-kernel goals alone: the GEMM at 16384^3 and the
+quantiser on the 16384^2 sweep tensor in its three modes.
 `--impl reference` times the CPU oracle on a bounded sample of the same step.
-Multi-GPU (torchrun): data parallel, each rank runs the full per-GPU step on its
-own tokens and the weight gradients are all-reduced with NCCL (weak scaling).
+Multi-GPU: data parallel, each rank runs the full per-GPU step on its own tokens
+and each linear's FP32 weight gradient is all-reduced with NCCL as soon as its
+wgrad is enqueued (weak scaling).  Under torchrun every rank reads RANK /
+WORLD_SIZE / LOCAL_RANK; `bench.py --gpus N` started as one process launches the
+N ranks itself.
 """
 
 import argparse
@@ -161,7 +166,7 @@ class Linear:
         self.dyq_col = QTensor.empty(N, M, SCALE_MMA, dev)
         self.y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         self.dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-        self.dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        self.dw = torch.empty((N, K), dtype=torch.float32, device=dev)   # FP32 partials, summed over ranks in FP32
 
     def gemm_flops(self):
         return 3 * 2.0 * self.M * self.N * self.K
@@ -185,10 +190,12 @@ def build_workload(device, rank):
     return [up, down]
 
 
-def instrumented_step(linears, ev, offset):
+def instrumented_step(linears, ev, offset, reducer=None):
     """One step from the quantiser and GEMM entry points, with CUDA events
     bracketing each GEMM and each quantiser call (same kernels, same order as
-    the linear_fwd / linear_dgrad / linear_wgrad entry points)."""
+    the linear_fwd / linear_dgrad / linear_wgrad entry points).  With a reducer
+    (data parallel), each linear's FP32 weight gradient starts its all-reduce as
+    soon as its wgrad is enqueued; the caller waits for them at the end."""
     from nvfp4_pretraining_linear_b200 import api
     for L in linears:
         ev.mark("q")
@@ -203,6 +210,8 @@ def instrumented_step(linears, ev, offset):
         ev.mark("g")
         api.gemm(L.dyq_row, L.wq_col, out=L.dx)
         api.gemm(L.dyq_col, L.xq_col, out=L.dw)
+        if reducer is not None:
+            reducer.start(L.dw)
     ev.mark("end")
 
 
@@ -229,7 +238,7 @@ class PhaseEvents:
         return out
 
 
-def public_step(linears, offset, ws):
+def public_step(linears, offset, reducer=None):
     """One step through the public linear entry points (as a user calls them)."""
     from nvfp4_pretraining_linear_b200 import api
     for L in linears:
@@ -238,6 +247,8 @@ def public_step(linears, offset, ws):
         api.linear_dgrad(L.dy, L.wq_col, seed=SR_SEED, offset=offset, rht_signs=RHT_SIGNS, out=L.dx,
                          dyq_row=L.dyq_row, dyq_col=L.dyq_col)
         api.linear_wgrad(L.dyq_col, L.xq_col, out=L.dw)
+        if reducer is not None:
+            reducer.start(L.dw)
 
 
 LAUNCHES_PER_LINEAR = 2 + 2 + 1 + 2 + 1 + 1   # W quant (amax+quant), X quant, fprop, dY quant, dgrad, wgrad
@@ -311,10 +322,10 @@ def run_reference(args):
         oracle_sample_step(state)
     dt = time.perf_counter() - t0
     value = flops * args.steps / dt / 1e12
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantise / f64 GEMM",
-            "data": "synthetic", "config": step_config(args.gpus),
+            "data": "synthetic", "config": step_config(world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -324,8 +335,66 @@ def run_reference(args):
 # ----------------------------------------------------------------------------- our arm
 
 
+def flushed_median_ms(fn, flush, warmup=3, steps=10):
+    """Median device time of fn() over `steps` launches, L2 flushed (a 256 MB write)
+    before each, CUDA events on the current stream."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
+
+
+TARGET_QUANT_MODES = {
+    "1d_rne": dict(emit_row=True, emit_col=True),
+    "1d_sr_rht": dict(emit_row=True, emit_col=True, stochastic=True, rht_row=True, rht_col=True, seed=SR_SEED,
+                      rht_signs=RHT_SIGNS),
+    "2d": dict(emit_row=True, emit_col=True, block_2d=True),
+}
+
+
+def measure_targets(fp4_burst, hbm):
+    """The two single-kernel targets, each timed alone (L2 flushed, medians of 10):
+    the NVFP4 GEMM at M = N = K = 16384 (BF16 output) against the dense FP4 peak, and
+    the quantiser on the 16384 x 16384 sweep tensor (Student-t nu = 3 x 0.1) in its
+    three modes with both layouts, two passes (amax, then quantise), against HBM."""
+    from nvfp4_pretraining_linear_b200 import api, synthetic as syn
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    n = 16384
+    a, b = syn.square(n, 2, device="cuda")
+    qa, _ = api.quantize(a)
+    qb, _ = api.quantize(b)
+    del a, b
+    c = torch.empty((n, n), dtype=torch.bfloat16, device="cuda")
+    ms = flushed_median_ms(lambda: api.gemm(qa, qb, out=c), flush)
+    tflops = 2.0 * n ** 3 / (ms * 1e-3) / 1e12
+    gemm = {"shape": [n, n, n], "ms": ms, "tflops": tflops, "frac_fp4_burst": tflops / fp4_burst,
+            "frac_fp4_nominal_9000": tflops / 9000.0, "target_frac_nominal": 0.60}
+    del qa, qb, c
+    x = syn.qsweep(n, device="cuda")
+    rq, cq = api.QTensor.empty(n, n), api.QTensor.empty(n, n)
+    quant = {}
+    for mode, kw in TARGET_QUANT_MODES.items():
+        ms = flushed_median_ms(lambda: api.quantize(x, out_row=rq, out_col=cq, **kw), flush)
+        gbs = n * n * 5.125 / (ms * 1e-3) / 1e9
+        quant[mode] = {"ms": ms, "gbs": gbs, "frac_hbm_measured": gbs / hbm, "frac_hbm_nominal_8000": gbs / 8000.0}
+    api.get_status()
+    return {"gemm_16384": gemm,
+            "quantizer_16384": dict(quant, bytes_per_elem="5.125 (two passes, row + col)", target_frac=0.70)}
+
+
 def run_ours(args):
     rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit("bench.py: --gpus %d but WORLD_SIZE is %d" % (args.gpus, world))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     group = None
@@ -334,13 +403,12 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
         group = dist.group.WORLD
-    from nvfp4_pretraining_linear_b200 import api, _lib
-    from nvfp4_pretraining_linear_b200.parallel import allreduce_grads, sr_offset
+    from nvfp4_pretraining_linear_b200 import api
+    from nvfp4_pretraining_linear_b200.parallel import GradReducer, sr_offset
 
     peaks, peak_src = load_peaks()
     linears = build_workload(device, rank)
-    ws = api.workspace(device)
-    offset = sr_offset(0, rank)
+    offset = sr_offset(0, rank, world)
 
     def barrier():
         torch.cuda.synchronize()
@@ -349,9 +417,9 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     def device_step(ev):
-        instrumented_step(linears, ev, offset)
-        if group is not None:
-            allreduce_grads([L.dw for L in linears], group)
+        reducer = GradReducer(group)
+        instrumented_step(linears, ev, offset, reducer)
+        reducer.wait()
 
     for _ in range(args.warmup):
         device_step(PhaseEvents(False))
@@ -382,7 +450,12 @@ def run_ours(args):
     qbytes = sum(L.quant_bytes() for L in linears)
     value = flops * world / (ms_step * 1e-3) / 1e12
 
-    fp4_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP4_OVER_BF16
+    # The timed region lasts well under a second, so the GEMM's roofline is the burst
+    # figure (a kernel timed alone, clocks at their maximum); the sustained figure (a
+    # seconds-long loop under the power cap) is reported beside it.
+    bf16_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    bf16_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    fp4_burst, fp4_sust = bf16_burst * FP4_OVER_BF16, bf16_sust * FP4_OVER_BF16
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
     quant_gbs = qbytes / (quant_ms * 1e-3) / 1e9
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -429,9 +502,9 @@ def run_ours(args):
             s_comp.wait_event(in_done[k])
             if i >= 2:
                 s_comp.wait_event(out_done[k])
-            public_step(sets[k], offset, ws)
-            if group is not None:
-                allreduce_grads([L.dw for L in sets[k]], group)
+            reducer = GradReducer(group)
+            public_step(sets[k], offset, reducer)
+            reducer.wait()
             comp_done[k].record(s_comp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[k])
@@ -449,30 +522,38 @@ def run_ours(args):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_value = flops * world / (e2e_ms / e2e_steps * 1e-3) / 1e12
+    del sets, host_in, host_out
 
     line = None
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3 block scales, fp32 accumulate), bf16 in/out",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3 block scales, fp32 accumulate), bf16 in/out, "
+                                          "fp32 weight gradients",
             "data": "synthetic",
             "config": step_config(world),
             "gpu_launches": LAUNCHES_PER_LINEAR * len(linears) * args.steps,
             "quantizer": {"gbs": quant_gbs, "frac_hbm": quant_gbs / hbm, "hbm_peak_gbs": hbm,
                           "peak_source": peak_src, "ms_per_step": quant_ms,
                           "bytes_per_elem": "4.5625 / layout-pair 5.125 (two-pass)"},
-            "gemm": {"tflops": gemm_tflops, "frac_fp4_peak": gemm_tflops / fp4_peak, "ms_per_step": gemm_ms},
-            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                         "frac": gemm_tflops / fp4_peak, "traffic": traffic,
+            "gemm": {"tflops": gemm_tflops, "frac_fp4_burst": gemm_tflops / fp4_burst,
+                     "frac_fp4_sustained": gemm_tflops / fp4_sust, "frac_fp4_nominal_9000": gemm_tflops / 9000.0,
+                     "ms_per_step": gemm_ms},
+            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_burst, "unit": "TFLOP/s",
+                         "frac": gemm_tflops / fp4_burst, "traffic": traffic,
                          "kernel": "nvfp4::gemm::gemm_kernel_pair",
-                         "peak_source": "%s bf16 sustained x %.0f (nominal FP4/BF16 ratio), of %s" % (
-                             peak_src, FP4_OVER_BF16, peak_src)},
+                         "peak_source": "%s bf16 burst x %.0f (nominal FP4/BF16 ratio), of %s; the timed region "
+                                        "is under a second" % (peak_src, FP4_OVER_BF16, peak_src)},
             "clocks": clock_info,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps, "path": "nvfp4_linear_fwd/dgrad/wgrad via the C ABI, pinned host buffers, "
                     "copies of neighbouring steps overlapped with compute on separate streams"},
         }
+        if world == 1 and not args.no_targets:
+            del linears
+            torch.cuda.empty_cache()
+            line["targets"] = measure_targets(fp4_burst, hbm)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = time_oracle(args.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -791,6 +872,19 @@ def run_layer(args):
     return 0
 
 
+def relaunch_with_ranks(args):
+    """`bench.py --gpus N` started as one process: start N ranks on this node with
+    torch.distributed.run (one per GPU) and return their exit status."""
+    import socket
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(args.gpus),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -800,6 +894,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-targets", action="store_true",
+                    help="skip the single-kernel target measurements (GEMM 16384^3, quantiser 16384^2)")
     ap.add_argument("--kernel", choices=["step", "gemm", "quantize", "chain", "ns", "layer", "lora"],
                     default="step",
                     help="step: the contract benchmark; gemm/quantize: one kernel on --shape; chain: GEMM then "
@@ -814,12 +910,16 @@ def main():
     ap.add_argument("--amax-in", action="store_true",
                     help="--kernel quantize: given maxima, no amax pass (2 B read + 0.5625 B per layout per element)")
     args = ap.parse_args()
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
     if args.kernel == "layer":
         return run_layer(args)
     if args.kernel != "step":
         return run_kernel(args)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch_with_ranks(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

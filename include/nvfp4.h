@@ -81,12 +81,23 @@ typedef struct {
 
 /* Quantiser options (recipe passage of the 12B NVFP4 page).
  *   stochastic : stochastic rounding of the elements of every emitted layout
- *                (gradients); otherwise round-to-nearest-even.  The random word
- *                of element i of a layout is word i%4 of Philox4x32-10 with key
- *                (seed lo32, seed hi32) and counter (i/4 lo32, i/4 hi32, tag,
- *                offset), tag 0 for the row layout and 1 for the col layout;
- *                the element rounds up iff (word >> 8) * 2^-24 is below its
- *                fractional position between the two neighbouring magnitudes.
+ *                (gradients); otherwise round-to-nearest-even.  Element i of a
+ *                layout (its linear index in the stored [rows x cols] order)
+ *                draws a 16-bit random integer n from Philox4x32-10 with key
+ *                (seed lo32, seed hi32):
+ *                  g = i / 4 (groups of four consecutive elements), and group g
+ *                  takes 32-bit word w = word g % 4 of the call with counter
+ *                  (g/4 lo32, g/4 hi32, tag, offset), tag 0 for the row layout
+ *                  and 1 for the col layout (one call per 16 elements);
+ *                  with e = i % 4:  n(e=0) = w[23:16] * 256 + w[7:0],
+ *                  n(e=1) = the 16-bit bit reversal of n(e=0),
+ *                  n(e=2) = w[31:24] * 256 + w[15:8],
+ *                  n(e=3) = the 16-bit bit reversal of n(e=2).
+ *                With lo <= |y| < hi the neighbouring magnitudes of the scaled
+ *                element y and f = (|y| - lo) / (hi - lo), the element rounds up
+ *                iff floor(f * 2^16) + n >= 2^16; |y| >= 6 gives 6, the sign is
+ *                kept.  The expected rounding error is below 2^-16 of a grid step
+ *                (a slight bias towards lo, from the floor).
  *   rht_row    : 16x16 random Hadamard transform along the blocks of the row layout.
  *   rht_col    : the same along the blocks of the col layout (the token axis of
  *                the weight-gradient operands).
@@ -120,7 +131,7 @@ typedef struct {
 int nvfp4_version(void);
 
 /* Bytes of caller workspace that nvfp4_quantize and the linear calls need
- * (device memory, 256-byte aligned; its contents need not be initialised). */
+ * (device memory, 16-byte aligned; its contents need not be initialised). */
 size_t nvfp4_workspace_size(void);
 
 /* Bytes of the scale buffer of an NVFP4 tensor of logical shape [rows x cols]
@@ -339,7 +350,12 @@ nvfp4_status nvfp4_check_conversions(unsigned long long* counts, uint64_t n_sr, 
 
 /* Synchronise `stream`, then report and clear any device-side error recorded
  * by this library's kernels on the current device since the last call
- * (NVFP4_ERR_TIMEOUT), or a pending CUDA error (NVFP4_ERR_CUDA). */
+ * (NVFP4_ERR_TIMEOUT), or a pending CUDA error (NVFP4_ERR_CUDA).
+ * A kernel whose bounded wait gives up (after 2 s) returns with its outputs
+ * partly written; the only sign of it is this call's status.  So the outputs of
+ * every call enqueued since the last clean status are valid only once this call
+ * returns NVFP4_OK: check it at least once per training step, before the step's
+ * results are used (for example before the optimizer update). */
 nvfp4_status nvfp4_get_status(void* stream);
 
 /* Text of the last non-OK status returned on the calling thread. */

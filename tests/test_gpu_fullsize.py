@@ -10,8 +10,8 @@ check takes what the oracle can compute one piece at a time:
   * GEMM outputs: every pair of sampled rows, C_ref[i, j] in FP64 from the oracle's
     dequantised rows, within the GEMM bound (BF16 output: plus one BF16 half-ulp).
 Workloads: the 12B hybrid MLP step that bench.py times (both linears, all six
-GEMMs), the 3B MLP step, the largest 3B-layer linear (QKV, 32768 tokens), and the
-16384^2 quantiser sweep tensor in its three modes.
+GEMMs), the 3B MLP step, the four linears of the 3B decoder layer (32768 tokens), and
+the 8192^2 and 16384^2 quantiser sweep tensors in their three modes.
 """
 
 import numpy as np
@@ -157,18 +157,22 @@ def test_mlp3b_step_fullsize():
     check_linear_step(bench.Linear("mlp3b", x, w, dy), offset=0, seed=200)
 
 
-def test_layer3b_qkv_fullsize():
-    """Largest linear of the 3B decoder layer at 32768 tokens: QKV 3072 -> 9216."""
-    x, w, dy = synthetic.layer3b_linear("qkv", device="cuda")
-    check_linear_step(bench.Linear("qkv", x, w, dy), offset=0, seed=300)
+@pytest.mark.parametrize("name", list(synthetic.LAYER3B["linears"]))
+def test_layer3b_linear_fullsize(name):
+    """The four linears of the 3B decoder layer at 32768 tokens: QKV 3072 -> 9216, O
+    3072 -> 3072, gate-up 3072 -> 16384, down 8192 -> 3072."""
+    x, w, dy = synthetic.layer3b_linear(name, device="cuda")
+    check_linear_step(bench.Linear(name, x, w, dy), offset=0, seed=300 + len(name))
+    torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("n", [8192, 16384])
 @pytest.mark.parametrize("mode", ["rne", "sr_rht", "2d"])
-def test_quantizer_sweep_16384(mode):
-    """Quantiser sweep tensor 16384 x 16384 (Student-t, nu = 3, x 0.1), with the col layout."""
-    x = synthetic.qsweep(16384, device="cuda")
+def test_quantizer_sweep_sampled(n, mode):
+    """Quantiser sweep tensor n x n (Student-t, nu = 3, x 0.1), with the col layout."""
+    x = synthetic.qsweep(n, device="cuda")
     xh = host_f32(x)
-    rows = sample_rows(16384, 400)
+    rows = sample_rows(n, 400)
     seed, offset, signs = 1234, 0, bench.RHT_SIGNS
     if mode == "2d":
         rq, cq = api.quantize(x, emit_row=True, emit_col=True, block_2d=True)
@@ -183,7 +187,7 @@ def test_quantizer_sweep_16384(mode):
                           offset=offset, rht_signs=signs)
     if sr:
         S_r = O.tensor_scale(np.float32(max(O.transformed_amax(xh[r0:r0 + 1024], True, signs)
-                                            for r0 in range(0, 16384, 1024))))
+                                            for r0 in range(0, n, 1024))))
         S_c = O.tensor_scale(rht_col_amax(xh, signs))
     else:
         S_r = S_c = O.tensor_scale(raw_amax(xh))

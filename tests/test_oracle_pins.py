@@ -426,3 +426,96 @@ def test_linear_layer_refs_compose():
     exact = dy.T.astype(np.float64) @ x.astype(np.float64)
     assert dw.shape == (N, K)
     assert np.linalg.norm(dw - exact) < 0.3 * np.linalg.norm(exact)
+
+
+# ---------------------------------------------------------------- recipe selection of the linear layer
+
+
+def _hadamard_tokens(v, signs):
+    """(1/4) H16 D applied to every 16-group along the last axis, from scipy's Sylvester
+    Hadamard matrix in FP64 (independent of the oracle's butterfly)."""
+    from scipy.linalg import hadamard
+    d = np.array([-1.0 if (signs >> j) & 1 else 1.0 for j in range(16)])
+    h = hadamard(16).astype(np.float64) / 4.0
+    g = np.asarray(v, dtype=np.float64).reshape(v.shape[0], -1, 16) * d
+    return (g @ h.T).reshape(v.shape)
+
+
+def _grid_neighbours(layout):
+    """Per element of a layout: its decoded value, and the magnitudes of the two grid
+    points around y = x / (s S) for the value x it encodes (from ml_dtypes' float4 cast)."""
+    import ml_dtypes
+    packed, scales, S = layout
+    codes = O.unpack_codes(packed)
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    mag = grid[codes & 7]
+    sv = np.repeat(O.e4m3_decode(scales).astype(np.float64), 16, axis=1)
+    return mag, sv, np.float64(S), ml_dtypes
+
+
+def _rel(a, b):
+    return np.linalg.norm(np.asarray(a, np.float64) - np.asarray(b, np.float64)) / np.linalg.norm(b)
+
+
+def test_linear_recipe_selection():
+    """Which operand gets which treatment in linear_fwd_ref / linear_dgrad_ref /
+    linear_wgrad_ref, against what the recipe passage of the 12B NVFP4 page fixes:
+    round-to-nearest for activations and weights, stochastic rounding for gradients
+    only, the 16x16 Hadamard transform on both wgrad operands along the tokens (so it
+    cancels in dY^T X), one 2D-quantised weight reused transposed by dgrad."""
+    import ml_dtypes
+    rng = np.random.default_rng(33)
+    M, K, N, signs = 64, 48, 32, 0x5A3C
+    x = _rand_tensor(rng, M, K)
+    x[5, 7] = F32(80.0)                                    # an outlier that the transform spreads
+    w = (rng.standard_normal((N, K)) * 0.02).astype(F32)
+    dy = (rng.standard_normal((M, N)) * 1e-3).astype(F32)
+    dy[9, 3] = F32(0.05)
+    wq = O.quantize_weight(w)
+    y, (xa, wb), xq = O.linear_fwd_ref(x, wq, rht_signs=signs)
+    dx, (da, wcol), dyq = O.linear_dgrad_ref(dy, wq, seed=1234, offset=0, rht_signs=signs)
+    dw, (ga, gb) = O.linear_wgrad_ref(dyq, xq)
+
+    # fprop reads X's and W's row layouts; dgrad dY's row layout and W's exact transpose
+    assert _rel(xa, x) < 0.1 and _rel(wb, w) < 0.2
+    assert _rel(da, dy) < 0.15
+    assert np.array_equal(wcol, wb.T)
+    wr_codes, wc_codes = O.unpack_codes(wq["row"][0]), O.unpack_codes(wq["col"][0])
+    assert np.array_equal(wc_codes, wr_codes.T)
+    assert np.array_equal(wq["col"][1], np.repeat(wq["row"][1][::16, :].T, 16, axis=0))
+
+    # wgrad reads both col layouts, each transformed along the tokens with the same signs
+    assert _rel(ga, _hadamard_tokens(dy.T, signs)) < 0.15
+    assert _rel(gb, _hadamard_tokens(x.T, signs)) < 0.1
+    assert _rel(ga, dy.T) > 0.5 and _rel(gb, x.T) > 0.5
+    assert _rel(dw, dy.T.astype(np.float64) @ x.astype(np.float64)) < 0.3
+
+    # the col layouts' tensor scales come from the transformed maxima
+    for q, v in ((xq, x), (dyq, dy)):
+        t_amax = np.abs(_hadamard_tokens(v.T, signs)).max()
+        assert abs(float(q["col"][2]) * 2688.0 / t_amax - 1.0) < 1e-6
+        assert abs(float(q["row"][2]) * 2688.0 / np.abs(v).max() - 1.0) < 1e-6
+
+    # round-to-nearest on X (both layouts) and W: each code is ml_dtypes' RNE cast of
+    # y = x / (s S) -- the activation codes do not depend on any seed
+    def rne_codes_match(layout, vals):
+        packed, scales, S = layout
+        sv = np.repeat(O.e4m3_decode(scales).astype(np.float32), 16, axis=1)
+        d = (sv * F32(S)).astype(F32)
+        r = np.where(d > 0, (F32(1.0) / np.where(d > 0, d, F32(1.0))).astype(F32), F32(0.0))
+        yv = (vals * r).astype(F32)
+        want = np.abs(np.clip(yv, -6, 6).astype(ml_dtypes.float4_e2m1fn).astype(np.float64))
+        got = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])[O.unpack_codes(packed) & 7]
+        return np.array_equal(got, want)
+
+    assert rne_codes_match(xq["row"], x)
+    assert rne_codes_match(xq["col"], _hadamard_tokens(x.T, signs).astype(F32)) or \
+        rne_codes_match(xq["col"], O.rht16(x.T.reshape(K, -1, 16), signs).reshape(K, M))
+    assert rne_codes_match(wq["row"], w)
+
+    # stochastic rounding on dY only: its codes change with the seed (both layouts),
+    # and some are not the nearest grid point
+    _, _, dyq2 = O.linear_dgrad_ref(dy, wq, seed=4321, offset=0, rht_signs=signs)
+    assert not np.array_equal(dyq["row"][0], dyq2["row"][0])
+    assert not np.array_equal(dyq["col"][0], dyq2["col"][0])
+    assert not rne_codes_match(dyq["row"], dy)
