@@ -590,8 +590,10 @@ def run_kernel(args):
         M, N, K = dims
         qa, _ = api.quantize(syn.normal((M, K), 1.0, seed=30, device="cuda"))
         qb, _ = api.quantize(syn.normal((N, K), 1.0, seed=31, device="cuda"))
-        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-        fn = lambda: api.gemm(qa, qb, out=out)  # noqa: E731
+        out = torch.empty((M, N), dtype=torch.float32 if args.out == "f32" else torch.bfloat16, device="cuda")
+        if args.accumulate:
+            out.zero_()
+        fn = lambda: api.gemm(qa, qb, out=out, accumulate=args.accumulate)  # noqa: E731
         work, unit = 2.0 * M * N * K, "TFLOP/s"
     else:
         R, C = dims
@@ -627,6 +629,8 @@ def run_kernel(args):
     ms = statistics.median(times)
     rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
     print(json.dumps({"kernel": args.kernel, "shape": dims, "mode": args.mode if args.kernel == "quantize" else None,
+                      "out": args.out if args.kernel == "gemm" else None,
+                      "accumulate": bool(args.accumulate) if args.kernel == "gemm" else None,
                       "amax_in": bool(args.amax_in) if args.kernel == "quantize" else None,
                       "ms": ms, "value": rate, "unit": unit, "steps": args.steps, "l2": "flushed (256 MB write)",
                       "clocks": clock_info}),
@@ -737,8 +741,10 @@ def run_ns(args, dims, flush):
 
 def run_lora(args, dims, flush):
     """The LoRA-SVD linear against the plain NVFP4 linear on one layer shape (M tokens,
-    N outputs, K inputs, --rank): fprop and dgrad each way, and the low-rank kernels
-    alone (residual, projection, expansion), L2 flushed before each timed call."""
+    N outputs, K inputs, --rank): fprop and dgrad each way (the LoRA-SVD calls add the
+    rank-r term inside the NVFP4 GEMM's accumulator), and the low-rank kernels alone
+    (residual, projections, the GEMM with and without its low-rank stage, the separate
+    expansion), L2 flushed before each timed call."""
     from nvfp4_pretraining_linear_b200 import api, synthetic as syn
     M, N, K = dims
     rank = args.rank
@@ -747,6 +753,7 @@ def run_lora(args, dims, flush):
     dy = syn.normal((M, N), 1e-3, seed=14, device="cuda")
     l = syn.normal((N, rank), 0.05, seed=15, device="cuda")
     r = syn.normal((rank, K), 0.05, seed=16, device="cuda")
+    rt = syn.normal((K, rank), 0.05, seed=17, device="cuda")       # R^T as the dgrad call takes it
     w_res = api.lora_residual(w, l, r)
     wq_row, wq_col = api.quantize_weight(w_res)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
@@ -776,9 +783,13 @@ def run_lora(args, dims, flush):
         "fwd_plain_ms": timed(lambda: api.linear_fwd(x, wq_row, **fkw)),
         "fwd_lora_ms": timed(lambda: api.lora_linear_fwd(x, wq_row, l, r, u=u, **fkw)),
         "dgrad_plain_ms": timed(lambda: api.linear_dgrad(dy, wq_col, **dkw)),
-        "dgrad_lora_ms": timed(lambda: api.lora_linear_dgrad(dy, wq_col, l, r, u=u, **dkw)),
+        "dgrad_lora_ms": timed(lambda: api.lora_linear_dgrad(dy, wq_col, l, rt, u=u, **dkw)),
         "residual_ms": timed(lambda: api.lora_residual(w, l, r, out=w_res)),
         "project_ms": timed(lambda: api.lowrank_project(x, r, out=u)),
+        "project_scaled_ms": timed(lambda: api.lowrank_project_scaled(x, r, xr.tensor_scale, wq_row.tensor_scale,
+                                                                      out=u)),
+        "gemm_plain_ms": timed(lambda: api.gemm(xr, wq_row, out=y)),
+        "gemm_lowrank_ms": timed(lambda: api.gemm_lowrank(xr, wq_row, u, l, out=y)),
         "expand_ms": timed(lambda: api.lowrank_expand_add(y, u, l)),
     }
     api.get_status()
@@ -907,6 +918,8 @@ def main():
     ap.add_argument("--rank", type=int, default=32, help="--kernel lora: rank of the BF16 branch")
     ap.add_argument("--shape", default="16384,16384,16384")
     ap.add_argument("--mode", choices=sorted(QUANT_MODES), default="grad")
+    ap.add_argument("--out", choices=["bf16", "f32"], default="bf16", help="--kernel gemm: output type")
+    ap.add_argument("--accumulate", action="store_true", help="--kernel gemm: add into the output")
     ap.add_argument("--amax-in", action="store_true",
                     help="--kernel quantize: given maxima, no amax pass (2 B read + 0.5625 B per layout per element)")
     args = ap.parse_args()

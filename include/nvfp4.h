@@ -266,7 +266,8 @@ nvfp4_status nvfp4_newton_schulz(const void* G, int64_t m, int64_t n, int64_t ld
  * residual; the page gives neither the rank nor the refresh of the factors, so
  * L [N x r] and R [r x K] (BF16, e.g. the top-r singular triplets of W) are the
  * caller's.  The residual takes the NVFP4 path (2D weight blocks); the rank-r part
- * stays in BF16 on the tensor cores (warp-level m16n8k16 MMA, FP32 accumulation).
+ * stays in BF16 and joins the NVFP4 GEMM's FP32 accumulator on the tensor cores
+ * (nvfp4_gemm_lowrank); the building blocks below also serve it separately.
  * Every call here takes r in {16, 32, 48, 64}. */
 
 /* W_res = BF16(fl32(W - s)), s = sum_j L[n][j] R[j][k] accumulated in FP32 in
@@ -286,6 +287,29 @@ nvfp4_status nvfp4_lora_residual(const void* W, int64_t N, int64_t K, int64_t ld
 nvfp4_status nvfp4_lowrank_project(const void* A, int64_t M, int64_t K, int64_t lda, const void* B, int64_t ldb,
                                    int32_t b_trans, int32_t rank, void* U, int64_t ldu, void* stream);
 
+/* nvfp4_lowrank_project with the sums divided by g = fl32(*scale_a * *scale_b) before
+ * the rounding: U' = BF16(fl32(fl32(A B^T) * fl32(1 / g))).  scale_a and scale_b are
+ * device floats, typically the tensor scales of the two operands of the NVFP4 GEMM
+ * that U' joins (nvfp4_gemm_lowrank multiplies its accumulator by that g). */
+nvfp4_status nvfp4_lowrank_project_scaled(const void* A, int64_t M, int64_t K, int64_t lda, const void* B,
+                                          int64_t ldb, int32_t b_trans, int32_t rank, const float* scale_a,
+                                          const float* scale_b, void* U, int64_t ldu, void* stream);
+
+/* NVFP4 GEMM with a rank-r BF16 term inside its accumulator (the LoRA-SVD linear
+ * above, fused; "Full-Stack FP4", linear-projection passage):
+ *   C[m][n] = BF16(g * (sum_k A[m][k] B[n][k] + sum_j U[m][j] V[n][j])),  g = fl32(S_A S_B)
+ * where the first sum is the block-scaled NVFP4 product (as in nvfp4_gemm) and the
+ * second a BF16 product on the tensor cores, both accumulated in the same FP32
+ * accumulator; each output tile ends with one extra pipeline stage that loads its
+ * U and V rows and issues r/16 BF16 MMAs.  A [M x K], B [N x K] as for nvfp4_gemm;
+ * U [M x r], V [N x r] BF16 device matrices, row strides ldu, ldv (elements);
+ * C [M x N] BF16, row stride ldc.  U is usually nvfp4_lowrank_project_scaled(...)
+ * with the tensor scales of A and B, so that g U V^T is the plain low-rank product.
+ * Requires the conditions of nvfp4_gemm, M >= 256, r in {16, 32, 48, 64}, 16-byte
+ * aligned U and V rows. */
+nvfp4_status nvfp4_gemm_lowrank(const nvfp4_tensor* A, const nvfp4_tensor* B, const void* U, int64_t ldu,
+                                const void* V, int64_t ldv, int32_t rank, void* C, int64_t ldc, void* stream);
+
 /* Y <- BF16(fl32(Y + U C^T)) in place: Y [M x N] BF16 (row stride ldy); U [M x r];
  * C [N x r] (c_trans == 0, row stride ldc) or given as its transpose [r x N]
  * (c_trans != 0).  FP32 accumulation of the product.  Requires M % 128 == 0,
@@ -293,22 +317,27 @@ nvfp4_status nvfp4_lowrank_project(const void* A, int64_t M, int64_t K, int64_t 
 nvfp4_status nvfp4_lowrank_expand_add(void* Y, int64_t M, int64_t N, int64_t ldy, const void* U, int64_t ldu,
                                       const void* C, int64_t ldc, int32_t c_trans, int32_t rank, void* stream);
 
-/* LoRA-SVD fprop: Y = BF16(fl32(Y4 + U L^T)) with Y4 = nvfp4_linear_fwd(X, Wq_res_row)
- * (BF16) and U = BF16(X R^T).  Arguments as nvfp4_linear_fwd, plus L [N x r] and
- * R [r x K] contiguous BF16 device matrices and U, caller scratch of M * r BF16
- * (16-byte aligned).  Y is BF16.  Work: the NVFP4 fprop, then one pass over X for U
- * and one read-modify-write pass over Y. */
+/* LoRA-SVD fprop: X is quantised as in nvfp4_linear_fwd, U' = BF16(X R^T / g) with
+ * g = fl32(S_X S_W) (nvfp4_lowrank_project_scaled), and
+ *   Y = BF16(g * (Q(X) Q(W_res)^T + U' L^T))   in one nvfp4_gemm_lowrank.
+ * Arguments as nvfp4_linear_fwd, plus L [N x r] and R [r x K] contiguous BF16 device
+ * matrices and U, caller scratch of M * r BF16 (16-byte aligned).  Y is BF16.
+ * Requires M >= 256 besides the conditions of nvfp4_linear_fwd.  Work: the
+ * quantisation of X, one pass over X for U', and the GEMM. */
 nvfp4_status nvfp4_lora_linear_fwd(const void* X, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* Wq_res_row,
                                    const void* L, const void* R, int32_t rank, void* Y, int64_t ldy,
                                    nvfp4_tensor* Xq_row, nvfp4_tensor* Xq_col, uint32_t rht_signs, void* U,
                                    void* workspace, size_t workspace_bytes, void* stream);
 
-/* LoRA-SVD dgrad: dX = BF16(fl32(dX4 + U R)) with dX4 = nvfp4_linear_dgrad(dY,
- * Wq_res_col) (BF16) and U = BF16(dY L).  Arguments as nvfp4_linear_dgrad, plus L,
- * R and U as for nvfp4_lora_linear_fwd.  The weight gradient is that of W itself:
- * nvfp4_linear_wgrad, unchanged. */
+/* LoRA-SVD dgrad: dY is quantised as in nvfp4_linear_dgrad, U' = BF16(dY L / g) with
+ * g = fl32(S_dY S_W), and
+ *   dX = BF16(g * (Q_sr(dY) Q(W_res) + U' R))   in one nvfp4_gemm_lowrank.
+ * Arguments as nvfp4_linear_dgrad, plus L [N x r] contiguous, Rt = R^T [K x r]
+ * contiguous (the tensor cores read R with its rank index contiguous), and U as for
+ * nvfp4_lora_linear_fwd.  Requires M >= 256.  The weight gradient is that of W
+ * itself: nvfp4_linear_wgrad, unchanged. */
 nvfp4_status nvfp4_lora_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ldy, const nvfp4_tensor* Wq_res_col,
-                                     const void* L, const void* R, int32_t rank, void* dX, int64_t ldx,
+                                     const void* L, const void* Rt, int32_t rank, void* dX, int64_t ldx,
                                      nvfp4_tensor* dYq_row, nvfp4_tensor* dYq_col, uint64_t seed, uint64_t offset,
                                      uint32_t rht_signs, void* U, void* workspace, size_t workspace_bytes,
                                      void* stream);

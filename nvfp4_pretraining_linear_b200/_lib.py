@@ -87,6 +87,10 @@ SIGNATURES = {
                                       c_int32, c_void_p, c_int64, c_void_p]),
     "nvfp4_lowrank_project": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_int32, c_int32,
                                         c_void_p, c_int64, c_void_p]),
+    "nvfp4_lowrank_project_scaled": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_int32,
+                                                c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_void_p]),
+    "nvfp4_gemm_lowrank": (c_int32, [T_P, T_P, c_void_p, c_int64, c_void_p, c_int64, c_int32, c_void_p, c_int64,
+                                      c_void_p]),
     "nvfp4_lowrank_expand_add": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_void_p, c_int64,
                                            c_int32, c_int32, c_void_p]),
     "nvfp4_lora_linear_fwd": (c_int32, [c_void_p, c_int64, c_int64, c_int64, T_P, c_void_p, c_void_p, c_int32,

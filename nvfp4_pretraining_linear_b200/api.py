@@ -247,6 +247,36 @@ def lowrank_project(a: torch.Tensor, b: torch.Tensor, *, b_trans=False, out: Opt
     return out
 
 
+def lowrank_project_scaled(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor, *,
+                           b_trans=False, out: Optional[torch.Tensor] = None, stream=None):
+    """nvfp4_lowrank_project_scaled: U' = BF16(A B^T / g), g = fl32(scale_a * scale_b) (two
+    1-float device tensors, e.g. the tensor scales of an NVFP4 GEMM's operands)."""
+    lib = _lib.load()
+    _bf16_matrix(a, "a")
+    _bf16_matrix(b, "b")
+    M, K = a.shape
+    rank = b.shape[1] if b_trans else b.shape[0]
+    if out is None:
+        out = torch.empty((M, rank), dtype=torch.bfloat16, device=a.device)
+    _lib.check(lib.nvfp4_lowrank_project_scaled(a.data_ptr(), M, K, a.stride(0), b.data_ptr(), b.stride(0),
+                                                int(b_trans), rank, scale_a.data_ptr(), scale_b.data_ptr(),
+                                                out.data_ptr(), out.stride(0), _stream_ptr(stream)))
+    return out
+
+
+def gemm_lowrank(A: QTensor, B: QTensor, u: torch.Tensor, v: torch.Tensor, out: Optional[torch.Tensor] = None,
+                 stream=None):
+    """nvfp4_gemm_lowrank: BF16 C = g (A . B^T + U V^T), g = S_A S_B; u [M, r], v [N, r] BF16."""
+    lib = _lib.load()
+    _bf16_matrix(u, "u")
+    _bf16_matrix(v, "v")
+    if out is None:
+        out = torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=A.codes.device)
+    _lib.check(lib.nvfp4_gemm_lowrank(A.struct(), B.struct(), u.data_ptr(), u.stride(0), v.data_ptr(), v.stride(0),
+                                      u.shape[1], out.data_ptr(), out.stride(0), _stream_ptr(stream)))
+    return out
+
+
 def lowrank_expand_add(y: torch.Tensor, u: torch.Tensor, c: torch.Tensor, *, c_trans=False, stream=None):
     """nvfp4_lowrank_expand_add: Y <- BF16(Y + U C^T) in place, C [N, r] (or [r, N] with c_trans)."""
     lib = _lib.load()
@@ -261,8 +291,9 @@ def lowrank_expand_add(y: torch.Tensor, u: torch.Tensor, c: torch.Tensor, *, c_t
 
 def lora_linear_fwd(x: torch.Tensor, wq_res_row: QTensor, l: torch.Tensor, r: torch.Tensor, *, save_col=True,
                     rht_signs=0, out=None, u=None, xq_row=None, xq_col=None, stream=None):
-    """nvfp4_lora_linear_fwd: Y = BF16(Q(X) Q(W_res)^T + BF16(X R^T) L^T); returns
-    (Y, Xq_row, Xq_col or None).  l [N, r] and r [r, K] contiguous."""
+    """nvfp4_lora_linear_fwd: Y = BF16(g (Q(X) Q(W_res)^T + U' L^T)), U' = BF16(X R^T / g),
+    g = S_X S_W, in one GEMM; returns (Y, Xq_row, Xq_col or None).  l [N, r] and r [r, K]
+    contiguous."""
     lib = _lib.load()
     for t, nm in ((x, "x"), (l, "l"), (r, "r")):
         _bf16_matrix(t, nm)
@@ -287,18 +318,19 @@ def lora_linear_fwd(x: torch.Tensor, wq_res_row: QTensor, l: torch.Tensor, r: to
     return out, xq_row, (xq_col if save_col else None)
 
 
-def lora_linear_dgrad(dy: torch.Tensor, wq_res_col: QTensor, l: torch.Tensor, r: torch.Tensor, *, seed, offset=0,
+def lora_linear_dgrad(dy: torch.Tensor, wq_res_col: QTensor, l: torch.Tensor, rt: torch.Tensor, *, seed, offset=0,
                       save_col=True, rht_signs=0, out=None, u=None, dyq_row=None, dyq_col=None, stream=None):
-    """nvfp4_lora_linear_dgrad: dX = BF16(Q_sr(dY) Q(W_res) + BF16(dY L) R); returns
-    (dX, dYq_row, dYq_col or None)."""
+    """nvfp4_lora_linear_dgrad: dX = BF16(g (Q_sr(dY) Q(W_res) + U' R)), U' = BF16(dY L / g),
+    g = S_dY S_W, in one GEMM; returns (dX, dYq_row, dYq_col or None).  l [N, r] and
+    rt = R^T [K, r] contiguous."""
     lib = _lib.load()
-    for t, nm in ((dy, "dy"), (l, "l"), (r, "r")):
+    for t, nm in ((dy, "dy"), (l, "l"), (rt, "rt")):
         _bf16_matrix(t, nm)
     M, N = dy.shape
     K = wq_res_col.rows
     rank = l.shape[1]
-    if l.shape != (N, rank) or r.shape != (rank, K) or not (l.is_contiguous() and r.is_contiguous()):
-        raise ValueError("l must be a contiguous [N, r] and r a contiguous [r, K] BF16 matrix")
+    if l.shape != (N, rank) or rt.shape != (K, rank) or not (l.is_contiguous() and rt.is_contiguous()):
+        raise ValueError("l must be a contiguous [N, r] and rt a contiguous [K, r] BF16 matrix")
     if out is None:
         out = torch.empty((M, K), dtype=torch.bfloat16, device=dy.device)
     if u is None:
@@ -310,7 +342,7 @@ def lora_linear_dgrad(dy: torch.Tensor, wq_res_col: QTensor, l: torch.Tensor, r:
     ws = workspace(dy.device, stream)
     dc = dyq_col.struct() if save_col else None
     _lib.check(lib.nvfp4_lora_linear_dgrad(dy.data_ptr(), M, N, dy.stride(0), wq_res_col.struct(), l.data_ptr(),
-                                           r.data_ptr(), rank, out.data_ptr(), out.stride(0), dyq_row.struct(), dc,
+                                           rt.data_ptr(), rank, out.data_ptr(), out.stride(0), dyq_row.struct(), dc,
                                            seed, offset, rht_signs, u.data_ptr(), ws.data_ptr(), ws.numel(),
                                            _stream_ptr(stream)))
     return out, dyq_row, (dyq_col if save_col else None)

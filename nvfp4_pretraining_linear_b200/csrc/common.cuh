@@ -135,6 +135,21 @@ __device__ __forceinline__ uint32_t e2m1x4_rs(float y0, float y1, float y2, floa
   return out;
 }
 
+// Two non-negative floats -> two E4M3 bytes (a in bits 0-7, b in bits 8-15), round to
+// nearest even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3x2_encode_hw(float a, float b) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(b), "f"(a));
+  return out;
+}
+
+// max(a, b, c) in one instruction (sm_100 three-input minimum / maximum).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Non-negative float -> E4M3 byte, round to nearest even, saturating at 448.
 __device__ __forceinline__ uint32_t e4m3_encode_hw(float v) {
   uint16_t out;
@@ -155,6 +170,20 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
     const uint64_t p0 = (uint64_t)0xD2511F53u * c.x;
     const uint64_t p1 = (uint64_t)0xCD9E8D57u * c.z;
     c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ k0, (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ k1, (uint32_t)p0);
+  }
+  return c;
+}
+
+// The same generator with its round keys precomputed (rk[r] = k0 + r * 0x9E3779B9,
+// rk[10 + r] = k1 + r * 0xBB67AE85, modulo 2^32): when rk lives in a kernel's
+// parameter space, a round is two wide multiplies and two three-input XORs.
+__device__ __forceinline__ uint4 philox4x32_10_rk(uint4 c, const uint32_t* rk) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c.x;
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * c.z;
+    c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ rk[r], (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ rk[10 + r],
+                   (uint32_t)p0);
   }
   return c;
 }

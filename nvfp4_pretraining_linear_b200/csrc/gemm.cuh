@@ -74,6 +74,10 @@ struct Params {
   int32_t accumulate;
   unsigned* amax_acc;       // nullptr, or 2 words receiving max|C| and max|RHT16 col(C)| (float bits)
   uint32_t rht_signs;       // sign mask of that transform
+  int64_t skip_stage;       // fault injection (pair kernel): CTA pair 0 never loads its K-stage
+                            // number skip_stage (counted over all its tiles); -1: off
+  int32_t lr_ksteps;        // pair kernel: BF16 MMAs (K = 16 each) of the low-rank stage that ends
+                            // every tile, accumulating U V^T into the same accumulator; 0: none
 };
 
 // Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), UE4M3
@@ -571,6 +575,13 @@ __device__ __forceinline__ uint32_t scale_pack_bf16x2(uint32_t lo, uint32_t hi, 
   return out;
 }
 
+// Two FP32 values rounded to BF16 (nearest even) and packed, a in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  uint32_t out;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(b), "f"(a));
+  return out;
+}
+
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
@@ -594,15 +605,35 @@ __host__ __device__ constexpr uint32_t make_idesc_pair() {
   return (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 }
 
+// Instruction descriptor of the low-rank stage's MMA, kind::f16: BF16 A and B (format 1),
+// FP32 accumulator (format 1), K-major, M = 256, N = 256, K = 16.
+__host__ __device__ constexpr uint32_t make_idesc_pair_bf16() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma_pair_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, 1, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc)
+      : "memory");
+}
+
 __device__ __forceinline__ TileCoord pair_tile_coord(const Params& p, int32_t t) {
   // p.num_m counts 256-row tiles here
   return tile_coord(p, t);
 }
 
+// Output modes of the pair kernel's epilogue (one instantiation each).
+enum EpiMode : int { EPI_BF16 = 0, EPI_BF16_ACC = 1, EPI_F32 = 2, EPI_F32_ACC = 3 };
+
+template <int EPI>
 __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     gemm_kernel_pair(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                      const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
-                     const __grid_constant__ CUtensorMap tma_c, const Params p) {
+                     const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ CUtensorMap tma_u,
+                     const __grid_constant__ CUtensorMap tma_v, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t smem_base = smem_u32(smem);
@@ -662,6 +693,8 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
 
   const int32_t num_tiles = p.num_m * p.num_n;
   const int32_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  // stages per tile: the NVFP4 K-stages, then the low-rank stage when there is one
+  const int tile_stages = p.num_k_stages + (p.lr_ksteps ? 1 : 0);
   const uint32_t leader_full0 = map_to_cta(full_bar(0), 0);
   const uint32_t leader_acc_empty = map_to_cta(acc_empty, 0);
 
@@ -675,22 +708,40 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       // tile are prefetched into L2: every pair starts its next tile at about the same
       // time, and without this those first loads all miss L2 at once.
       const int pf_n = min(P_PREFETCH, p.num_k_stages);
+      int64_t q = 0;                                    // stage sequence number over this pair's tiles
       for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
         const TileCoord tc = pair_tile_coord(p, t);
         const bool has_next = t + num_pairs < num_tiles;
         const TileCoord nc = pair_tile_coord(p, has_next ? t + num_pairs : t);
-        for (int ks = 0; ks < p.num_k_stages; ++ks) {
+        for (int ks = 0; ks < tile_stages; ++ks, ++q) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
+          if (pair == 0 && q == p.skip_stage) {
+            // fault injection: neither CTA loads this stage and the leader never arms its
+            // barrier, so the MMA issuers' bounded wait on it expires (kErrTimeout) and
+            // every role winds down; nothing is in flight for this stage
+            if (++stage == P_STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           const uint32_t fb = leader_full0 + 8u * stage;
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * P_AB_BYTES);
-          const int32_t kx = ks * BK_BYTES;
-          tma_load_2d_pair(a_smem(stage), &tma_a, kx, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
-          tma_load_2d_pair(b_smem(stage), &tma_b, kx, tc.n_blk * BN + (int32_t)rank * 128, fb);
+          if (ks == p.num_k_stages) {
+            // low-rank stage: 128 rows x 64 BF16 of U (this CTA's A rows) and of V (its half
+            // of the B rows), zero-filled past the rank
+            tma_load_2d_pair(a_smem(stage), &tma_u, 0, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
+            tma_load_2d_pair(b_smem(stage), &tma_v, 0, tc.n_blk * BN + (int32_t)rank * 128, fb);
+          } else {
+            const int32_t kx = ks * BK_BYTES;
+            tma_load_2d_pair(a_smem(stage), &tma_a, kx, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
+            tma_load_2d_pair(b_smem(stage), &tma_b, kx, tc.n_blk * BN + (int32_t)rank * 128, fb);
+          }
           const int pf = ks - (p.num_k_stages - pf_n);
-          if (has_next && pf >= 0) {
+          if (has_next && pf >= 0 && pf < pf_n) {
             tma_prefetch_2d(&tma_a, pf * BK_BYTES, nc.m_blk * P_BM + (int32_t)rank * 128);
             tma_prefetch_2d(&tma_b, pf * BK_BYTES, nc.n_blk * BN + (int32_t)rank * 128);
           }
@@ -720,9 +771,9 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       int stage = 0, slot = 0;                          // operand stage, scale slot (q % P_SF_SLOTS)
       uint32_t phase = 0, acc_phase = 0;
       const int64_t my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
-      const int64_t total = my_tiles * p.num_k_stages;
+      const int64_t total = my_tiles * tile_stages;
       for (int32_t t = pair; t < num_tiles; t += num_pairs) {
-        for (int ks = 0; ks < p.num_k_stages; ++ks, ++q) {
+        for (int ks = 0; ks < tile_stages; ++ks, ++q) {
           if ((q & 1) == me) {
             if (ok && ks == 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag));
             if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(full_bar(stage), phase, abort_flag));
@@ -730,14 +781,21 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             if (q > 0) asm volatile("bar.sync %0, 64;" ::"r"(me == 0 ? 2 : 1) : "memory");
             tc_fence_after();
             if (ok && lane == 0) {
-              const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
-              const uint32_t sfa = tmem + P_SF_COL0 + P_SF_SLOT_COLS * slot, sfb = sfa + 16;
-              for (int kk = 0; kk < atoms; ++kk)
-                tc_mma_pair(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * (MMA_K / 2)),
-                            sw128_desc(b_smem(stage) + kk * (MMA_K / 2)), idesc, (ks | kk) != 0 ? 1u : 0u,
-                            sfa + 4 * kk, sfb + 8 * kk);
+              if (ks == p.num_k_stages) {
+                // low-rank stage: U V^T (BF16, K = 16 per MMA) into the same accumulator
+                for (int kk = 0; kk < p.lr_ksteps; ++kk)
+                  tc_mma_pair_bf16(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * 32),
+                                   sw128_desc(b_smem(stage) + kk * 32), make_idesc_pair_bf16());
+              } else {
+                const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
+                const uint32_t sfa = tmem + P_SF_COL0 + P_SF_SLOT_COLS * slot, sfb = sfa + 16;
+                for (int kk = 0; kk < atoms; ++kk)
+                  tc_mma_pair(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * (MMA_K / 2)),
+                              sw128_desc(b_smem(stage) + kk * (MMA_K / 2)), idesc, (ks | kk) != 0 ? 1u : 0u,
+                              sfa + 4 * kk, sfb + 8 * kk);
+              }
               tc_commit_pair(empty_bar(stage));
-              if (ks == p.num_k_stages - 1) tc_commit_pair(acc_full);
+              if (ks == tile_stages - 1) tc_commit_pair(acc_full);
             }
             tc_fence_before();
             __syncwarp();
@@ -773,9 +831,9 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
         const TileCoord tc = pair_tile_coord(p, t);
         const bool has_next = t + num_pairs < num_tiles;
         const TileCoord nc = pair_tile_coord(p, has_next ? t + num_pairs : t);
-        for (int ks = 0; ks < p.num_k_stages; ++ks) {
+        for (int ks = 0; ks < tile_stages; ++ks) {
           const int pf = ks - (p.num_k_stages - pf_n);
-          if (has_next && pf >= 0) {             // the next tile's scales, as for the operands
+          if (has_next && pf >= 0 && pf < pf_n) {  // the next tile's scales, as for the operands
             const int32_t pk = pf * (BK / MMA_K);
             tma_prefetch_2d(&tma_sfa, 0, (int32_t)((nc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + pk);
             tma_prefetch_2d(&tma_sfb, 0, (int32_t)((nc.n_blk * 2) * p.sf_kgroups) + pk);
@@ -786,6 +844,16 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             break;
           }
           const uint32_t sb = sf_full_bar(j);
+          if (ks == p.num_k_stages) {
+            // the low-rank stage has no block scales: complete the slot's phase without
+            // loading, so the writers' and issuers' stage counts stay in step
+            mbar_arrive(sb);
+            if (++j == P_SF_STAGES) {
+              j = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           mbar_arrive_expect_tx(sb, (uint32_t)P_SF_BYTES);
           const int32_t katom = ks * (BK / MMA_K);
           tma_load_2d(sfa_smem(j), &tma_sfa, 0, (int32_t)((tc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + katom,
@@ -821,7 +889,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     int64_t q = 0;
     bool ok = true;
     for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
-      for (int ks = 0; ks < p.num_k_stages; ++ks, ++q) {
+      for (int ks = 0; ks < tile_stages; ++ks, ++q) {
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(sf_full_bar(j), sf_phase, abort_flag));
         if (!ok) break;
         const uint8_t* sa = smem + P_SF_OFFSET + j * P_SF_BYTES + lane * 16;
@@ -875,53 +943,90 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    // Output paths, by output type:
+    //   BF16            scale and round while reading the accumulator (64 registers for
+    //                   the warp's 128 columns), release it, then two 32 x 64 TMA stores;
+    //   BF16 + C        the warp's 128 old values of C are loaded into registers before
+    //                   the accumulator is ready (while the main loop runs), added while
+    //                   reading it (BF16(fl32(fl32(acc * g) + C))), then as BF16;
+    //   FP32            four 32 x 32 boxes, each staged and stored as soon as read; the
+    //                   accumulator is released after the last read;
+    //   FP32 + C        32 columns at a time, direct loads and stores.
+    // Staging uses the warp's own 4 KB of shared memory, rows of 128 bytes with the
+    // 128-byte swizzle (lane r puts 16-byte chunk c of its row at chunk c ^ (r % 8),
+    // which keeps each quarter-warp on distinct banks); whole-line bulk stores instead
+    // of per-row 16-byte stores keep the output burst at every tile change off the
+    // operand loads.
     const int ew = warp - EPI_WARP0;
     const int quarter = warp & 3;
     const int half = ew >> 2;
     const int row_in_tile = (int)rank * 128 + quarter * 32 + lane;
     const float g = __fmul_rn(__fmul_rn(*p.scale_a, *p.scale_b), p.alpha);
-    const bool packed = !p.out_f32 && !p.accumulate;
+    constexpr bool bf16_out = EPI == EPI_BF16 || EPI == EPI_BF16_ACC;
+    constexpr bool accumulate = EPI == EPI_BF16_ACC || EPI == EPI_F32_ACC;
+    uint8_t* stg = smem + P_EPI_OFFSET + ew * P_EPI_BOX_BYTES;
     uint32_t acc_phase = 0;
     for (int32_t t = pair; t < num_tiles; t += num_pairs) {
       const TileCoord tc = pair_tile_coord(p, t);
       const int n_cols = min(BN, p.N - tc.n_blk * BN);
       const int64_t m = (int64_t)tc.m_blk * P_BM + row_in_tile;
-      const bool mine = n_cols > half * 128;
+      const bool mine = n_cols > half * 128;          // N % 128 == 0: a half is whole or absent
+      const int64_t n0 = (int64_t)tc.n_blk * BN + half * 128;
+      const int32_t m0 = tc.m_blk * P_BM + (int32_t)rank * 128 + quarter * 32;
+      const bool rows_in = m0 < p.M;                  // M % 128 == 0: the warp's 32 rows are all in or all out
+      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + half * 128;
+      uint32_t pk[64];                                // BF16 pairs: old C, then the result
+      if constexpr (EPI == EPI_BF16_ACC) {
+        if (mine && rows_in) {
+          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.C) + m * p.ldc + n0);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const uint4 v = src[q];
+            pk[4 * q] = v.x, pk[4 * q + 1] = v.y, pk[4 * q + 2] = v.z, pk[4 * q + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 64; ++q) pk[q] = 0u;
+        }
+      }
       const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, acc_phase, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + half * 128;
-      const int64_t n0 = (int64_t)tc.n_blk * BN + half * 128;
-      const int chunks = mine ? min(4, (n_cols - half * 128) / 32) : 0;
-      if (packed) {
-        // BF16 without accumulation: scale and round while reading, so the 128
-        // columns of this warp stay in 64 registers; release the accumulator, then
-        // write the warp's 32 x 128 block out as two 32 x 64 TMA stores staged in
-        // its own 4 KB of shared memory (128-byte swizzle: lane r puts 16-byte chunk
-        // c of its row at chunk c ^ (r % 8), which keeps each quarter-warp on
-        // distinct banks).  Whole-line bulk stores instead of per-row 16-byte
-        // stores keep the output burst at every tile change off the operand loads.
-        uint32_t pk[64];
+      if constexpr (bf16_out) {
         if (mine) {
+          if constexpr (accumulate) {
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t r[64];
-            tc_load_32cols(taddr + 64 * hh, r);
-            tc_load_32cols(taddr + 64 * hh + 32, r + 32);
-            tc_wait_loads();
+            for (int k = 0; k < 4; ++k) {
+              uint32_t r[32];
+              tc_load_32cols(taddr + 32 * k, r);
+              tc_wait_loads();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) pk[32 * hh + j] = scale_pack_bf16x2(r[2 * j], r[2 * j + 1], g);
+              for (int j = 0; j < 16; ++j) {
+                const uint32_t o = pk[16 * k + j];
+                const float v0 = __fadd_rn(__fmul_rn(__uint_as_float(r[2 * j]), g), bf16_lo(o));
+                const float v1 = __fadd_rn(__fmul_rn(__uint_as_float(r[2 * j + 1]), g), bf16_hi(o));
+                pk[16 * k + j] = pack_bf16x2(v0, v1);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t r[64];
+              tc_load_32cols(taddr + 64 * hh, r);
+              tc_load_32cols(taddr + 64 * hh + 32, r + 32);
+              tc_wait_loads();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) pk[32 * hh + j] = scale_pack_bf16x2(r[2 * j], r[2 * j + 1], g);
+            }
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster_tc(leader_acc_empty);
-        const int32_t m0 = tc.m_blk * P_BM + (int32_t)rank * 128 + quarter * 32;
-        uint8_t* stg = smem + P_EPI_OFFSET + ew * P_EPI_BOX_BYTES;
         float mraw = 0.0f, mrht = 0.0f;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          if (n_cols <= half * 128 + hh * P_EPI_BOX_COLS || m0 >= p.M) continue;   // box outside C
+          if (!mine || !rows_in) continue;                                 // box outside C
           if (lane == 0) bulk_wait_read();                                 // staging buffer free again
           __syncwarp();
 #pragma unroll
@@ -935,9 +1040,9 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             tma_store_2d(&tma_c, (int32_t)n0 + hh * P_EPI_BOX_COLS, m0, smem_u32(stg));
             bulk_commit();
           }
-          if (p.amax_acc) box_amax(stg, lane, p.rht_signs, mraw, mrht);
+          if (EPI == EPI_BF16 && p.amax_acc) box_amax(stg, lane, p.rht_signs, mraw, mrht);
         }
-        if (p.amax_acc) {
+        if (EPI == EPI_BF16 && p.amax_acc) {
           // boxes past the end of C hold zeros (their operand rows were zero-filled), so
           // the maxima need no masking; 0.25 * max |w| = max |w / 4| (scaling by 1/4 is
           // monotonic in round-to-nearest)
@@ -952,17 +1057,45 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             atomicMax(p.amax_acc + 1, __float_as_uint(mrht));
           }
         }
+      } else if constexpr (!accumulate) {
+        // FP32: 32 columns (one 128-byte box row per lane) at a time
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+          uint32_t r[32];
+          if (mine) {
+            tc_load_32cols(taddr + 32 * k, r);
+            tc_wait_loads();
+          }
+          if (k == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_tc(leader_acc_empty);
+          }
+          if (!mine || !rows_in) continue;
+          if (lane == 0) bulk_wait_read();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<float4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_float4(__fmul_rn(__uint_as_float(r[4 * c]), g), __fmul_rn(__uint_as_float(r[4 * c + 1]), g),
+                            __fmul_rn(__uint_as_float(r[4 * c + 2]), g), __fmul_rn(__uint_as_float(r[4 * c + 3]), g));
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tma_c, (int32_t)n0 + 32 * k, m0, smem_u32(stg));
+            bulk_commit();
+          }
+        }
       } else {
-        // FP32 output or accumulation into C: 32 columns at a time, released at the end.
-        const size_t esz = p.out_f32 ? 4 : 2;
-        uint8_t* crow = static_cast<uint8_t*>(p.C) + (size_t)(m * p.ldc + n0) * esz;
+        // FP32 accumulation into C: 32 columns at a time, released at the end.
+        uint8_t* crow = static_cast<uint8_t*>(p.C) + (size_t)(m * p.ldc + n0) * 4;
         if (mine) {
 #pragma unroll 1
           for (int k = 0; k < 4; ++k) {
             uint32_t r[32];
             tc_load_32cols(taddr + 32 * k, r);
             tc_wait_loads();
-            if (k < chunks && m < p.M) store_32cols(p, r, g, crow + (size_t)32 * k * esz);
+            if (rows_in) store_32cols(p, r, g, crow + (size_t)32 * k * 4);
           }
         }
         tc_fence_before();

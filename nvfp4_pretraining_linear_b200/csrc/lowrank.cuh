@@ -122,11 +122,16 @@ __device__ __forceinline__ uint32_t pack_bf16_pair(const uint16_t* lo, const uin
 // CTA.  B is staged as given: [r x K] rows (BT false) give each MMA operand register
 // as one 32-bit load; [K x r] rows (BT true, e.g. L in dgrad) are staged unchanged and
 // each register is packed from two 16-bit loads.
+//
+// With scale_a and scale_b given, the sums are divided by g = fl32(*scale_a * *scale_b)
+// before the rounding: U' = BF16(fl32(fl32(sum) * fl32(1 / g))) -- the projection that
+// joins an NVFP4 GEMM's accumulator, which that GEMM multiplies by g.
 template <int RT, bool BT>
 __global__ void __launch_bounds__(kProjThreads) lowrank_project_kernel(const uint16_t* __restrict__ a, int64_t lda,
                                                                        const uint16_t* __restrict__ b, int64_t ldb,
                                                                        int64_t K, uint16_t* __restrict__ u,
-                                                                       int64_t ldu) {
+                                                                       int64_t ldu, const float* scale_a,
+                                                                       const float* scale_b) {
   constexpr int R = RT * 8, RSn = R + 8;          // RSn: row stride of a staged [K x r] chunk
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint16_t (*As)[kProjRows][kPad] = reinterpret_cast<uint16_t (*)[kProjRows][kPad]>(smem_raw);
@@ -200,6 +205,13 @@ __global__ void __launch_bounds__(kProjThreads) lowrank_project_kernel(const uin
   }
   cp_async_wait_pending<0>();
   const int64_t row = m0 + warp * 16 + g;
+  if (scale_a) {
+    const float inv = __fdiv_rn(1.0f, __fmul_rn(*scale_a, *scale_b));
+#pragma unroll
+    for (int nt = 0; nt < RT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][e] = __fmul_rn(acc[nt][e], inv);
+  }
 #pragma unroll
   for (int nt = 0; nt < RT; ++nt) {
     const int col = nt * 8 + 2 * t;

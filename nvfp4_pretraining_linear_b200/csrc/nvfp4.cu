@@ -68,9 +68,13 @@ nvfp4_status device_info(DeviceInfo** out) {
     e = cudaFuncSetAttribute(nvfp4::gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              nvfp4::gemm::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-    e = cudaFuncSetAttribute(nvfp4::gemm::gemm_kernel_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             nvfp4::gemm::P_SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
+    for (auto kernel : {nvfp4::gemm::gemm_kernel_pair<nvfp4::gemm::EPI_BF16>,
+                        nvfp4::gemm::gemm_kernel_pair<nvfp4::gemm::EPI_BF16_ACC>,
+                        nvfp4::gemm::gemm_kernel_pair<nvfp4::gemm::EPI_F32>,
+                        nvfp4::gemm::gemm_kernel_pair<nvfp4::gemm::EPI_F32_ACC>}) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, nvfp4::gemm::P_SMEM_BYTES);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
+    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -83,7 +87,7 @@ nvfp4_status device_info(DeviceInfo** out) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, nvfp4::gemm::gemm_kernel_pair, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&clusters, nvfp4::gemm::gemm_kernel_pair<nvfp4::gemm::EPI_BF16>, &cfg);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
     d.pair_clusters = clusters;
     d.gemm_attr = true;
@@ -108,50 +112,53 @@ nvfp4_status get_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
   return NVFP4_OK;
 }
 
-// Tensor map of packed E2M1 codes [rows][cols/2 bytes]: box of box_rows x 128
-// bytes, 128-byte swizzle (the tensor cores' K-major operand layout).
-nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t, uint32_t box_rows) {
+// Tensor map of packed E2M1 codes [rows][cols/2 bytes]: box of box_rows x box_bytes
+// bytes, swizzled with box_bytes (128 or 64): the tensor cores' K-major operand layout.
+nvfp4_status make_code_map(CUtensorMap* map, const nvfp4_tensor* t, uint32_t box_rows, uint32_t box_bytes) {
   PFN_cuTensorMapEncodeTiled_v12000 encode;
   nvfp4_status st = get_encoder(&encode);
   if (st != NVFP4_OK) return st;
   const cuuint64_t dims[2] = {(cuuint64_t)(t->cols / 2), (cuuint64_t)t->rows};
   const cuuint64_t strides[1] = {(cuuint64_t)(t->cols / 2)};
-  const cuuint32_t box[2] = {128u, box_rows};
+  const cuuint32_t box[2] = {box_bytes, box_rows};
   const cuuint32_t estr[2] = {1u, 1u};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, t->codes, dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                      CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      box_bytes == 128u ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return NVFP4_OK;
 }
 
-// Tensor map of a BF16 output C [M x N] (row stride ldc elements) for the pair
-// GEMM's epilogue stores: boxes of 32 rows x 64 columns, 128-byte swizzle.
-nvfp4_status make_out_map(CUtensorMap* map, void* C, int64_t M, int64_t N, int64_t ldc) {
+// Tensor map of the output C [M x N] (row stride ldc elements) for the pair GEMM's
+// epilogue stores: boxes of 32 rows x 128 bytes (64 BF16 or 32 FP32 columns),
+// 128-byte swizzle.
+nvfp4_status make_out_map(CUtensorMap* map, void* C, int64_t M, int64_t N, int64_t ldc, bool f32) {
   PFN_cuTensorMapEncodeTiled_v12000 encode;
   nvfp4_status st = get_encoder(&encode);
   if (st != NVFP4_OK) return st;
+  const cuuint64_t esz = f32 ? 4u : 2u;
   const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)ldc * 2u};
-  const cuuint32_t box[2] = {(cuuint32_t)nvfp4::gemm::P_EPI_BOX_COLS, 32u};
+  const cuuint64_t strides[1] = {(cuuint64_t)ldc * esz};
+  const cuuint32_t box[2] = {(cuuint32_t)(128u / esz), 32u};
   const cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encode(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled(C) failed (%d)", (int)r);
   return NVFP4_OK;
 }
 
-// Tensor map over the tensor-core scale layout viewed as rows of 512-byte
-// atoms (128 x 32-bit words): box of 4 atoms = one 128-row block x 256 K.
-nvfp4_status make_scale_map(CUtensorMap* map, const nvfp4_tensor* t) {
+// Tensor map over the tensor-core scale layout viewed as rows of 512-byte atoms (128 x
+// 32-bit words): box of box_atoms atoms = one 128-row block x 64 * box_atoms K.
+nvfp4_status make_scale_map(CUtensorMap* map, const nvfp4_tensor* t, uint32_t box_atoms) {
   PFN_cuTensorMapEncodeTiled_v12000 encode;
   nvfp4_status st = get_encoder(&encode);
   if (st != NVFP4_OK) return st;
   const int64_t atoms = ceil_div(t->rows, 128) * ceil_div(t->cols / 16, 4);
   const cuuint64_t dims[2] = {128u, (cuuint64_t)atoms};
   const cuuint64_t strides[1] = {512u};
-  const cuuint32_t box[2] = {128u, 4u};
+  const cuuint32_t box[2] = {128u, box_atoms};
   const cuuint32_t estr[2] = {1u, 1u};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, t->scales, dims, strides, box, estr,
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -182,7 +189,6 @@ nvfp4::QuantLayout layout_of(const nvfp4_tensor* t) {
   L.tensor_scale = t->tensor_scale;
   L.kgroups = ceil_div(t->cols / 16, 4);
   L.mma_layout = t->scale_layout == NVFP4_SCALE_MMA;
-  L.vec16 = ((t->cols / 2) % 16) == 0;
   return L;
 }
 
@@ -207,6 +213,16 @@ cudaError_t ensure_smem(Kernel kernel, int bytes, bool (&done)[kMaxDevices], std
 // faults, traps or hangs; unset (the default) it costs one getenv per call.
 int64_t injected_skip_tile() {
   const char* v = std::getenv("NVFP4_INJECT_SKIP_TILE");
+  if (!v || !*v) return -1;
+  char* end = nullptr;
+  const long long n = std::strtoll(v, &end, 10);
+  return (end && *end == '\0' && n >= 0) ? (int64_t)n : -1;
+}
+
+// The same for the pair GEMM: with NVFP4_INJECT_GEMM_SKIP_STAGE=n, CTA pair 0 never
+// loads its K-stage number n, so the MMA issuers' bounded wait expires.
+int64_t injected_gemm_skip_stage() {
+  const char* v = std::getenv("NVFP4_INJECT_GEMM_SKIP_STAGE");
   if (!v || !*v) return -1;
   char* end = nullptr;
   const long long n = std::strtoll(v, &end, 10);
@@ -389,8 +405,11 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
   p.row = layout_of(out_row);
   p.col = layout_of(out_col);
   p.amax_out = opts->amax_out;
-  p.key0 = (uint32_t)opts->seed;
-  p.key1 = (uint32_t)(opts->seed >> 32);
+  // Philox round keys of the seed (the key schedule of Philox4x32-10, precomputed)
+  for (int r = 0; r < 10; ++r) {
+    p.rk[r] = (uint32_t)opts->seed + (uint32_t)r * 0x9E3779B9u;
+    p.rk[10 + r] = (uint32_t)(opts->seed >> 32) + (uint32_t)r * 0xBB67AE85u;
+  }
   p.offset = (uint32_t)opts->offset;
   p.signs = opts->rht_signs;
   p.skip_tile = -1;
@@ -435,9 +454,39 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor* q, void* out, int64_t ldo, int
 }
 
 namespace {
-// nvfp4_gemm, and with amax_out (3 floats) the maxima of nvfp4_gemm_amax.
+// Low-rank operands of a GEMM that adds U V^T inside its accumulator (nvfp4_gemm_lowrank):
+// U [M x rank], V [N x rank], BF16, row strides ldu, ldv elements.
+struct LowRank {
+  const void* U = nullptr;
+  int64_t ldu = 0;
+  const void* V = nullptr;
+  int64_t ldv = 0;
+  int32_t rank = 0;
+};
+
+// Tensor map of a BF16 low-rank factor [rows x rank] (row stride ld elements): boxes of
+// 128 rows x 64 elements (128 bytes, zero-filled past the rank), 128-byte swizzle -- the
+// K-major operand layout of the low-rank stage's BF16 MMAs.
+nvfp4_status make_lowrank_map(CUtensorMap* map, const void* X, int64_t rows, int64_t ld, int32_t rank) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  nvfp4_status st = get_encoder(&encode);
+  if (st != NVFP4_OK) return st;
+  const cuuint64_t dims[2] = {(cuuint64_t)rank, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2u};
+  const cuuint32_t box[2] = {64u, 128u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled(low-rank factor) failed (%d)", (int)r);
+  return NVFP4_OK;
+}
+
+// nvfp4_gemm; with amax_out (3 floats) the maxima of nvfp4_gemm_amax; with a low-rank
+// pair the U V^T term of nvfp4_gemm_lowrank.
 nvfp4_status gemm_impl(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc, int32_t out_dtype,
-                       float alpha, int32_t accumulate, float* amax_out, uint32_t rht_signs, void* stream) {
+                       float alpha, int32_t accumulate, float* amax_out, uint32_t rht_signs, void* stream,
+                       const LowRank* lr = nullptr) {
   nvfp4_status st;
   if ((st = check_tensor(A, "A")) != NVFP4_OK) return st;
   if ((st = check_tensor(B, "B")) != NVFP4_OK) return st;
@@ -495,20 +544,31 @@ nvfp4_status gemm_impl(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, in
   p.accumulate = accumulate != 0;
   p.amax_acc = reinterpret_cast<unsigned*>(amax_out);
   p.rht_signs = rht_signs & 0xFFFFu;
+  p.skip_stage = injected_gemm_skip_stage();
   cudaError_t e;
   if (amax_out && dev->pair_clusters == 0)
     return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the output maxima need the CTA-pair GEMM, not available on this device");
+  if (lr && (M < 256 || dev->pair_clusters == 0))
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the low-rank term needs M >= 256 and the CTA-pair GEMM");
+  p.lr_ksteps = lr ? lr->rank / 16 : 0;
   if (M >= 256 && dev->pair_clusters > 0) {
     // CTA pairs, 256 x 256 tiles
-    CUtensorMap map_a, map_b, map_sfa, map_sfb, map_c;
-    if ((st = make_code_map(&map_a, A, 128)) != NVFP4_OK) return st;
-    if ((st = make_code_map(&map_b, B, 128)) != NVFP4_OK) return st;
-    if ((st = make_scale_map(&map_sfa, A)) != NVFP4_OK) return st;
-    if ((st = make_scale_map(&map_sfb, B)) != NVFP4_OK) return st;
-    // the BF16 store map is only read by the BF16, non-accumulating epilogue
+    CUtensorMap map_a, map_b, map_sfa, map_sfb, map_c, map_u, map_v;
+    // 256-element K-stages: 128-byte code boxes, four scale tiles per stage
+    if ((st = make_code_map(&map_a, A, 128, nvfp4::gemm::BK_BYTES)) != NVFP4_OK) return st;
+    if ((st = make_code_map(&map_b, B, 128, nvfp4::gemm::BK_BYTES)) != NVFP4_OK) return st;
+    if ((st = make_scale_map(&map_sfa, A, nvfp4::gemm::BK / nvfp4::gemm::MMA_K)) != NVFP4_OK) return st;
+    if ((st = make_scale_map(&map_sfb, B, nvfp4::gemm::BK / nvfp4::gemm::MMA_K)) != NVFP4_OK) return st;
+    // the store map is read by every epilogue but the FP32 accumulating one
     std::memset(&map_c, 0, sizeof(map_c));
-    if (out_dtype == NVFP4_OUT_BF16 && !accumulate && (st = make_out_map(&map_c, C, M, N, ldc)) != NVFP4_OK)
-      return st;
+    const bool f32 = out_dtype == NVFP4_OUT_F32;
+    if (!(f32 && accumulate) && (st = make_out_map(&map_c, C, M, N, ldc, f32)) != NVFP4_OK) return st;
+    std::memset(&map_u, 0, sizeof(map_u));
+    std::memset(&map_v, 0, sizeof(map_v));
+    if (lr) {
+      if ((st = make_lowrank_map(&map_u, lr->U, M, lr->ldu, lr->rank)) != NVFP4_OK) return st;
+      if ((st = make_lowrank_map(&map_v, lr->V, N, lr->ldv, lr->rank)) != NVFP4_OK) return st;
+    }
     p.num_m = (int32_t)ceil_div(M, nvfp4::gemm::P_BM);
     p.group_m = 16;
     const int64_t tiles = (int64_t)p.num_m * p.num_n;
@@ -525,11 +585,14 @@ nvfp4_status gemm_impl(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, in
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, nvfp4::gemm::gemm_kernel_pair, map_a, map_b, map_sfa, map_sfb, map_c, p);
+    using namespace nvfp4::gemm;
+    auto kernel = f32 ? (accumulate ? gemm_kernel_pair<EPI_F32_ACC> : gemm_kernel_pair<EPI_F32>)
+                      : (accumulate ? gemm_kernel_pair<EPI_BF16_ACC> : gemm_kernel_pair<EPI_BF16>);
+    e = cudaLaunchKernelEx(&cfg, kernel, map_a, map_b, map_sfa, map_sfb, map_c, map_u, map_v, p);
   } else {
     CUtensorMap map_a, map_b;
-    if ((st = make_code_map(&map_a, A, nvfp4::gemm::BM)) != NVFP4_OK) return st;
-    if ((st = make_code_map(&map_b, B, nvfp4::gemm::BN)) != NVFP4_OK) return st;
+    if ((st = make_code_map(&map_a, A, nvfp4::gemm::BM, nvfp4::gemm::BK_BYTES)) != NVFP4_OK) return st;
+    if ((st = make_code_map(&map_b, B, nvfp4::gemm::BN, nvfp4::gemm::BK_BYTES)) != NVFP4_OK) return st;
     p.num_m = (int32_t)(M / nvfp4::gemm::BM);
     p.group_m = 16;
     const int64_t tiles = (int64_t)p.num_m * p.num_n;
@@ -552,6 +615,23 @@ nvfp4_status nvfp4_gemm_amax(const nvfp4_tensor* A, const nvfp4_tensor* B, void*
   if (!amax_out) return fail(NVFP4_ERR_INVALID_ARG, "amax_out is NULL");
   if (reinterpret_cast<uintptr_t>(amax_out) % 4) return fail(NVFP4_ERR_MISALIGNED, "amax_out is not 4-byte aligned");
   return gemm_impl(A, B, C, ldc, NVFP4_OUT_BF16, alpha, 0, amax_out, rht_signs, stream);
+}
+
+nvfp4_status nvfp4_gemm_lowrank(const nvfp4_tensor* A, const nvfp4_tensor* B, const void* U, int64_t ldu,
+                                const void* V, int64_t ldv, int32_t rank, void* C, int64_t ldc, void* stream) {
+  if (rank != 16 && rank != 32 && rank != 48 && rank != 64)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
+  if (!U || !V) return fail(NVFP4_ERR_INVALID_ARG, "U or V is NULL");
+  if (ldu < rank || ldv < rank) return fail(NVFP4_ERR_INVALID_ARG, "ldu or ldv < rank");
+  if (!aligned16(U) || !aligned16(V) || ldu % 8 || ldv % 8)
+    return fail(NVFP4_ERR_MISALIGNED, "U and V rows must be 16-byte aligned");
+  LowRank lr;
+  lr.U = U;
+  lr.ldu = ldu;
+  lr.V = V;
+  lr.ldv = ldv;
+  lr.rank = rank;
+  return gemm_impl(A, B, C, ldc, NVFP4_OUT_BF16, 1.0f, 0, nullptr, 0u, stream, &lr);
 }
 
 nvfp4_status nvfp4_linear_fwd(const void* X, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* Wq_row, void* Y,
@@ -705,22 +785,22 @@ bool rank_ok(int32_t rank) { return rank >= 16 && rank <= nvfp4::lowrank::kMaxRa
 
 template <int RT, bool BT>
 cudaError_t launch_project(const uint16_t* a, int64_t lda, const uint16_t* b, int64_t ldb, int64_t M, int64_t K,
-                           uint16_t* u, int64_t ldu, cudaStream_t s) {
+                           uint16_t* u, int64_t ldu, const float* sa, const float* sb, cudaStream_t s) {
   static bool done[kMaxDevices] = {};
   static std::mutex m;
   auto kernel = nvfp4::lowrank::lowrank_project_kernel<RT, BT>;
   cudaError_t e = ensure_smem(kernel, nvfp4::lowrank::kProjSmemBytes, done, m);
   if (e != cudaSuccess) return e;
   kernel<<<(unsigned)(M / nvfp4::lowrank::kProjRows), nvfp4::lowrank::kProjThreads, nvfp4::lowrank::kProjSmemBytes,
-           s>>>(a, lda, b, ldb, K, u, ldu);
+           s>>>(a, lda, b, ldb, K, u, ldu, sa, sb);
   return cudaGetLastError();
 }
 
 template <int RT>
 cudaError_t dispatch_project(bool bt, const uint16_t* a, int64_t lda, const uint16_t* b, int64_t ldb, int64_t M,
-                             int64_t K, uint16_t* u, int64_t ldu, cudaStream_t s) {
-  return bt ? launch_project<RT, true>(a, lda, b, ldb, M, K, u, ldu, s)
-            : launch_project<RT, false>(a, lda, b, ldb, M, K, u, ldu, s);
+                             int64_t K, uint16_t* u, int64_t ldu, const float* sa, const float* sb, cudaStream_t s) {
+  return bt ? launch_project<RT, true>(a, lda, b, ldb, M, K, u, ldu, sa, sb, s)
+            : launch_project<RT, false>(a, lda, b, ldb, M, K, u, ldu, sa, sb, s);
 }
 
 template <int KS, bool CT>
@@ -771,14 +851,19 @@ nvfp4_status nvfp4_lora_residual(const void* W, int64_t N, int64_t K, int64_t ld
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "lora residual launch");
 }
 
-nvfp4_status nvfp4_lowrank_project(const void* A, int64_t M, int64_t K, int64_t lda, const void* B, int64_t ldb,
-                                   int32_t b_trans, int32_t rank, void* U, int64_t ldu, void* stream) {
+}  // extern "C"
+
+namespace {
+nvfp4_status lowrank_project_impl(const void* A, int64_t M, int64_t K, int64_t lda, const void* B, int64_t ldb,
+                                  int32_t b_trans, int32_t rank, const float* sa, const float* sb, void* U,
+                                  int64_t ldu, void* stream) {
   if (!rank_ok(rank)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
   if (M < 0 || K < 0) return fail(NVFP4_ERR_INVALID_ARG, "negative extent");
   if (M % nvfp4::lowrank::kProjRows || K % nvfp4::lowrank::kProjKc || K == 0)
     return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "projection needs M %% 64 == 0 and K a positive multiple of 64");
   if (M == 0) return NVFP4_OK;
   if (!A || !B || !U) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
+  if ((sa == nullptr) != (sb == nullptr)) return fail(NVFP4_ERR_INVALID_ARG, "give both tensor scales or neither");
   if (lda < K || ldu < rank || ldb < (b_trans ? (int64_t)rank : K))
     return fail(NVFP4_ERR_INVALID_ARG, "leading dimension too small");
   if (!aligned16(A) || !aligned16(B) || !aligned16(U) || lda % 8 || ldb % 8 || ldu % 8)
@@ -790,12 +875,27 @@ nvfp4_status nvfp4_lowrank_project(const void* A, int64_t M, int64_t K, int64_t 
   const bool bt = b_trans != 0;
   cudaError_t e;
   switch (rank / 8) {
-    case 2: e = dispatch_project<2>(bt, a, lda, b, ldb, M, K, u, ldu, s); break;
-    case 4: e = dispatch_project<4>(bt, a, lda, b, ldb, M, K, u, ldu, s); break;
-    case 6: e = dispatch_project<6>(bt, a, lda, b, ldb, M, K, u, ldu, s); break;
-    default: e = dispatch_project<8>(bt, a, lda, b, ldb, M, K, u, ldu, s); break;
+    case 2: e = dispatch_project<2>(bt, a, lda, b, ldb, M, K, u, ldu, sa, sb, s); break;
+    case 4: e = dispatch_project<4>(bt, a, lda, b, ldb, M, K, u, ldu, sa, sb, s); break;
+    case 6: e = dispatch_project<6>(bt, a, lda, b, ldb, M, K, u, ldu, sa, sb, s); break;
+    default: e = dispatch_project<8>(bt, a, lda, b, ldb, M, K, u, ldu, sa, sb, s); break;
   }
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "low-rank projection launch");
+}
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_lowrank_project(const void* A, int64_t M, int64_t K, int64_t lda, const void* B, int64_t ldb,
+                                   int32_t b_trans, int32_t rank, void* U, int64_t ldu, void* stream) {
+  return lowrank_project_impl(A, M, K, lda, B, ldb, b_trans, rank, nullptr, nullptr, U, ldu, stream);
+}
+
+nvfp4_status nvfp4_lowrank_project_scaled(const void* A, int64_t M, int64_t K, int64_t lda, const void* B,
+                                          int64_t ldb, int32_t b_trans, int32_t rank, const float* scale_a,
+                                          const float* scale_b, void* U, int64_t ldu, void* stream) {
+  if (!scale_a || !scale_b) return fail(NVFP4_ERR_INVALID_ARG, "scale_a or scale_b is NULL");
+  return lowrank_project_impl(A, M, K, lda, B, ldb, b_trans, rank, scale_a, scale_b, U, ldu, stream);
 }
 
 nvfp4_status nvfp4_lowrank_expand_add(void* Y, int64_t M, int64_t N, int64_t ldy, const void* U, int64_t ldu,
@@ -861,27 +961,46 @@ nvfp4_status nvfp4_lora_linear_fwd(const void* X, int64_t M, int64_t K, int64_t 
                                    void* workspace, size_t workspace_bytes, void* stream) {
   nvfp4_status st = lora_precheck(Wq_res_row, L, R, rank, U, M, Wq_res_row ? Wq_res_row->rows : 0, K, ldx, ldy);
   if (st != NVFP4_OK) return st;
-  st = nvfp4_linear_fwd(X, M, K, ldx, Wq_res_row, Y, ldy, NVFP4_OUT_BF16, Xq_row, Xq_col, rht_signs,
-                                     workspace, workspace_bytes, stream);
-  if (st != NVFP4_OK) return st;
-  const int64_t N = Wq_res_row->rows;
-  if ((st = nvfp4_lowrank_project(X, M, K, ldx, R, K, 0, rank, U, rank, stream)) != NVFP4_OK) return st;
-  return nvfp4_lowrank_expand_add(Y, M, N, ldy, U, rank, L, rank, 0, rank, stream);
+  if ((st = check_tensor(Wq_res_row, "Wq_res_row")) != NVFP4_OK) return st;
+  if (!Xq_row) return fail(NVFP4_ERR_INVALID_ARG, "Xq_row is NULL");
+  if (Wq_res_row->cols != K) return fail(NVFP4_ERR_INVALID_ARG, "Wq_res_row.cols != K");
+  if (M < 256) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the fused LoRA-SVD linear needs M >= 256");
+  nvfp4_quant_opts o{};
+  o.rht_col = Xq_col != nullptr;
+  o.rht_signs = rht_signs;
+  if ((st = nvfp4_quantize(X, M, K, ldx, &o, Xq_row, Xq_col, workspace, workspace_bytes, stream)) != NVFP4_OK)
+    return st;
+  // U' = BF16(X R^T / (S_X S_W)), then Y = BF16(S_X S_W (Q(X) Q(W_res)^T + U' L^T)) in one GEMM
+  if ((st = lowrank_project_impl(X, M, K, ldx, R, K, 0, rank, Xq_row->tensor_scale, Wq_res_row->tensor_scale, U,
+                                 rank, stream)) != NVFP4_OK)
+    return st;
+  return nvfp4_gemm_lowrank(Xq_row, Wq_res_row, U, rank, L, rank, rank, Y, ldy, stream);
 }
 
 nvfp4_status nvfp4_lora_linear_dgrad(const void* dY, int64_t M, int64_t N, int64_t ldy, const nvfp4_tensor* Wq_res_col,
-                                     const void* L, const void* R, int32_t rank, void* dX, int64_t ldx,
+                                     const void* L, const void* Rt, int32_t rank, void* dX, int64_t ldx,
                                      nvfp4_tensor* dYq_row, nvfp4_tensor* dYq_col, uint64_t seed, uint64_t offset,
                                      uint32_t rht_signs, void* U, void* workspace, size_t workspace_bytes,
                                      void* stream) {
-  nvfp4_status st = lora_precheck(Wq_res_col, L, R, rank, U, M, Wq_res_col ? Wq_res_col->rows : 0, N, ldy, ldx);
+  nvfp4_status st = lora_precheck(Wq_res_col, L, Rt, rank, U, M, Wq_res_col ? Wq_res_col->rows : 0, N, ldy, ldx);
   if (st != NVFP4_OK) return st;
-  st = nvfp4_linear_dgrad(dY, M, N, ldy, Wq_res_col, dX, ldx, NVFP4_OUT_BF16, dYq_row, dYq_col, seed,
-                                       offset, rht_signs, workspace, workspace_bytes, stream);
-  if (st != NVFP4_OK) return st;
-  const int64_t K = Wq_res_col->rows;
-  if ((st = nvfp4_lowrank_project(dY, M, N, ldy, L, rank, 1, rank, U, rank, stream)) != NVFP4_OK) return st;
-  return nvfp4_lowrank_expand_add(dX, M, K, ldx, U, rank, R, K, 1, rank, stream);
+  if ((st = check_tensor(Wq_res_col, "Wq_res_col")) != NVFP4_OK) return st;
+  if (!dYq_row) return fail(NVFP4_ERR_INVALID_ARG, "dYq_row is NULL");
+  if (Wq_res_col->cols != N) return fail(NVFP4_ERR_INVALID_ARG, "Wq_res_col.cols != N");
+  if (M < 256) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the fused LoRA-SVD linear needs M >= 256");
+  nvfp4_quant_opts o{};
+  o.stochastic = 1;
+  o.rht_col = dYq_col != nullptr;
+  o.seed = seed;
+  o.offset = offset;
+  o.rht_signs = rht_signs;
+  if ((st = nvfp4_quantize(dY, M, N, ldy, &o, dYq_row, dYq_col, workspace, workspace_bytes, stream)) != NVFP4_OK)
+    return st;
+  // U' = BF16(dY L / (S_dY S_W)), then dX = BF16(S_dY S_W (Q(dY) Q(W_res) + U' R)) in one GEMM
+  if ((st = lowrank_project_impl(dY, M, N, ldy, L, rank, 1, rank, dYq_row->tensor_scale, Wq_res_col->tensor_scale,
+                                 U, rank, stream)) != NVFP4_OK)
+    return st;
+  return nvfp4_gemm_lowrank(dYq_row, Wq_res_col, U, rank, Rt, rank, rank, dX, ldx, stream);
 }
 
 nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,

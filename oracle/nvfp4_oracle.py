@@ -89,11 +89,17 @@ stated where it is used:
     top-r singular triplets of W), W_res = BF16(fl32(W - s)) where s accumulates
     L[n, j] R[j, k] in FP32 over j = 0, 1, ... (each product of BF16 values exact).
     W_res takes the NVFP4 path of the linear layer (2D blocks); the low-rank part
-    stays in BF16:  Y = BF16(fl32(Y4 + V)) with Y4 = BF16(Q(X) Q(W_res)^T) and
-    V = fl32((BF16(X R^T)) L^T);  dX = BF16(fl32(dX4 + V')) with dX4 the NVFP4
-    dgrad against W_res and V' = fl32((BF16(dY L)) R).  The weight gradient is that
-    of W itself (the NVFP4 wgrad, unchanged).  Products of the low-rank branch are
-    taken exactly and rounded once (the hardware accumulates in FP32).
+    stays in BF16 and joins the NVFP4 product inside its FP32 accumulator, before the
+    tensor scales are applied.  With g = fl32(S_X * S_W) the product of the two NVFP4
+    tensor scales (the factor the GEMM applies to its accumulator), the projection is
+    pre-divided by g:  U' = BF16(fl32(fl32(X R^T) * fl32(1 / g))), and
+        Y = BF16(g * (sum_k a_k b_k + sum_j U'[m, j] L[n, j]))
+    where a_k b_k are the block-scaled NVFP4 products (x_hat w_hat = g a b up to the
+    rounding of g); the reference is that expression in FP64,
+    Y_ref = Q(X) Q(W_res)^T + g U' L^T, checked within the GEMM bound over both sums.
+    dgrad likewise with g = fl32(S_dY * S_W), U' = BF16(fl32(fl32(dY L) * fl32(1/g)))
+    and the low-rank product U' R.  The weight gradient is that of W itself (the NVFP4
+    wgrad, unchanged).  The projection's sum is taken exactly and rounded once to FP32.
 """
 
 from __future__ import annotations
@@ -600,32 +606,55 @@ def lora_expand_add(y: np.ndarray, u: np.ndarray, c: np.ndarray) -> np.ndarray:
     return add_product_bf16(gemm_ref(u, c), y)
 
 
+def lora_project_scaled(a: np.ndarray, b: np.ndarray, g) -> np.ndarray:
+    """U' = BF16(fl32(fl32(A B^T) * fl32(1 / g))): the projection pre-divided by the
+    NVFP4 tensor-scale product g, A [M x K], B [r x K]."""
+    inv = F32(F32(1.0) / F32(g))
+    return bf16_round((gemm_ref(a, b).astype(F32) * inv).astype(F32))
+
+
+def _lora_compose(prod_exact, a_hat, b_hat, u, c, g):
+    """Reference and bound scale of the fused LoRA-SVD output: the NVFP4 product (exact,
+    FP64) plus g * U' C^T, and sum |a b| + g * sum |U'| |C| over both."""
+    low = float(g) * gemm_ref(u, c)
+    scale = gemm_abs_ref(a_hat, b_hat) + float(g) * gemm_abs_ref(u, c)
+    return prod_exact + low, scale
+
+
 def lora_linear_fwd(x: np.ndarray, w_res_q: dict, l: np.ndarray, r: np.ndarray, rht_signs: int = 0,
                     quantize_operands: bool = True):
-    """Y = BF16(fl32(Y4 + fl32(U L^T))), U = BF16(X R^T), Y4 = BF16(Q(X) Q(W_res)^T).
+    """Y_ref = Q(X) Q(W_res)^T + g U' L^T in FP64, U' = BF16(fl32(fl32(X R^T) / g)),
+    g = fl32(S_X S_W) (reading 12).  Returns (Y_ref, parts); parts["abs_scale"] is the
+    sum |a b| over both products, the scale of the GEMM bound.
 
-    w_res_q is quantize_weight(W_res); with quantize_operands=False it is W_res itself
-    and Y4 uses the unquantised values (the identity check of the decomposition)."""
+    w_res_q is quantize_weight(W_res); with quantize_operands=False it is W_res itself,
+    the products use the unquantised values and g = 1 (the identity check)."""
     x = np.asarray(x, dtype=F32)
     if quantize_operands:
-        y4_exact, (a_hat, b_hat), xq = linear_fwd_ref(x, w_res_q, rht_signs=rht_signs)
+        prod, (a_hat, b_hat), xq = linear_fwd_ref(x, w_res_q, rht_signs=rht_signs)
+        g = F32(F32(xq["row"][2]) * F32(w_res_q["row"][2]))
     else:
-        y4_exact, (a_hat, b_hat), xq = gemm_ref(x, w_res_q), (x, w_res_q), None
-    y4 = bf16_round(y4_exact.astype(F32))
-    u = lora_project(x, r)
-    return lora_expand_add(y4, u, l), {"y4": y4, "y4_exact": y4_exact, "u": u, "a_hat": a_hat,
-                                       "b_hat": b_hat, "xq": xq}
+        prod, (a_hat, b_hat), xq = gemm_ref(x, w_res_q), (x, np.asarray(w_res_q, dtype=F32)), None
+        g = F32(1.0)
+    u = lora_project_scaled(x, r, g)
+    y_ref, scale = _lora_compose(prod, a_hat, b_hat, u, np.asarray(l, dtype=F32), g)
+    return y_ref, {"prod": prod, "u": u, "g": g, "a_hat": a_hat, "b_hat": b_hat, "xq": xq,
+                   "abs_scale": scale}
 
 
 def lora_linear_dgrad(dy: np.ndarray, w_res_q: dict, l: np.ndarray, r: np.ndarray, seed: int, offset: int,
                       rht_signs: int = 0, quantize_operands: bool = True):
-    """dX = BF16(fl32(dX4 + fl32(U' R))), U' = BF16(dY L), dX4 = BF16(Q_sr(dY) Q(W_res))."""
+    """dX_ref = Q_sr(dY) Q(W_res) + g U' R in FP64, U' = BF16(fl32(fl32(dY L) / g)),
+    g = fl32(S_dY S_W) (reading 12).  Returns (dX_ref, parts) as lora_linear_fwd."""
     dy = np.asarray(dy, dtype=F32)
     if quantize_operands:
-        dx4_exact, (a_hat, b_hat), dyq = linear_dgrad_ref(dy, w_res_q, seed, offset, rht_signs=rht_signs)
+        prod, (a_hat, b_hat), dyq = linear_dgrad_ref(dy, w_res_q, seed, offset, rht_signs=rht_signs)
+        g = F32(F32(dyq["row"][2]) * F32(w_res_q["col"][2]))
     else:
-        dx4_exact, (a_hat, b_hat), dyq = gemm_ref(dy, np.asarray(w_res_q, dtype=F32).T), (dy, None), None
-    dx4 = bf16_round(dx4_exact.astype(F32))
-    u = lora_project(dy, np.asarray(l, dtype=F32).T)
-    return lora_expand_add(dx4, u, np.asarray(r, dtype=F32).T), {"dx4": dx4, "dx4_exact": dx4_exact, "u": u,
-                                                                  "a_hat": a_hat, "b_hat": b_hat, "dyq": dyq}
+        w_res = np.asarray(w_res_q, dtype=F32)
+        prod, (a_hat, b_hat), dyq = gemm_ref(dy, w_res.T), (dy, w_res.T.copy()), None
+        g = F32(1.0)
+    u = lora_project_scaled(dy, np.asarray(l, dtype=F32).T, g)
+    dx_ref, scale = _lora_compose(prod, a_hat, b_hat, u, np.asarray(r, dtype=F32).T, g)
+    return dx_ref, {"prod": prod, "u": u, "g": g, "a_hat": a_hat, "b_hat": b_hat, "dyq": dyq,
+                    "abs_scale": scale}

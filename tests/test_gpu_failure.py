@@ -26,3 +26,32 @@ def test_skipped_tile_load_reports_timeout_and_context_survives(monkeypatch):
     assert_layout_equal(rq, ref["row"], "row after the injected timeout")
     assert_layout_equal(cq, ref["col"], "col after the injected timeout")
     api.get_status()
+
+
+def test_gemm_skipped_stage_reports_timeout_and_context_survives(monkeypatch):
+    """The same for the CTA-pair GEMM: with NVFP4_INJECT_GEMM_SKIP_STAGE=3 the first CTA
+    pair never loads its fourth K-stage, so the MMA issuers' bounded wait runs out; every
+    role of both CTAs winds down with bounded waits and frees its tensor memory, the
+    library reports NVFP4_ERR_TIMEOUT, and the next GEMM is within the bound."""
+    import torch
+
+    from tests.helpers import gemm_check
+
+    M, N, K = 512, 512, 2048                                 # 8 K-stages per tile, 4 tiles
+    a = synthetic.normal((M, K), 1.0, seed=17, device="cuda")
+    b = synthetic.normal((N, K), 1.0, seed=18, device="cuda")
+    qa, _ = api.quantize(a)
+    qb, _ = api.quantize(b)
+    api.get_status()
+    monkeypatch.setenv("NVFP4_INJECT_GEMM_SKIP_STAGE", "3")
+    api.gemm(qa, qb, out_dtype=torch.float32)
+    with pytest.raises(_lib.NVFP4Error) as err:
+        api.get_status()
+    assert err.value.status == _lib.NVFP4_ERR_TIMEOUT
+    api.get_status()
+    monkeypatch.delenv("NVFP4_INJECT_GEMM_SKIP_STAGE")
+    c = api.gemm(qa, qb, out_dtype=torch.float32)
+    api.get_status()
+    ra = O.quantize(bf16_to_np(a))["row"]
+    rb = O.quantize(bf16_to_np(b))["row"]
+    assert gemm_check(c.cpu().numpy(), O.dequantize(*ra), O.dequantize(*rb)) <= 1.0

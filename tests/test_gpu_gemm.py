@@ -113,3 +113,21 @@ def test_gemm_large_k_accumulation():
 
 def test_status_clean_after_gemms():
     api.get_status()
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_accumulate_multiwave(out_dtype):
+    """C += alpha * A . B^T over many persistent tiles (2304 x 3200: 9 x 12.5 tiles of
+    256 x 256, a ragged raster group and a 128-column N tail), every element checked."""
+    M, N, K = 2304, 3200, 512
+    a, b = operands(M, N, K, seed=77)
+    qa, qb, ah, bh = quantised_pair(a, b)
+    g = torch.Generator(device="cuda").manual_seed(9)
+    c0 = (torch.randn((M, N), generator=g, device="cuda") * 4).to(out_dtype)
+    c = c0.clone()
+    api.gemm(qa, qb, alpha=-0.5, accumulate=True, out=c)
+    torch.cuda.synchronize()
+    ratio = gemm_check(c.float().cpu().numpy(), ah, bh, alpha=-0.5, c0=c0.float().cpu().numpy(),
+                       bf16=out_dtype == torch.bfloat16)
+    assert ratio <= 1.0, ratio
+    api.get_status()

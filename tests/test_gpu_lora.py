@@ -4,9 +4,13 @@
 - U = BF16(A B^T) and Y <- BF16(Y + U C^T): tensor-core products with FP32
   accumulation, held to the GEMM bound of the exact product plus one BF16 half-ulp
   (the BF16 reading), for every rank, both operand layouts, several CTAs and tiles.
-- The composed fprop and dgrad: within the bound derived from those steps (each side
-  rounds U and the NVFP4 product to BF16 on its own, so they may differ by an ulp of
-  each), plus the page's claim that the decomposition lowers the output error.
+- U' = BF16(A B^T / g) (the projection pre-divided by the tensor-scale product g) and
+  the NVFP4 GEMM with the rank-r term in its accumulator, BF16(g (A B^T + U V^T)):
+  within the GEMM bound over both products plus one BF16 half-ulp, several ranks,
+  tiles, a ragged N and a half-empty last row block.
+- The composed fprop and dgrad: within that bound plus one BF16 ulp of each U' (each
+  side rounds U' on its own), plus the page's claim that the decomposition lowers the
+  output error.
 - At the 12B up-projection size, sampled rows of every step.
 """
 
@@ -87,12 +91,57 @@ def test_expand_add_within_bound(rank, c_trans):
     within(bf16_to_np(yd), pre, O.gemm_abs_ref(u, c), "Y + U C^T")
 
 
-def lora_bound(parts_u, l_like, y4_exact, y4_ref, y_ref, a_hat, b_hat):
-    """|Y_gpu - Y_ref|: the NVFP4 GEMM bound and one BF16 ulp of its rounded value, the
-    low-rank product's bound and one ulp of each U (2^-7 |U| |L|), one ulp of Y."""
-    ul = np.abs(parts_u).astype(np.float64) @ np.abs(l_like).astype(np.float64).T
-    return (O.gemm_tolerance(a_hat, b_hat) + 2.0 ** -7 * np.abs(y4_ref) + 1e-5 * ul + 2.0 ** -7 * ul
-            + 2.0 ** -7 * np.abs(y_ref) + 1e-6)
+def lora_bound(parts, c_like, y_ref):
+    """|Y_gpu - Y_ref| for the fused LoRA-SVD output: the GEMM bound over both products
+    (1e-5 sum|ab| + 1e-6), one BF16 ulp of each U' (2^-7 g |U'| |C|), and one BF16
+    half-ulp of the output (2^-8 |Y_ref|)."""
+    ul = float(parts["g"]) * (np.abs(parts["u"]).astype(np.float64) @ np.abs(c_like).astype(np.float64).T)
+    return 1e-5 * parts["abs_scale"] + 1e-6 + 2.0 ** -7 * ul + 2.0 ** -8 * np.abs(y_ref)
+
+
+@pytest.mark.parametrize("rank", [16, 32, 48, 64])
+@pytest.mark.parametrize("b_trans", [False, True])
+def test_project_scaled_within_bound(rank, b_trans):
+    m, k = 192, 320
+    a = synthetic.normal((m, k), 1.0, seed=rank + 7, device="cuda")
+    b = synthetic.normal((rank, k), 0.05, seed=rank + 8, device="cuda")
+    sa = torch.tensor([3.0e-3], device="cuda")
+    sb = torch.tensor([5.5e-5], device="cuda")
+    av, bv = bf16_to_np(a), bf16_to_np(b)
+    arg = b.t().contiguous() if b_trans else b
+    u = api.lowrank_project_scaled(a, arg, sa, sb, b_trans=b_trans)
+    g = np.float32(np.float32(3.0e-3) * np.float32(5.5e-5))
+    inv = np.float32(np.float32(1.0) / g)
+    # the sum's FP32 rounding may differ from the exact one; then the scaled value is
+    # within the GEMM bound of fl32(exact) * inv, and BF16 rounding adds a half-ulp
+    pre = O.gemm_ref(av, bv) * float(inv)
+    within(bf16_to_np(u), pre, O.gemm_abs_ref(av, bv) * float(inv), "U'")
+    exact_path = O.lora_project_scaled(av, bv, g)
+    assert np.mean(bf16_to_np(u) == exact_path) > 0.95
+
+
+@pytest.mark.parametrize("m,n,k,rank", [(256, 256, 256, 32), (384, 640, 512, 16), (512, 384, 1024 + 64, 64),
+                                        (768, 512, 768, 48)])
+def test_gemm_lowrank_within_bound(m, n, k, rank):
+    a = synthetic.normal((m, k), 1.0, seed=m + 1, device="cuda", outlier_frac=0.01, outlier_mult=50.0)
+    b = synthetic.normal((n, k), 0.02, seed=n + 2, device="cuda")
+    qa, _ = api.quantize(a)
+    qb, _ = api.quantize(b)
+    ra, rb = O.quantize(bf16_to_np(a))["row"], O.quantize(bf16_to_np(b))["row"]
+    ah, bh = O.dequantize(*ra), O.dequantize(*rb)
+    rng = np.random.default_rng(rank)
+    uv = O.bf16_round(rng.standard_normal((m, rank)).astype(np.float32) * 50)
+    vv = O.bf16_round((0.3 * rng.standard_normal((n, rank))).astype(np.float32))
+    c = api.gemm_lowrank(qa, qb, to_dev(uv), to_dev(vv))
+    api.get_status()
+    g = np.float32(np.float32(ra[2]) * np.float32(rb[2]))
+    ref = O.gemm_ref(ah, bh) + float(g) * O.gemm_ref(uv, vv)
+    scale = O.gemm_abs_ref(ah, bh) + float(g) * O.gemm_abs_ref(uv, vv)
+    bound = 1e-5 * scale + 1e-6 + 2.0 ** -8 * np.abs(ref)
+    ratio = np.abs(bf16_to_np(c).astype(np.float64) - ref) / bound
+    assert (ratio <= 1.0).all(), float(ratio.max())
+    # the low-rank term is really there: it moves the output by far more than the bound
+    assert np.abs(float(g) * O.gemm_ref(uv, vv)).max() > 100 * bound.max()
 
 
 def spiked_weight(n, k, seed):
@@ -116,7 +165,7 @@ def test_lora_fwd_and_dgrad(m, n, k, rank):
     xv = bf16_to_np(x)
     y, _, _ = api.lora_linear_fwd(x, wq_row, ld, rd, rht_signs=SIGNS)
     y_ref, p = O.lora_linear_fwd(xv, wq, l, r, rht_signs=SIGNS)
-    bound = lora_bound(p["u"], l, p["y4_exact"], p["y4"], y_ref, p["a_hat"], p["b_hat"])
+    bound = lora_bound(p, l, y_ref)
     err = np.abs(bf16_to_np(y).astype(np.float64) - y_ref)
     assert (err <= bound).all(), float((err / bound).max())
     exact = xv.astype(np.float64) @ wv.T.astype(np.float64)
@@ -127,9 +176,9 @@ def test_lora_fwd_and_dgrad(m, n, k, rank):
 
     dy = synthetic.normal((m, n), 1e-3, seed=m + 1, device="cuda")
     dyv = bf16_to_np(dy)
-    dx, _, _ = api.lora_linear_dgrad(dy, wq_col, ld, rd, seed=77, offset=3, rht_signs=SIGNS)
+    dx, _, _ = api.lora_linear_dgrad(dy, wq_col, ld, to_dev(r.T.copy()), seed=77, offset=3, rht_signs=SIGNS)
     dx_ref, p = O.lora_linear_dgrad(dyv, wq, l, r, seed=77, offset=3, rht_signs=SIGNS)
-    bound = lora_bound(p["u"], r.T, p["dx4_exact"], p["dx4"], dx_ref, p["a_hat"], p["b_hat"])
+    bound = lora_bound(p, r.T, dx_ref)
     err = np.abs(bf16_to_np(dx).astype(np.float64) - dx_ref)
     assert (err <= bound).all(), float((err / bound).max())
     api.get_status()

@@ -1,8 +1,10 @@
 """Pins of the oracle's LoRA-SVD linear (NVFP4 residual weight plus a BF16 low-rank
-branch): the decomposition is an identity without quantisation, zero factors reduce it
-to the plain NVFP4 linear, the residual's FP32 accumulation order is the stated one, the
-low-rank products match brute force, and -- the claim of the page -- moving the top
-singular directions out of the 4-bit path lowers the error of the layer's output."""
+branch that joins the NVFP4 accumulator): the decomposition is an identity without
+quantisation, zero factors reduce it to the plain NVFP4 linear, the residual's FP32
+accumulation order is the stated one, the low-rank products (plain and pre-divided by
+the tensor-scale product) match brute force, a power-of-two scale product divides out
+exactly, and -- the claim of the page -- moving the top singular directions out of the
+4-bit path lowers the error of the layer's output."""
 
 import numpy as np
 import pytest
@@ -56,13 +58,14 @@ def test_zero_factors_reduce_to_the_plain_linear():
     w = O.bf16_round((0.02 * rng.standard_normal((96, 128))).astype(np.float32))
     l, r = np.zeros((96, 16), np.float32), O.bf16_round(rng.standard_normal((16, 128)).astype(np.float32))
     wq = O.quantize_weight(O.lora_residual(w, l, r))
-    y, _ = O.lora_linear_fwd(x, wq, l, r, rht_signs=0x5A3C)
-    y_plain, _, _ = O.linear_fwd_ref(x, O.quantize_weight(w), rht_signs=0x5A3C)
-    assert np.array_equal(y, O.bf16_round(y_plain.astype(np.float32)))
+    y, parts = O.lora_linear_fwd(x, wq, l, r, rht_signs=0x5A3C)
+    y_plain, (ah, bh), _ = O.linear_fwd_ref(x, O.quantize_weight(w), rht_signs=0x5A3C)
+    assert np.array_equal(y, y_plain)
+    assert np.array_equal(parts["abs_scale"], O.gemm_abs_ref(ah, bh))
     dy = O.bf16_round((1e-3 * rng.standard_normal((64, 96))).astype(np.float32))
     dx, _ = O.lora_linear_dgrad(dy, wq, l, r, seed=5, offset=0, rht_signs=0x5A3C)
     dx_plain, _, _ = O.linear_dgrad_ref(dy, O.quantize_weight(w), 5, 0, rht_signs=0x5A3C)
-    assert np.array_equal(dx, O.bf16_round(dx_plain.astype(np.float32)))
+    assert np.array_equal(dx, dx_plain)
 
 
 def test_low_rank_products_match_brute_force():
@@ -100,3 +103,45 @@ def test_moving_top_singular_directions_out_of_fp4_lowers_the_error():
     e_plain = np.linalg.norm(y_plain - exact) / np.linalg.norm(exact)
     e_lora = np.linalg.norm(y_lora - exact) / np.linalg.norm(exact)
     assert e_lora < 0.5 * e_plain, (e_lora, e_plain)
+
+
+def test_scaled_projection_matches_brute_force():
+    """U' = BF16(fl32(fl32(sum) * fl32(1 / g))) element by element, for a g that is not a
+    power of two; and for g = 2^-9 the division is exact, so U' g equals the plain U."""
+    rng = np.random.default_rng(11)
+    a = O.bf16_round(rng.standard_normal((6, 48)).astype(np.float32))
+    b = O.bf16_round(rng.standard_normal((5, 48)).astype(np.float32))
+    g = np.float32(3.0e-4)
+    inv = np.float32(np.float32(1.0) / g)
+    u = O.lora_project_scaled(a, b, g)
+    for i in range(6):
+        for j in range(5):
+            s = np.float32(sum(float(a[i, k]) * float(b[j, k]) for k in range(48)))
+            assert u[i, j] == O.bf16_round(np.float32(s * inv))
+    g2 = np.float32(2.0 ** -9)
+    assert np.array_equal(O.lora_project_scaled(a, b, g2) * g2, O.lora_project(a, b))
+
+
+def test_fused_reference_adds_the_scaled_low_rank_product():
+    """The fused reference is the NVFP4 product plus g U' L^T, where g is the product of
+    the two tensor scales: checked against a hand composition from the quantised layouts
+    (a wrong scale, a missing factor g or a transposed factor fails it)."""
+    rng = np.random.default_rng(12)
+    m, n, k, rank = 32, 64, 96, 16
+    x = O.bf16_round(rng.standard_normal((m, k)).astype(np.float32))
+    w = O.bf16_round((0.02 * rng.standard_normal((n, k))).astype(np.float32))
+    l = O.bf16_round((0.05 * rng.standard_normal((n, rank))).astype(np.float32))
+    r = O.bf16_round((0.05 * rng.standard_normal((rank, k))).astype(np.float32))
+    wq = O.quantize_weight(O.lora_residual(w, l, r))
+    y, parts = O.lora_linear_fwd(x, wq, l, r)
+    xq = O.quantize(x, emit_row=True)["row"]
+    g = np.float32(np.float32(xq[2]) * np.float32(wq["row"][2]))
+    assert parts["g"] == g
+    u = O.bf16_round((np.float32(1.0) / g * (x.astype(np.float64) @ r.T.astype(np.float64)).astype(np.float32))
+                     .astype(np.float32))
+    want = O.dequantize(*xq).astype(np.float64) @ O.dequantize(*wq["row"]).astype(np.float64).T + \
+        float(g) * (u.astype(np.float64) @ l.T.astype(np.float64))
+    assert np.allclose(y, want, rtol=1e-12, atol=1e-12)
+    # g U' approximates the plain projection within one BF16 rounding
+    plain = x.astype(np.float64) @ r.T.astype(np.float64)
+    assert np.all(np.abs(float(g) * parts["u"] - plain) <= 2.0 ** -8 * np.abs(plain) + 1e-30)
