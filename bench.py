@@ -807,9 +807,11 @@ def run_layer(args):
     """The four linears of a 3B-class decoder layer at 32768 tokens (QKV 3072->9216, O
     3072->3072, gate-up 3072->16384, down 8192->3072): forward through the layer, then
     backward in reverse, every linear with W quantised (2D), fprop, dgrad and wgrad.
-    Timed two ways on one GPU: everything in order on one stream, and each wgrad on a
+    Timed three ways on one GPU: everything in order on one stream; each wgrad on a
     second stream so it can fill the SMs that the next dgrad's quantiser and GEMM leave
-    idle.  Inputs are resident and each larger than L2."""
+    idle; and the four wgrads deferred to the end of the backward pass and run as one
+    grouped launch (nvfp4_gemm_grouped).  The four wgrad GEMMs alone are also timed
+    separately and grouped.  Inputs are resident and each larger than L2."""
     from nvfp4_pretraining_linear_b200 import api, synthetic as syn
     torch.cuda.set_device(0)
     names = list(syn.LAYER3B["linears"])
@@ -851,6 +853,14 @@ def run_layer(args):
         done.record(side)
         main.wait_event(done)
 
+    def step_grouped(ev):
+        forward(PhaseEvents(False))
+        for L in reversed(linears):
+            api.linear_dgrad(L.dy, L.wq_col, seed=SR_SEED, rht_signs=RHT_SIGNS, out=L.dx, dyq_row=L.dyq_row,
+                             dyq_col=L.dyq_col)
+        # the four weight gradients in one persistent launch over all their tiles
+        api.gemm_grouped([(L.dyq_col, L.xq_col) for L in linears], outs=[L.dw for L in linears])
+
     def timed(fn):
         for _ in range(args.warmup):
             fn(PhaseEvents(False))
@@ -865,10 +875,32 @@ def run_layer(args):
             ts.append(a.elapsed_time(b))
         return statistics.median(ts)
 
+    def timed_wgrads(grouped):
+        def fn():
+            if grouped:
+                api.gemm_grouped([(L.dyq_col, L.xq_col) for L in linears], outs=[L.dw for L in linears])
+            else:
+                for L in linears:
+                    api.gemm(L.dyq_col, L.xq_col, out=L.dw)
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
     clocks = ClockSampler(0)
     t_seq = timed(step_in_order)
     clock_info = clocks.stop()
     t_side = timed(step_side_stream)
+    t_grouped = timed(step_grouped)
+    t_wg_sep, t_wg_grp = timed_wgrads(False), timed_wgrads(True)
     ev = PhaseEvents(True)
     step_in_order(ev)
     torch.cuda.synchronize()
@@ -876,7 +908,8 @@ def run_layer(args):
     api.get_status()
     print(json.dumps({
         "kernel": "layer", "workload": "layer3b-decoder-linears-32768-tokens", "gemm_tflop_per_step": flops / 1e12,
-        "ms_in_order": t_seq, "ms_wgrad_side_stream": t_side, "value": flops / (t_seq * 1e-3) / 1e12,
+        "ms_in_order": t_seq, "ms_wgrad_side_stream": t_side, "ms_wgrad_grouped": t_grouped,
+        "wgrads_ms_separate": t_wg_sep, "wgrads_ms_grouped": t_wg_grp, "value": flops / (t_seq * 1e-3) / 1e12,
         "unit": "TFLOP/s (12 GEMMs, 2MNK each, per step time)", "phase_ms": phases,
         "gemm_tflops_in_step": flops / (phases.get("g", float("nan")) * 1e-3) / 1e12,
         "steps": args.steps, "l2": "inputs larger than L2, no flush", "clocks": clock_info}), flush=True)

@@ -184,6 +184,19 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, i
 nvfp4_status nvfp4_gemm_amax(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc,
                              float alpha, uint32_t rht_signs, float* amax_out, void* stream);
 
+/* Several NVFP4 GEMMs in one persistent launch: C_i = S_Ai * S_Bi * A_i . B_i^T for
+ * i < count (count <= 8), each as nvfp4_gemm with alpha 1 and no accumulation, all with
+ * the same output type.  The output tiles of all problems form one queue that the CTA
+ * pairs of a single grid work through, so the last, partial wave of one problem's tiles
+ * overlaps the next problem's instead of leaving SMs idle between launches -- e.g. the
+ * weight-gradient GEMMs of a layer's linears, deferred to the end of its backward pass
+ * (whole-layer scheduling of the linears whose GEMMs the 12B NVFP4 page's recipe
+ * quantises).  A[i], B[i]: host arrays of count tensor pointers; C[i], ldc[i]: outputs.
+ * Requires per problem M, N, K > 0, M % 128 == 0, N % 128 == 0, K % 64 == 0, 16-byte
+ * aligned C rows, and the CTA-pair kernel. */
+nvfp4_status nvfp4_gemm_grouped(const nvfp4_tensor* const* A, const nvfp4_tensor* const* B, void* const* C,
+                                const int64_t* ldc, int32_t count, int32_t out_dtype, void* stream);
+
 /* Linear forward (fprop): Y [M x N] = Q(X) . Q(W)^T.
  *   X      : BF16 [M x K] activations (device, row stride ldx), quantised here
  *            row-wise with round-to-nearest-even into Xq_row (caller buffers,

@@ -89,6 +89,8 @@ SIGNATURES = {
                                         c_void_p, c_int64, c_void_p]),
     "nvfp4_lowrank_project_scaled": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_int32,
                                                 c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_void_p]),
+    "nvfp4_gemm_grouped": (c_int32, [ctypes.POINTER(T_P), ctypes.POINTER(T_P), ctypes.POINTER(c_void_p),
+                                      ctypes.POINTER(c_int64), c_int32, c_int32, c_void_p]),
     "nvfp4_gemm_lowrank": (c_int32, [T_P, T_P, c_void_p, c_int64, c_void_p, c_int64, c_int32, c_void_p, c_int64,
                                       c_void_p]),
     "nvfp4_lowrank_expand_add": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_void_p, c_int64,

@@ -6,6 +6,7 @@ library.  There is no CPU path: calls fail when the library or a GPU is missing.
 """
 
 import ctypes
+import os
 from dataclasses import dataclass
 from typing import Optional
 
@@ -15,6 +16,18 @@ from . import _lib
 from ._lib import OUT_BF16, OUT_F32, SCALE_MMA, SCALE_ROWMAJOR, NVFP4Error  # noqa: F401
 
 _workspaces = {}
+
+# With NVFP4_CHECK_STATUS=1 in the environment every call below synchronises its stream
+# and raises on a recorded device-side error (a bounded wait that gave up), at the call
+# that caused it.  Off by default: the library's calls are asynchronous, and a training
+# step normally checks nvfp4_get_status once (get_status() here) before using results.
+_CHECK_EACH_CALL = os.environ.get("NVFP4_CHECK_STATUS", "") not in ("", "0")
+
+
+def _checked(status, stream=None):
+    _lib.check(status)
+    if _CHECK_EACH_CALL:
+        _lib.check(_lib.load().nvfp4_get_status(_stream_ptr(stream)))
 
 
 def _stream_ptr(stream=None):
@@ -79,8 +92,8 @@ def quantize(x: torch.Tensor, *, emit_row=True, emit_col=False, stochastic=False
     ws = workspace(x.device, stream)
     rs = out_row.struct() if emit_row else None
     cs = out_col.struct() if emit_col else None
-    _lib.check(lib.nvfp4_quantize(x.data_ptr(), rows, cols, x.stride(0), opts, rs, cs, ws.data_ptr(), ws.numel(),
-                                  _stream_ptr(stream)))
+    _checked(lib.nvfp4_quantize(x.data_ptr(), rows, cols, x.stride(0), opts, rs, cs, ws.data_ptr(), ws.numel(),
+                                  _stream_ptr(stream)), stream)
     return (out_row if emit_row else None), (out_col if emit_col else None)
 
 
@@ -89,7 +102,7 @@ def dequantize(q: QTensor, out_dtype=torch.float32, out: Optional[torch.Tensor] 
     if out is None:
         out = torch.empty((q.rows, q.cols), dtype=out_dtype, device=q.codes.device)
     code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
-    _lib.check(lib.nvfp4_dequantize(q.struct(), out.data_ptr(), out.stride(0), code, _stream_ptr(stream)))
+    _checked(lib.nvfp4_dequantize(q.struct(), out.data_ptr(), out.stride(0), code, _stream_ptr(stream)), stream)
     return out
 
 
@@ -100,9 +113,29 @@ def gemm(A: QTensor, B: QTensor, out_dtype=torch.bfloat16, alpha=1.0, accumulate
     if out is None:
         out = (torch.zeros if accumulate else torch.empty)((A.rows, B.rows), dtype=out_dtype, device=A.codes.device)
     code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
-    _lib.check(lib.nvfp4_gemm(A.struct(), B.struct(), out.data_ptr(), out.stride(0), code, alpha, int(accumulate),
-                              _stream_ptr(stream)))
+    _checked(lib.nvfp4_gemm(A.struct(), B.struct(), out.data_ptr(), out.stride(0), code, alpha, int(accumulate),
+                              _stream_ptr(stream)), stream)
     return out
+
+
+def gemm_grouped(problems, out_dtype=torch.float32, outs=None, stream=None):
+    """nvfp4_gemm_grouped: C_i = S_Ai S_Bi A_i . B_i^T for up to 8 (A_i, B_i) pairs in one
+    persistent launch (the tiles of all problems form one queue).  Returns the outputs."""
+    lib = _lib.load()
+    n = len(problems)
+    if outs is None:
+        outs = [torch.empty((a.rows, b.rows), dtype=out_dtype, device=a.codes.device) for a, b in problems]
+    code = OUT_F32 if outs[0].dtype == torch.float32 else OUT_BF16
+    if any(o.dtype != outs[0].dtype for o in outs):
+        raise ValueError("all outputs of a grouped GEMM have one type")
+    sa = [a.struct() for a, _ in problems]
+    sb = [b.struct() for _, b in problems]
+    arr_a = (ctypes.POINTER(_lib.NVFP4Tensor) * n)(*[ctypes.pointer(x) for x in sa])
+    arr_b = (ctypes.POINTER(_lib.NVFP4Tensor) * n)(*[ctypes.pointer(x) for x in sb])
+    arr_c = (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs])
+    arr_ld = (ctypes.c_int64 * n)(*[o.stride(0) for o in outs])
+    _checked(lib.nvfp4_gemm_grouped(arr_a, arr_b, arr_c, arr_ld, n, code, _stream_ptr(stream)), stream)
+    return outs
 
 
 def gemm_amax(A: QTensor, B: QTensor, alpha=1.0, rht_signs=0, out: Optional[torch.Tensor] = None,
@@ -114,8 +147,8 @@ def gemm_amax(A: QTensor, B: QTensor, alpha=1.0, rht_signs=0, out: Optional[torc
         out = torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=A.codes.device)
     if amax is None:
         amax = torch.empty(3, dtype=torch.float32, device=A.codes.device)
-    _lib.check(lib.nvfp4_gemm_amax(A.struct(), B.struct(), out.data_ptr(), out.stride(0), alpha, rht_signs & 0xFFFF,
-                                   amax.data_ptr(), _stream_ptr(stream)))
+    _checked(lib.nvfp4_gemm_amax(A.struct(), B.struct(), out.data_ptr(), out.stride(0), alpha, rht_signs & 0xFFFF,
+                                   amax.data_ptr(), _stream_ptr(stream)), stream)
     return out, amax
 
 
@@ -140,8 +173,8 @@ def linear_fwd(x: torch.Tensor, wq_row: QTensor, *, save_col=True, rht_signs=0, 
     code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
     xr = xq_row.struct()
     xc = xq_col.struct() if save_col else None
-    _lib.check(lib.nvfp4_linear_fwd(x.data_ptr(), M, K, x.stride(0), wq_row.struct(), out.data_ptr(), out.stride(0),
-                                    code, xr, xc, rht_signs, ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
+    _checked(lib.nvfp4_linear_fwd(x.data_ptr(), M, K, x.stride(0), wq_row.struct(), out.data_ptr(), out.stride(0),
+                                    code, xr, xc, rht_signs, ws.data_ptr(), ws.numel(), _stream_ptr(stream)), stream)
     return out, xq_row, (xq_col if save_col else None)
 
 
@@ -161,9 +194,9 @@ def linear_dgrad(dy: torch.Tensor, wq_col: QTensor, *, seed, offset=0, save_col=
     code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
     dr = dyq_row.struct()
     dc = dyq_col.struct() if save_col else None
-    _lib.check(lib.nvfp4_linear_dgrad(dy.data_ptr(), M, N, dy.stride(0), wq_col.struct(), out.data_ptr(),
+    _checked(lib.nvfp4_linear_dgrad(dy.data_ptr(), M, N, dy.stride(0), wq_col.struct(), out.data_ptr(),
                                       out.stride(0), code, dr, dc, seed, offset, rht_signs, ws.data_ptr(), ws.numel(),
-                                      _stream_ptr(stream)))
+                                      _stream_ptr(stream)), stream)
     return out, dyq_row, (dyq_col if save_col else None)
 
 
@@ -175,8 +208,8 @@ def linear_wgrad(dyq_col: QTensor, xq_col: QTensor, *, out_dtype=torch.bfloat16,
         out = (torch.zeros if accumulate else torch.empty)((dyq_col.rows, xq_col.rows), dtype=out_dtype,
                                                            device=dyq_col.codes.device)
     code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
-    _lib.check(lib.nvfp4_linear_wgrad(dyq_col.struct(), xq_col.struct(), out.data_ptr(), out.stride(0), code,
-                                      int(accumulate), _stream_ptr(stream)))
+    _checked(lib.nvfp4_linear_wgrad(dyq_col.struct(), xq_col.struct(), out.data_ptr(), out.stride(0), code,
+                                      int(accumulate), _stream_ptr(stream)), stream)
     return out
 
 
@@ -206,9 +239,9 @@ def newton_schulz(g: torch.Tensor, iters: int, *, normalize=True, out: Optional[
         norm = torch.empty(1, dtype=torch.float32, device=g.device)
     if workspace is None:
         workspace = newton_schulz_workspace(m, n, g.device)
-    _lib.check(lib.nvfp4_newton_schulz(g.data_ptr(), m, n, g.stride(0), out.data_ptr(), out.stride(0), int(iters),
+    _checked(lib.nvfp4_newton_schulz(g.data_ptr(), m, n, g.stride(0), out.data_ptr(), out.stride(0), int(iters),
                                        int(normalize), _ptr(norm) if normalize else None, workspace.data_ptr(),
-                                       workspace.numel(), _stream_ptr(stream)))
+                                       workspace.numel(), _stream_ptr(stream)), stream)
     return out, (norm if normalize else None)
 
 
@@ -227,8 +260,8 @@ def lora_residual(w: torch.Tensor, l: torch.Tensor, r: torch.Tensor, out: Option
     rank = l.shape[1]
     if out is None:
         out = torch.empty_like(w)
-    _lib.check(lib.nvfp4_lora_residual(w.data_ptr(), N, K, w.stride(0), l.data_ptr(), l.stride(0), r.data_ptr(),
-                                       r.stride(0), rank, out.data_ptr(), out.stride(0), _stream_ptr(stream)))
+    _checked(lib.nvfp4_lora_residual(w.data_ptr(), N, K, w.stride(0), l.data_ptr(), l.stride(0), r.data_ptr(),
+                                       r.stride(0), rank, out.data_ptr(), out.stride(0), _stream_ptr(stream)), stream)
     return out
 
 
@@ -242,8 +275,8 @@ def lowrank_project(a: torch.Tensor, b: torch.Tensor, *, b_trans=False, out: Opt
     rank = b.shape[1] if b_trans else b.shape[0]
     if out is None:
         out = torch.empty((M, rank), dtype=torch.bfloat16, device=a.device)
-    _lib.check(lib.nvfp4_lowrank_project(a.data_ptr(), M, K, a.stride(0), b.data_ptr(), b.stride(0), int(b_trans),
-                                         rank, out.data_ptr(), out.stride(0), _stream_ptr(stream)))
+    _checked(lib.nvfp4_lowrank_project(a.data_ptr(), M, K, a.stride(0), b.data_ptr(), b.stride(0), int(b_trans),
+                                         rank, out.data_ptr(), out.stride(0), _stream_ptr(stream)), stream)
     return out
 
 
@@ -258,9 +291,9 @@ def lowrank_project_scaled(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tens
     rank = b.shape[1] if b_trans else b.shape[0]
     if out is None:
         out = torch.empty((M, rank), dtype=torch.bfloat16, device=a.device)
-    _lib.check(lib.nvfp4_lowrank_project_scaled(a.data_ptr(), M, K, a.stride(0), b.data_ptr(), b.stride(0),
+    _checked(lib.nvfp4_lowrank_project_scaled(a.data_ptr(), M, K, a.stride(0), b.data_ptr(), b.stride(0),
                                                 int(b_trans), rank, scale_a.data_ptr(), scale_b.data_ptr(),
-                                                out.data_ptr(), out.stride(0), _stream_ptr(stream)))
+                                                out.data_ptr(), out.stride(0), _stream_ptr(stream)), stream)
     return out
 
 
@@ -272,8 +305,8 @@ def gemm_lowrank(A: QTensor, B: QTensor, u: torch.Tensor, v: torch.Tensor, out: 
     _bf16_matrix(v, "v")
     if out is None:
         out = torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=A.codes.device)
-    _lib.check(lib.nvfp4_gemm_lowrank(A.struct(), B.struct(), u.data_ptr(), u.stride(0), v.data_ptr(), v.stride(0),
-                                      u.shape[1], out.data_ptr(), out.stride(0), _stream_ptr(stream)))
+    _checked(lib.nvfp4_gemm_lowrank(A.struct(), B.struct(), u.data_ptr(), u.stride(0), v.data_ptr(), v.stride(0),
+                                      u.shape[1], out.data_ptr(), out.stride(0), _stream_ptr(stream)), stream)
     return out
 
 
@@ -284,8 +317,8 @@ def lowrank_expand_add(y: torch.Tensor, u: torch.Tensor, c: torch.Tensor, *, c_t
         _bf16_matrix(t, nm)
     M, N = y.shape
     rank = u.shape[1]
-    _lib.check(lib.nvfp4_lowrank_expand_add(y.data_ptr(), M, N, y.stride(0), u.data_ptr(), u.stride(0), c.data_ptr(),
-                                            c.stride(0), int(c_trans), rank, _stream_ptr(stream)))
+    _checked(lib.nvfp4_lowrank_expand_add(y.data_ptr(), M, N, y.stride(0), u.data_ptr(), u.stride(0), c.data_ptr(),
+                                            c.stride(0), int(c_trans), rank, _stream_ptr(stream)), stream)
     return y
 
 
@@ -312,9 +345,9 @@ def lora_linear_fwd(x: torch.Tensor, wq_res_row: QTensor, l: torch.Tensor, r: to
         xq_col = QTensor.empty(K, M, SCALE_MMA, x.device)
     ws = workspace(x.device, stream)
     xc = xq_col.struct() if save_col else None
-    _lib.check(lib.nvfp4_lora_linear_fwd(x.data_ptr(), M, K, x.stride(0), wq_res_row.struct(), l.data_ptr(),
+    _checked(lib.nvfp4_lora_linear_fwd(x.data_ptr(), M, K, x.stride(0), wq_res_row.struct(), l.data_ptr(),
                                          r.data_ptr(), rank, out.data_ptr(), out.stride(0), xq_row.struct(), xc,
-                                         rht_signs, u.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
+                                         rht_signs, u.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream)), stream)
     return out, xq_row, (xq_col if save_col else None)
 
 
@@ -341,10 +374,10 @@ def lora_linear_dgrad(dy: torch.Tensor, wq_res_col: QTensor, l: torch.Tensor, rt
         dyq_col = QTensor.empty(N, M, SCALE_MMA, dy.device)
     ws = workspace(dy.device, stream)
     dc = dyq_col.struct() if save_col else None
-    _lib.check(lib.nvfp4_lora_linear_dgrad(dy.data_ptr(), M, N, dy.stride(0), wq_res_col.struct(), l.data_ptr(),
+    _checked(lib.nvfp4_lora_linear_dgrad(dy.data_ptr(), M, N, dy.stride(0), wq_res_col.struct(), l.data_ptr(),
                                            rt.data_ptr(), rank, out.data_ptr(), out.stride(0), dyq_row.struct(), dc,
                                            seed, offset, rht_signs, u.data_ptr(), ws.data_ptr(), ws.numel(),
-                                           _stream_ptr(stream)))
+                                           _stream_ptr(stream)), stream)
     return out, dyq_row, (dyq_col if save_col else None)
 
 
@@ -353,7 +386,7 @@ def check_conversions(n_sr=1 << 26, stream=None):
     conversions against their definitions on the current device; all 0 when conforming."""
     lib = _lib.load()
     counts = torch.zeros(4, dtype=torch.int64, device="cuda")
-    _lib.check(lib.nvfp4_check_conversions(counts.data_ptr(), n_sr, _stream_ptr(stream)))
+    _checked(lib.nvfp4_check_conversions(counts.data_ptr(), n_sr, _stream_ptr(stream)), stream)
     return [int(v) for v in counts[:3].cpu().tolist()]
 
 

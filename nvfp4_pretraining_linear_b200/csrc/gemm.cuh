@@ -628,12 +628,48 @@ __device__ __forceinline__ TileCoord pair_tile_coord(const Params& p, int32_t t)
 // Output modes of the pair kernel's epilogue (one instantiation each).
 enum EpiMode : int { EPI_BF16 = 0, EPI_BF16_ACC = 1, EPI_F32 = 2, EPI_F32_ACC = 3 };
 
-template <int EPI>
+// Tensor maps of one GEMM problem of the pair kernel.
+struct PairMaps {
+  CUtensorMap a, b, sfa, sfb, c;
+};
+
+// The problems one pair-kernel launch works through: MAXP = 1 for a single GEMM, more for
+// a grouped launch (one persistent grid over several GEMMs of the same output mode, e.g.
+// a layer's weight gradients).  Their output tiles form one queue: problem i owns the
+// global tile indices tile_end[i - 1] .. tile_end[i] - 1.  u and v are the low-rank
+// factors of a single GEMM's low-rank stage (unused otherwise).
+template <int MAXP>
+struct PairGroup {
+  PairMaps maps[MAXP];
+  CUtensorMap u, v;
+  Params p[MAXP];
+  int32_t tile_end[MAXP];
+  int32_t count;
+};
+constexpr int kMaxGroup = 8;
+
+struct TileRef {
+  int pi;       // problem
+  int32_t lt;   // tile within the problem
+};
+
+template <int MAXP>
+__device__ __forceinline__ TileRef locate(const PairGroup<MAXP>& g, int32_t t) {
+  int pi = 0;
+  if constexpr (MAXP > 1) {
+    while (pi + 1 < g.count && t >= g.tile_end[pi]) ++pi;
+  }
+  return TileRef{pi, t - (pi ? g.tile_end[pi - 1] : 0)};
+}
+
+template <int MAXP>
+__device__ __forceinline__ int stages_of(const Params& p) {
+  return p.num_k_stages + (p.lr_ksteps ? 1 : 0);
+}
+
+template <int EPI, int MAXP>
 __global__ void __launch_bounds__(P_NUM_THREADS, 1)
-    gemm_kernel_pair(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                     const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
-                     const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ CUtensorMap tma_u,
-                     const __grid_constant__ CUtensorMap tma_v, const Params p) {
+    gemm_kernel_pair(const __grid_constant__ PairGroup<MAXP> grp) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t smem_base = smem_u32(smem);
@@ -691,10 +727,10 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int32_t num_tiles = p.num_m * p.num_n;
+  const int32_t num_tiles = grp.tile_end[grp.count - 1];
   const int32_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
-  // stages per tile: the NVFP4 K-stages, then the low-rank stage when there is one
-  const int tile_stages = p.num_k_stages + (p.lr_ksteps ? 1 : 0);
+  // Each tile's problem p (tensor maps M, parameters p); its stages: the NVFP4 K-stages,
+  // then the low-rank stage when there is one.
   const uint32_t leader_full0 = map_to_cta(full_bar(0), 0);
   const uint32_t leader_acc_empty = map_to_cta(acc_empty, 0);
 
@@ -707,18 +743,25 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       // During the last P_PREFETCH stages of a tile, the first stages of the pair's next
       // tile are prefetched into L2: every pair starts its next tile at about the same
       // time, and without this those first loads all miss L2 at once.
-      const int pf_n = min(P_PREFETCH, p.num_k_stages);
       int64_t q = 0;                                    // stage sequence number over this pair's tiles
       for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
-        const TileCoord tc = pair_tile_coord(p, t);
+        const TileRef tr = locate(grp, t);
+        const Params& p = grp.p[tr.pi];
+        const PairMaps& M = grp.maps[tr.pi];
+        const int tile_stages = stages_of<MAXP>(p);
+        const int pf_n = min(P_PREFETCH, p.num_k_stages);
+        const TileCoord tc = pair_tile_coord(p, tr.lt);
         const bool has_next = t + num_pairs < num_tiles;
-        const TileCoord nc = pair_tile_coord(p, has_next ? t + num_pairs : t);
+        const TileRef nr = locate(grp, has_next ? t + num_pairs : t);
+        const Params& pn = grp.p[nr.pi];
+        const PairMaps& Mn = grp.maps[nr.pi];
+        const TileCoord nc = pair_tile_coord(pn, nr.lt);
         for (int ks = 0; ks < tile_stages; ++ks, ++q) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
-          if (pair == 0 && q == p.skip_stage) {
+          if (pair == 0 && q == grp.p[0].skip_stage) {
             // fault injection: neither CTA loads this stage and the leader never arms its
             // barrier, so the MMA issuers' bounded wait on it expires (kErrTimeout) and
             // every role winds down; nothing is in flight for this stage
@@ -733,17 +776,17 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           if (ks == p.num_k_stages) {
             // low-rank stage: 128 rows x 64 BF16 of U (this CTA's A rows) and of V (its half
             // of the B rows), zero-filled past the rank
-            tma_load_2d_pair(a_smem(stage), &tma_u, 0, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
-            tma_load_2d_pair(b_smem(stage), &tma_v, 0, tc.n_blk * BN + (int32_t)rank * 128, fb);
+            tma_load_2d_pair(a_smem(stage), &grp.u, 0, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
+            tma_load_2d_pair(b_smem(stage), &grp.v, 0, tc.n_blk * BN + (int32_t)rank * 128, fb);
           } else {
             const int32_t kx = ks * BK_BYTES;
-            tma_load_2d_pair(a_smem(stage), &tma_a, kx, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
-            tma_load_2d_pair(b_smem(stage), &tma_b, kx, tc.n_blk * BN + (int32_t)rank * 128, fb);
+            tma_load_2d_pair(a_smem(stage), &M.a, kx, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
+            tma_load_2d_pair(b_smem(stage), &M.b, kx, tc.n_blk * BN + (int32_t)rank * 128, fb);
           }
           const int pf = ks - (p.num_k_stages - pf_n);
-          if (has_next && pf >= 0 && pf < pf_n) {
-            tma_prefetch_2d(&tma_a, pf * BK_BYTES, nc.m_blk * P_BM + (int32_t)rank * 128);
-            tma_prefetch_2d(&tma_b, pf * BK_BYTES, nc.n_blk * BN + (int32_t)rank * 128);
+          if (has_next && pf >= 0 && pf < pf_n && pf < pn.num_k_stages) {
+            tma_prefetch_2d(&Mn.a, pf * BK_BYTES, nc.m_blk * P_BM + (int32_t)rank * 128);
+            tma_prefetch_2d(&Mn.b, pf * BK_BYTES, nc.n_blk * BN + (int32_t)rank * 128);
           }
           if (++stage == P_STAGES) {
             stage = 0;
@@ -770,9 +813,11 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       int64_t q = 0;                                    // stage sequence number
       int stage = 0, slot = 0;                          // operand stage, scale slot (q % P_SF_SLOTS)
       uint32_t phase = 0, acc_phase = 0;
-      const int64_t my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
-      const int64_t total = my_tiles * tile_stages;
+      int64_t total = 0;                                // stages over all tiles of this pair
+      for (int32_t t = pair; t < num_tiles; t += num_pairs) total += stages_of<MAXP>(grp.p[locate(grp, t).pi]);
       for (int32_t t = pair; t < num_tiles; t += num_pairs) {
+        const Params& p = grp.p[locate(grp, t).pi];
+        const int tile_stages = stages_of<MAXP>(p);
         for (int ks = 0; ks < tile_stages; ++ks, ++q) {
           if ((q & 1) == me) {
             if (ok && ks == 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag));
@@ -826,18 +871,25 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       int j = 0;
       uint32_t phase = 0;
       bool ok = true;
-      const int pf_n = min(P_PREFETCH, p.num_k_stages);
       for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
-        const TileCoord tc = pair_tile_coord(p, t);
+        const TileRef tr = locate(grp, t);
+        const Params& p = grp.p[tr.pi];
+        const PairMaps& M = grp.maps[tr.pi];
+        const int tile_stages = stages_of<MAXP>(p);
+        const int pf_n = min(P_PREFETCH, p.num_k_stages);
+        const TileCoord tc = pair_tile_coord(p, tr.lt);
         const bool has_next = t + num_pairs < num_tiles;
-        const TileCoord nc = pair_tile_coord(p, has_next ? t + num_pairs : t);
+        const TileRef nr = locate(grp, has_next ? t + num_pairs : t);
+        const Params& pn = grp.p[nr.pi];
+        const PairMaps& Mn = grp.maps[nr.pi];
+        const TileCoord nc = pair_tile_coord(pn, nr.lt);
         for (int ks = 0; ks < tile_stages; ++ks) {
           const int pf = ks - (p.num_k_stages - pf_n);
-          if (has_next && pf >= 0 && pf < pf_n) {  // the next tile's scales, as for the operands
+          if (has_next && pf >= 0 && pf < pf_n && pf < pn.num_k_stages) {   // the next tile's scales
             const int32_t pk = pf * (BK / MMA_K);
-            tma_prefetch_2d(&tma_sfa, 0, (int32_t)((nc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + pk);
-            tma_prefetch_2d(&tma_sfb, 0, (int32_t)((nc.n_blk * 2) * p.sf_kgroups) + pk);
-            tma_prefetch_2d(&tma_sfb, 0, (int32_t)((nc.n_blk * 2 + 1) * p.sf_kgroups) + pk);
+            tma_prefetch_2d(&Mn.sfa, 0, (int32_t)((nc.m_blk * 2 + (int32_t)rank) * pn.sf_kgroups_a) + pk);
+            tma_prefetch_2d(&Mn.sfb, 0, (int32_t)((nc.n_blk * 2) * pn.sf_kgroups) + pk);
+            tma_prefetch_2d(&Mn.sfb, 0, (int32_t)((nc.n_blk * 2 + 1) * pn.sf_kgroups) + pk);
           }
           if (!mbar_wait(sf_empty_bar(j), phase ^ 1u, abort_flag)) {
             ok = false;
@@ -856,10 +908,10 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           }
           mbar_arrive_expect_tx(sb, (uint32_t)P_SF_BYTES);
           const int32_t katom = ks * (BK / MMA_K);
-          tma_load_2d(sfa_smem(j), &tma_sfa, 0, (int32_t)((tc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + katom,
+          tma_load_2d(sfa_smem(j), &M.sfa, 0, (int32_t)((tc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + katom,
                       sb);
-          tma_load_2d(sfb_smem(j), &tma_sfb, 0, (int32_t)((tc.n_blk * 2) * p.sf_kgroups) + katom, sb);
-          tma_load_2d(sfb_smem(j) + (BK / MMA_K) * SF_ATOM, &tma_sfb, 0,
+          tma_load_2d(sfb_smem(j), &M.sfb, 0, (int32_t)((tc.n_blk * 2) * p.sf_kgroups) + katom, sb);
+          tma_load_2d(sfb_smem(j) + (BK / MMA_K) * SF_ATOM, &M.sfb, 0,
                       (int32_t)((tc.n_blk * 2 + 1) * p.sf_kgroups) + katom, sb);
           if (++j == P_SF_STAGES) {
             j = 0;
@@ -889,6 +941,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     int64_t q = 0;
     bool ok = true;
     for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
+      const int tile_stages = stages_of<MAXP>(grp.p[locate(grp, t).pi]);
       for (int ks = 0; ks < tile_stages; ++ks, ++q) {
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(sf_full_bar(j), sf_phase, abort_flag));
         if (!ok) break;
@@ -961,13 +1014,16 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     const int quarter = warp & 3;
     const int half = ew >> 2;
     const int row_in_tile = (int)rank * 128 + quarter * 32 + lane;
-    const float g = __fmul_rn(__fmul_rn(*p.scale_a, *p.scale_b), p.alpha);
     constexpr bool bf16_out = EPI == EPI_BF16 || EPI == EPI_BF16_ACC;
     constexpr bool accumulate = EPI == EPI_BF16_ACC || EPI == EPI_F32_ACC;
     uint8_t* stg = smem + P_EPI_OFFSET + ew * P_EPI_BOX_BYTES;
     uint32_t acc_phase = 0;
     for (int32_t t = pair; t < num_tiles; t += num_pairs) {
-      const TileCoord tc = pair_tile_coord(p, t);
+      const TileRef tr = locate(grp, t);
+      const Params& p = grp.p[tr.pi];
+      const CUtensorMap* tma_c = &grp.maps[tr.pi].c;
+      const float g = __fmul_rn(__fmul_rn(*p.scale_a, *p.scale_b), p.alpha);
+      const TileCoord tc = pair_tile_coord(p, tr.lt);
       const int n_cols = min(BN, p.N - tc.n_blk * BN);
       const int64_t m = (int64_t)tc.m_blk * P_BM + row_in_tile;
       const bool mine = n_cols > half * 128;          // N % 128 == 0: a half is whole or absent
@@ -1037,7 +1093,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tma_c, (int32_t)n0 + hh * P_EPI_BOX_COLS, m0, smem_u32(stg));
+            tma_store_2d(tma_c, (int32_t)n0 + hh * P_EPI_BOX_COLS, m0, smem_u32(stg));
             bulk_commit();
           }
           if (EPI == EPI_BF16 && p.amax_acc) box_amax(stg, lane, p.rht_signs, mraw, mrht);
@@ -1082,7 +1138,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tma_c, (int32_t)n0 + 32 * k, m0, smem_u32(stg));
+            tma_store_2d(tma_c, (int32_t)n0 + 32 * k, m0, smem_u32(stg));
             bulk_commit();
           }
         }

@@ -68,12 +68,15 @@ nvfp4_status device_info(DeviceInfo** out) {
     e = cudaFuncSetAttribute(nvfp4::gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              nvfp4::gemm::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-    for (auto kernel : {nvfp4::gemm::gemm_kernel_pair<nvfp4::gemm::EPI_BF16>,
-                        nvfp4::gemm::gemm_kernel_pair<nvfp4::gemm::EPI_BF16_ACC>,
-                        nvfp4::gemm::gemm_kernel_pair<nvfp4::gemm::EPI_F32>,
-                        nvfp4::gemm::gemm_kernel_pair<nvfp4::gemm::EPI_F32_ACC>}) {
-      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, nvfp4::gemm::P_SMEM_BYTES);
+    using namespace nvfp4::gemm;
+    for (auto kernel : {gemm_kernel_pair<EPI_BF16, 1>, gemm_kernel_pair<EPI_BF16_ACC, 1>, gemm_kernel_pair<EPI_F32, 1>,
+                        gemm_kernel_pair<EPI_F32_ACC, 1>}) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
+    }
+    for (auto kernel : {gemm_kernel_pair<EPI_BF16, kMaxGroup>, gemm_kernel_pair<EPI_F32, kMaxGroup>}) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(grouped gemm pair)");
     }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -87,7 +90,7 @@ nvfp4_status device_info(DeviceInfo** out) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, nvfp4::gemm::gemm_kernel_pair<nvfp4::gemm::EPI_BF16>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel_pair<EPI_BF16, 1>, &cfg);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
     d.pair_clusters = clusters;
     d.gemm_attr = true;
@@ -482,6 +485,42 @@ nvfp4_status make_lowrank_map(CUtensorMap* map, const void* X, int64_t rows, int
   return NVFP4_OK;
 }
 
+// Tensor maps and the per-problem fields of one CTA-pair GEMM problem (p holds the shape,
+// stage and scale fields filled by the caller): 256-element K-stages (128-byte code
+// boxes, four scale tiles per stage), 256-row tiles; the output store map unless the
+// epilogue accumulates in FP32 (which writes C directly).
+nvfp4_status pair_problem(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc, int32_t out_dtype,
+                          int32_t accumulate, nvfp4::gemm::Params* p, nvfp4::gemm::PairMaps* maps) {
+  nvfp4_status st;
+  if ((st = make_code_map(&maps->a, A, 128, nvfp4::gemm::BK_BYTES)) != NVFP4_OK) return st;
+  if ((st = make_code_map(&maps->b, B, 128, nvfp4::gemm::BK_BYTES)) != NVFP4_OK) return st;
+  if ((st = make_scale_map(&maps->sfa, A, nvfp4::gemm::BK / nvfp4::gemm::MMA_K)) != NVFP4_OK) return st;
+  if ((st = make_scale_map(&maps->sfb, B, nvfp4::gemm::BK / nvfp4::gemm::MMA_K)) != NVFP4_OK) return st;
+  const bool f32 = out_dtype == NVFP4_OUT_F32;
+  if (!(f32 && accumulate) && (st = make_out_map(&maps->c, C, A->rows, B->rows, ldc, f32)) != NVFP4_OK) return st;
+  p->num_m = (int32_t)ceil_div(A->rows, nvfp4::gemm::P_BM);
+  p->group_m = 16;
+  return NVFP4_OK;
+}
+
+// Launch configuration of the pair kernel: clusters of 2 CTAs, one pair per two SMs up to
+// the co-resident maximum, never more pairs than tiles.
+void pair_launch_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, int64_t tiles, int pair_clusters,
+                        cudaStream_t s) {
+  std::memset(cfg, 0, sizeof(*cfg));
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  const int pairs = (int)std::min<int64_t>(tiles, pair_clusters);
+  cfg->gridDim = dim3(2 * pairs, 1, 1);
+  cfg->blockDim = dim3(nvfp4::gemm::P_NUM_THREADS, 1, 1);
+  cfg->dynamicSmemBytes = nvfp4::gemm::P_SMEM_BYTES;
+  cfg->stream = s;
+  cfg->attrs = attr;
+  cfg->numAttrs = 1;
+}
+
 // nvfp4_gemm; with amax_out (3 floats) the maxima of nvfp4_gemm_amax; with a low-rank
 // pair the U V^T term of nvfp4_gemm_lowrank.
 nvfp4_status gemm_impl(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, int64_t ldc, int32_t out_dtype,
@@ -552,43 +591,25 @@ nvfp4_status gemm_impl(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, in
     return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the low-rank term needs M >= 256 and the CTA-pair GEMM");
   p.lr_ksteps = lr ? lr->rank / 16 : 0;
   if (M >= 256 && dev->pair_clusters > 0) {
-    // CTA pairs, 256 x 256 tiles
-    CUtensorMap map_a, map_b, map_sfa, map_sfb, map_c, map_u, map_v;
-    // 256-element K-stages: 128-byte code boxes, four scale tiles per stage
-    if ((st = make_code_map(&map_a, A, 128, nvfp4::gemm::BK_BYTES)) != NVFP4_OK) return st;
-    if ((st = make_code_map(&map_b, B, 128, nvfp4::gemm::BK_BYTES)) != NVFP4_OK) return st;
-    if ((st = make_scale_map(&map_sfa, A, nvfp4::gemm::BK / nvfp4::gemm::MMA_K)) != NVFP4_OK) return st;
-    if ((st = make_scale_map(&map_sfb, B, nvfp4::gemm::BK / nvfp4::gemm::MMA_K)) != NVFP4_OK) return st;
-    // the store map is read by every epilogue but the FP32 accumulating one
-    std::memset(&map_c, 0, sizeof(map_c));
-    const bool f32 = out_dtype == NVFP4_OUT_F32;
-    if (!(f32 && accumulate) && (st = make_out_map(&map_c, C, M, N, ldc, f32)) != NVFP4_OK) return st;
-    std::memset(&map_u, 0, sizeof(map_u));
-    std::memset(&map_v, 0, sizeof(map_v));
+    // CTA pairs, 256 x 256 tiles: a table of one problem
+    nvfp4::gemm::PairGroup<1> grp;
+    std::memset(&grp, 0, sizeof(grp));
+    if ((st = pair_problem(A, B, C, ldc, out_dtype, accumulate, &p, &grp.maps[0])) != NVFP4_OK) return st;
     if (lr) {
-      if ((st = make_lowrank_map(&map_u, lr->U, M, lr->ldu, lr->rank)) != NVFP4_OK) return st;
-      if ((st = make_lowrank_map(&map_v, lr->V, N, lr->ldv, lr->rank)) != NVFP4_OK) return st;
+      if ((st = make_lowrank_map(&grp.u, lr->U, M, lr->ldu, lr->rank)) != NVFP4_OK) return st;
+      if ((st = make_lowrank_map(&grp.v, lr->V, N, lr->ldv, lr->rank)) != NVFP4_OK) return st;
     }
-    p.num_m = (int32_t)ceil_div(M, nvfp4::gemm::P_BM);
-    p.group_m = 16;
-    const int64_t tiles = (int64_t)p.num_m * p.num_n;
-    const int pairs = (int)std::min<int64_t>(tiles, dev->pair_clusters);
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(nvfp4::gemm::P_NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = nvfp4::gemm::P_SMEM_BYTES;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    grp.p[0] = p;
+    grp.tile_end[0] = p.num_m * p.num_n;
+    grp.count = 1;
     using namespace nvfp4::gemm;
-    auto kernel = f32 ? (accumulate ? gemm_kernel_pair<EPI_F32_ACC> : gemm_kernel_pair<EPI_F32>)
-                      : (accumulate ? gemm_kernel_pair<EPI_BF16_ACC> : gemm_kernel_pair<EPI_BF16>);
-    e = cudaLaunchKernelEx(&cfg, kernel, map_a, map_b, map_sfa, map_sfb, map_c, map_u, map_v, p);
+    const bool f32 = out_dtype == NVFP4_OUT_F32;
+    auto kernel = f32 ? (accumulate ? gemm_kernel_pair<EPI_F32_ACC, 1> : gemm_kernel_pair<EPI_F32, 1>)
+                      : (accumulate ? gemm_kernel_pair<EPI_BF16_ACC, 1> : gemm_kernel_pair<EPI_BF16, 1>);
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    pair_launch_config(&cfg, attr, grp.tile_end[0], dev->pair_clusters, s);
+    e = cudaLaunchKernelEx(&cfg, kernel, grp);
   } else {
     CUtensorMap map_a, map_b;
     if ((st = make_code_map(&map_a, A, nvfp4::gemm::BM, nvfp4::gemm::BK_BYTES)) != NVFP4_OK) return st;
@@ -632,6 +653,76 @@ nvfp4_status nvfp4_gemm_lowrank(const nvfp4_tensor* A, const nvfp4_tensor* B, co
   lr.ldv = ldv;
   lr.rank = rank;
   return gemm_impl(A, B, C, ldc, NVFP4_OUT_BF16, 1.0f, 0, nullptr, 0u, stream, &lr);
+}
+
+nvfp4_status nvfp4_gemm_grouped(const nvfp4_tensor* const* A, const nvfp4_tensor* const* B, void* const* C,
+                                const int64_t* ldc, int32_t count, int32_t out_dtype, void* stream) {
+  if (!A || !B || !C || !ldc) return fail(NVFP4_ERR_INVALID_ARG, "NULL problem array");
+  if (count < 1 || count > nvfp4::gemm::kMaxGroup)
+    return fail(NVFP4_ERR_INVALID_ARG, "count %d outside 1 .. %d", count, nvfp4::gemm::kMaxGroup);
+  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return fail(NVFP4_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
+  nvfp4::gemm::PairGroup<nvfp4::gemm::kMaxGroup> grp;
+  std::memset(&grp, 0, sizeof(grp));
+  nvfp4_status st;
+  for (int i = 0; i < count; ++i) {
+    char an[16], bn[16];
+    std::snprintf(an, sizeof(an), "A[%d]", i);
+    std::snprintf(bn, sizeof(bn), "B[%d]", i);
+    if ((st = check_tensor(A[i], an)) != NVFP4_OK) return st;
+    if ((st = check_tensor(B[i], bn)) != NVFP4_OK) return st;
+    if (A[i]->cols != B[i]->cols) return fail(NVFP4_ERR_INVALID_ARG, "problem %d: A.cols != B.cols", i);
+    if (A[i]->scale_layout != NVFP4_SCALE_MMA || B[i]->scale_layout != NVFP4_SCALE_MMA)
+      return fail(NVFP4_ERR_INVALID_ARG, "problem %d: GEMM operands need the tensor-core scale layout", i);
+    const int64_t M = A[i]->rows, N = B[i]->rows, K = A[i]->cols;
+    if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 64)
+      return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "problem %d: needs M, N, K > 0, M %% 128, N %% 128, K %% 64 == 0", i);
+    if (M > (1ll << 31) - 128 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256)
+      return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "problem %d: extent above 2^31", i);
+    if (!C[i]) return fail(NVFP4_ERR_INVALID_ARG, "C[%d] is NULL", i);
+    if (ldc[i] < N) return fail(NVFP4_ERR_INVALID_ARG, "ldc[%d] < N", i);
+    if (!aligned16(C[i]) || (ldc[i] * (out_dtype == NVFP4_OUT_F32 ? 4 : 2)) % 16)
+      return fail(NVFP4_ERR_MISALIGNED, "C[%d] rows are not 16-byte aligned", i);
+    if (!aligned16(A[i]->scales) || !aligned16(B[i]->scales))
+      return fail(NVFP4_ERR_MISALIGNED, "problem %d: scales not 16-byte aligned", i);
+  }
+  DeviceInfo* dev;
+  if ((st = device_info(&dev)) != NVFP4_OK) return st;
+  if (dev->pair_clusters == 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the grouped GEMM needs the CTA-pair kernel");
+  int64_t tiles = 0;
+  for (int i = 0; i < count; ++i) {
+    nvfp4::gemm::Params& p = grp.p[i];
+    const int64_t M = A[i]->rows, N = B[i]->rows, K = A[i]->cols;
+    p.M = (int32_t)M;
+    p.N = (int32_t)N;
+    p.K = (int32_t)K;
+    p.num_n = (int32_t)ceil_div(N, nvfp4::gemm::BN);
+    p.num_k_stages = (int32_t)ceil_div(K, nvfp4::gemm::BK);
+    const int64_t tail = K % nvfp4::gemm::BK;
+    p.tail_atoms = tail ? (int32_t)(tail / nvfp4::gemm::MMA_K) : nvfp4::gemm::BK / nvfp4::gemm::MMA_K;
+    p.sfa = A[i]->scales;
+    p.sfb = B[i]->scales;
+    p.sf_kgroups = K / 64;
+    p.sf_kgroups_a = K / 64;
+    p.scale_a = A[i]->tensor_scale;
+    p.scale_b = B[i]->tensor_scale;
+    p.alpha = 1.0f;
+    p.C = C[i];
+    p.ldc = ldc[i];
+    p.out_f32 = out_dtype == NVFP4_OUT_F32;
+    p.skip_stage = i == 0 ? injected_gemm_skip_stage() : -1;
+    if ((st = pair_problem(A[i], B[i], C[i], ldc[i], out_dtype, 0, &p, &grp.maps[i])) != NVFP4_OK) return st;
+    tiles += (int64_t)p.num_m * p.num_n;
+    if (tiles > INT32_MAX) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "more than 2^31 tiles");
+    grp.tile_end[i] = (int32_t)tiles;
+  }
+  grp.count = count;
+  using namespace nvfp4::gemm;
+  auto kernel = out_dtype == NVFP4_OUT_F32 ? gemm_kernel_pair<EPI_F32, kMaxGroup> : gemm_kernel_pair<EPI_BF16, kMaxGroup>;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  pair_launch_config(&cfg, attr, tiles, dev->pair_clusters, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, grp);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "grouped gemm launch");
 }
 
 nvfp4_status nvfp4_linear_fwd(const void* X, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* Wq_row, void* Y,

@@ -173,3 +173,35 @@ def test_lora_linear_checks_its_branch_before_launching(lib):
     assert fwd(w=None) == 1
     assert lib.nvfp4_lora_linear_dgrad(y, 256, 256, 256, ctypes.byref(_tensor(384, 256)), l, r, 32, x, 384,
                                        ctypes.byref(_tensor(256, 256)), None, 1, 0, 0, None, ws, 256, None) == 1
+
+
+def test_grouped_lowrank_and_scaled_projection_argument_errors(lib):
+    """The grouped GEMM, the GEMM with a low-rank term and the scaled projection reject
+    bad arguments before any launch."""
+    T_P = ctypes.POINTER(_lib.NVFP4Tensor)
+    a, b = _tensor(256, 512), _tensor(384, 512)
+    arr_a = (T_P * 2)(ctypes.pointer(a), ctypes.pointer(a))
+    arr_b = (T_P * 2)(ctypes.pointer(b), ctypes.pointer(b))
+    arr_c = (ctypes.c_void_p * 2)(0x700000, 0x800000)
+    arr_ld = (ctypes.c_int64 * 2)(384, 384)
+    assert lib.nvfp4_gemm_grouped(arr_a, arr_b, arr_c, arr_ld, 0, 1, None) == 1          # count 0
+    assert lib.nvfp4_gemm_grouped(arr_a, arr_b, arr_c, arr_ld, 9, 1, None) == 1          # count above 8
+    assert lib.nvfp4_gemm_grouped(arr_a, arr_b, arr_c, arr_ld, 2, 7, None) == 1          # out_dtype
+    assert lib.nvfp4_gemm_grouped(None, arr_b, arr_c, arr_ld, 2, 1, None) == 1
+    bad_k = _tensor(384, 320)
+    arr_b2 = (T_P * 2)(ctypes.pointer(b), ctypes.pointer(bad_k))
+    assert lib.nvfp4_gemm_grouped(arr_a, arr_b2, arr_c, arr_ld, 2, 1, None) == 1         # A.cols != B.cols
+    arr_ld2 = (ctypes.c_int64 * 2)(384, 100)
+    assert lib.nvfp4_gemm_grouped(arr_a, arr_b, arr_c, arr_ld2, 2, 1, None) == 1         # ldc < N
+    arr_c2 = (ctypes.c_void_p * 2)(0x700000, 0x800008)
+    assert lib.nvfp4_gemm_grouped(arr_a, arr_b, arr_c2, arr_ld, 2, 1, None) == 3         # misaligned C
+    u, v = 0x900000, 0xA00000
+    assert lib.nvfp4_gemm_lowrank(ctypes.byref(a), ctypes.byref(b), u, 32, v, 32, 24, 0x700000, 384, None) == 2
+    assert lib.nvfp4_gemm_lowrank(ctypes.byref(a), ctypes.byref(b), None, 32, v, 32, 32, 0x700000, 384, None) == 1
+    assert lib.nvfp4_gemm_lowrank(ctypes.byref(a), ctypes.byref(b), u, 16, v, 32, 32, 0x700000, 384, None) == 1
+    assert lib.nvfp4_gemm_lowrank(ctypes.byref(a), ctypes.byref(b), u + 8, 32, v, 32, 32, 0x700000, 384, None) == 3
+    s = 0xB00000
+    assert lib.nvfp4_lowrank_project_scaled(0x100000, 128, 256, 256, 0x200000, 256, 0, 32, None, s, u, 32,
+                                            None) == 1
+    assert lib.nvfp4_lowrank_project_scaled(0x100000, 128, 256, 256, 0x200000, 256, 0, 24, s, s, u, 24,
+                                            None) == 2

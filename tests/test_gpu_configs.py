@@ -122,3 +122,43 @@ def test_square_gemm_sampled(i, n):
     check_gemm(c, ra_rows, rb_rows, a_hat, b_hat, "square %d^3" % n)
     del c, qa, qb
     torch.cuda.empty_cache()
+
+
+def test_layer3b_grouped_wgrad_matches_separate_launches():
+    """The four weight-gradient GEMMs of the 3B decoder layer at 32768 tokens (QKV, O,
+    gate-up, down) in one grouped launch give, tile for tile, the same FP32 outputs as
+    four separate launches (bit for bit: the same accumulation order in every tile), and
+    sampled rows of each agree with the oracle within the GEMM bound."""
+    import bench
+    from tests.test_gpu_fullsize import host_f32, layout_rows_1d, check_rows
+    names = list(synthetic.LAYER3B["linears"])
+    problems, singles, refs = [], [], []
+    for i, name in enumerate(names):
+        x, w, dy = synthetic.layer3b_linear(name, device="cuda")
+        _, xc = api.quantize(x, emit_row=False, emit_col=True, rht_col=True, rht_signs=bench.RHT_SIGNS)
+        _, dc = api.quantize(dy, emit_row=False, emit_col=True, stochastic=True, rht_col=True, seed=bench.SR_SEED,
+                             rht_signs=bench.RHT_SIGNS)
+        problems.append((dc, xc))
+        singles.append(api.gemm(dc, xc, out_dtype=torch.float32))
+        if name == "o":
+            refs.append((name, x, dy, dc, xc))
+        del x, w, dy
+    outs = api.gemm_grouped(problems, out_dtype=torch.float32)
+    api.get_status()
+    for name, a, b in zip(names, outs, singles):
+        assert torch.equal(a, b), name
+    # the O projection's dW rows against the oracle: dY^T X over 32768 tokens
+    name, x, dy, dc, xc = refs[0]
+    xh, dyh = host_f32(x), host_f32(dy)
+    n_rows, k_rows = sample_rows(dyh.shape[1], 700)[:8], sample_rows(xh.shape[1], 701)[:8]
+    S_dc = np.float32(dc.tensor_scale.cpu().item())
+    S_xc = np.float32(xc.tensor_scale.cpu().item())
+    c, s = layout_rows_1d(dyh, n_rows, S_dc, col=True, rht=True, stochastic=True, seed=bench.SR_SEED, offset=0,
+                          signs=bench.RHT_SIGNS)
+    a_hat = check_rows(dc, n_rows, c, s, S_dc, "dY col")
+    c, s = layout_rows_1d(xh, k_rows, S_xc, col=True, rht=True, stochastic=False, signs=bench.RHT_SIGNS)
+    b_hat = check_rows(xc, k_rows, c, s, S_xc, "X col")
+    got = outs[names.index("o")][torch.as_tensor(n_rows, device="cuda")][:, torch.as_tensor(k_rows, device="cuda")]
+    ref = O.gemm_ref(a_hat, b_hat)
+    ratio = np.abs(got.cpu().numpy().astype(np.float64) - ref) / O.gemm_tolerance(a_hat, b_hat)
+    assert ratio.max() <= 1.0, float(ratio.max())

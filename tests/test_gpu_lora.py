@@ -129,19 +129,21 @@ def test_gemm_lowrank_within_bound(m, n, k, rank):
     qb, _ = api.quantize(b)
     ra, rb = O.quantize(bf16_to_np(a))["row"], O.quantize(bf16_to_np(b))["row"]
     ah, bh = O.dequantize(*ra), O.dequantize(*rb)
+    g = np.float32(np.float32(ra[2]) * np.float32(rb[2]))
     rng = np.random.default_rng(rank)
-    uv = O.bf16_round(rng.standard_normal((m, rank)).astype(np.float32) * 50)
+    # U of magnitude 1/g, so that g U V^T is as large as the NVFP4 product
+    uv = O.bf16_round((rng.standard_normal((m, rank)) / float(g)).astype(np.float32))
     vv = O.bf16_round((0.3 * rng.standard_normal((n, rank))).astype(np.float32))
     c = api.gemm_lowrank(qa, qb, to_dev(uv), to_dev(vv))
     api.get_status()
-    g = np.float32(np.float32(ra[2]) * np.float32(rb[2]))
     ref = O.gemm_ref(ah, bh) + float(g) * O.gemm_ref(uv, vv)
     scale = O.gemm_abs_ref(ah, bh) + float(g) * O.gemm_abs_ref(uv, vv)
     bound = 1e-5 * scale + 1e-6 + 2.0 ** -8 * np.abs(ref)
     ratio = np.abs(bf16_to_np(c).astype(np.float64) - ref) / bound
     assert (ratio <= 1.0).all(), float(ratio.max())
-    # the low-rank term is really there: it moves the output by far more than the bound
-    assert np.abs(float(g) * O.gemm_ref(uv, vv)).max() > 100 * bound.max()
+    # the low-rank term is really there: the plain GEMM misses the reference by far
+    plain = bf16_to_np(api.gemm(qa, qb)).astype(np.float64)
+    assert (np.abs(plain - ref) / bound).max() > 100
 
 
 def spiked_weight(n, k, seed):
