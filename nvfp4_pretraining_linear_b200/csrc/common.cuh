@@ -135,21 +135,6 @@ __device__ __forceinline__ uint32_t e2m1x4_rs(float y0, float y1, float y2, floa
   return out;
 }
 
-// Two non-negative floats -> two E4M3 bytes (a in bits 0-7, b in bits 8-15), round to
-// nearest even, saturating at 448.
-__device__ __forceinline__ uint32_t e4m3x2_encode_hw(float a, float b) {
-  uint16_t out;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(b), "f"(a));
-  return out;
-}
-
-// max(a, b, c) in one instruction (sm_100 three-input minimum / maximum).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // Non-negative float -> E4M3 byte, round to nearest even, saturating at 448.
 __device__ __forceinline__ uint32_t e4m3_encode_hw(float v) {
   uint16_t out;
@@ -188,12 +173,6 @@ __device__ __forceinline__ uint4 philox4x32_10_rk(uint4 c, const uint32_t* rk) {
   return c;
 }
 
-// The four random words of Philox call `ctr` of a layout: word k drives the
-// four elements 16*ctr + 4k .. 16*ctr + 4k + 3.
-__device__ __forceinline__ uint4 philox_block(uint64_t ctr, uint32_t tag, uint32_t offset,
-                                              uint32_t k0, uint32_t k1) {
-  return philox4x32_10(make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), tag, offset), k0, k1);
-}
 
 // ----------------------------------------------------------------- Hadamard
 

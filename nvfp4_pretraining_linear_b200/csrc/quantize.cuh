@@ -17,23 +17,12 @@
 //              so that every quarter-warp hits distinct banks);
 //   col pass   thread t owns columns 2(t%64), 2(t%64)+1 and rows 32(t/64)..+31,
 //              reading one 32-bit word per row (a warp reads 128 contiguous
-//              bytes), so its column blocks are whole in registers; the two
-//              columns share each register pair, so the 16-point transform and
-//              the encode multiply run on both at once, in packed FP32.
+//              bytes), so its column blocks are whole in registers.
 // Both layouts come from one read of the tile.  Codes go straight to global
 // memory (row: 8 B per lane, 64 B per row segment; col: 16 B per column);
 // block scales are gathered with shuffles into 4-byte (row) or 2-byte (col)
-// stores in the tensor-core scale order.  The same kernel, in amax
-// mode, is the first pass (maximum of |x| and of the transformed blocks).
-//
-// Block scales.  The scale byte of a block is E4M3(fl(fl(b / 6) / S)) for its
-// maximum b.  For a fixed tensor scale S that map is monotone in b, so each CTA
-// tabulates, at start, the smallest b at which every byte value is reached (a
-// bisection over the float bit patterns, with the same two divisions); a block
-// then takes the E4M3 conversion of fl(b * fl(1 / fl(6 S))), which is within one
-// byte value of the exact one (a few float ulps apart, against E4M3 steps of at
-// least 1/16), and corrects it with two table lookups -- the exact byte, without
-// the divisions.
+// stores in the tensor-core scale order.  The same kernel, in amax mode, is the
+// first pass (maximum of |x| and of the transformed blocks).
 #pragma once
 
 #include <cuda.h>
@@ -50,8 +39,7 @@ constexpr int kQStages = 3;
 constexpr int kQComputeWarps = 8;
 constexpr int kQThreads = 32 * (kQComputeWarps + 1);  // 288
 constexpr int kQCtasPerSm = 2;
-constexpr int kQTableBytes = 4 * 128 * 4;            // encode multipliers and scale thresholds, row and col
-constexpr int kQSmemBytes = kQStages * kTileBytes + 256 + kQTableBytes + 128;   // tiles, barriers, tables
+constexpr int kQSmemBytes = kQStages * kTileBytes + 256 + 1024 + 128;   // tiles, barriers, scale tables
 
 struct QuantLayout {
   uint8_t* codes;       // nullptr when the layout is not emitted
@@ -69,7 +57,7 @@ struct QuantParams {
   const float* amax;    // quantise mode: 3 floats (raw, transformed col, transformed row)
   unsigned* amax_acc;   // amax mode: 3 accumulators (float bits)
   float* amax_out;      // nullptr or 3 floats
-  uint32_t rk[20];      // Philox round keys of the seed (philox4x32_10_rk)
+  uint32_t rk[20];      // Philox round keys of the seed (philox4x32_10_rk), in the kernel's parameter space
   uint32_t offset;      // Philox counter word 3
   uint32_t signs;       // RHT sign mask
   int64_t skip_tile;    // fault injection: the producer never loads this tile (-1: off)
@@ -160,125 +148,17 @@ __device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* m
       : "memory");
 }
 
-// Smallest non-negative finite b whose block scale E4M3(fl(fl(b / 6) / S)) is at
-// least k (1 <= k <= 126), or +inf if none is: bisection over the bit patterns of
-// non-negative floats, which order like the floats themselves.
-__device__ __forceinline__ float scale_threshold(uint32_t k, float S) {
-  uint32_t lo = 0u, hi = 0x7F800000u;          // byte(lo) < k; hi: first pattern known to reach k
-  while (hi - lo > 1u) {
-    const uint32_t mid = lo + ((hi - lo) >> 1);
-    if (e4m3_encode_hw(__fdiv_rn(__fdiv_rn(__uint_as_float(mid), 6.0f), S)) >= k) hi = mid;
-    else lo = mid;
-  }
-  return __uint_as_float(hi);                  // 0x7F800000 is +inf: k is never reached
-}
-
-// Per-tensor scale tables in shared memory: for each tensor scale S (row and col),
-// rtab[k] the encode multiplier of scale byte k and thr[k] the smallest block
-// maximum with scale byte >= k (thr[0] = 0, thr[127] = +inf).
-struct ScaleTables {
-  const float* rtab;
-  const float* thr;
-  float c;       // fl(1 / fl(6 S)): the approximate map b -> fl(b * c)
-  bool exact;    // c is not a positive finite float: divide instead
-  float S;
-};
-
-// Scale byte of a block with maximum b (see the comment at the top of this file).
-__device__ __forceinline__ uint32_t scale_byte(float b, const ScaleTables& t) {
-  if (t.exact) return e4m3_encode_hw(__fdiv_rn(__fdiv_rn(b, 6.0f), t.S));
-  uint32_t k = min(e4m3_encode_hw(__fmul_rn(b, t.c)), 126u);
-  return k - (uint32_t)(b < t.thr[k]) + (uint32_t)(b >= t.thr[k + 1]);
-}
-
-// The same for two blocks at once (one conversion instruction).
-__device__ __forceinline__ void scale_byte2(float b0, float b1, const ScaleTables& t, uint32_t& k0, uint32_t& k1) {
-  if (t.exact) {
-    k0 = e4m3_encode_hw(__fdiv_rn(__fdiv_rn(b0, 6.0f), t.S));
-    k1 = e4m3_encode_hw(__fdiv_rn(__fdiv_rn(b1, 6.0f), t.S));
-    return;
-  }
-  const uint32_t kk = e4m3x2_encode_hw(__fmul_rn(b0, t.c), __fmul_rn(b1, t.c));
-  const uint32_t a = min(kk & 0xFFu, 126u), b = min(kk >> 8, 126u);
-  k0 = a - (uint32_t)(b0 < t.thr[a]) + (uint32_t)(b0 >= t.thr[a + 1]);
-  k1 = b - (uint32_t)(b1 < t.thr[b]) + (uint32_t)(b1 >= t.thr[b + 1]);
-}
-
-__device__ __forceinline__ float absmax16_3(const float* v) {
-  float m = fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
-#pragma unroll
-  for (int j = 3; j < 15; j += 2) m = fmax3(m, fabsf(v[j]), fabsf(v[j + 1]));
-  return fmaxf(m, fabsf(v[15]));
-}
-
-// Column-pair helpers: element i of two neighbouring columns in one 64-bit register
-// pair (low word: the even column).
-__device__ __forceinline__ float f2_lo(uint64_t p) { return __uint_as_float((uint32_t)p); }
-__device__ __forceinline__ float f2_hi(uint64_t p) { return __uint_as_float((uint32_t)(p >> 32)); }
-
-// The 16-point transform's butterflies (stages 1, 2, 4, 8) and 1/4 normalisation,
-// along the 16 rows held in v[0..15], for both columns of the pair at once.
-__device__ __forceinline__ void wht16_pairs(uint64_t* v) {
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (!(i & h)) {
-        const uint64_t a = v[i], b = v[i + h];
-        v[i] = f2_add(a, b);
-        v[i + h] = f2_sub(a, b);
-      }
-    }
-  }
-  const uint64_t quarter = f2_pack(0.25f, 0.25f);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = f2_mul(v[i], quarter);
-}
-
-// max over the 16 rows of |v|, for the low (even) and high (odd) column of the pair.
-__device__ __forceinline__ void absmax_pairs(const uint64_t* v, float& m_lo, float& m_hi) {
-  m_lo = fmax3(fabsf(f2_lo(v[0])), fabsf(f2_lo(v[1])), fabsf(f2_lo(v[2])));
-  m_hi = fmax3(fabsf(f2_hi(v[0])), fabsf(f2_hi(v[1])), fabsf(f2_hi(v[2])));
-#pragma unroll
-  for (int i = 3; i < 15; i += 2) {
-    m_lo = fmax3(m_lo, fabsf(f2_lo(v[i])), fabsf(f2_lo(v[i + 1])));
-    m_hi = fmax3(m_hi, fabsf(f2_hi(v[i])), fabsf(f2_hi(v[i + 1])));
-  }
-  m_lo = fmaxf(m_lo, fabsf(f2_lo(v[15])));
-  m_hi = fmaxf(m_hi, fabsf(f2_hi(v[15])));
-}
-
-// Codes of one column of a pair (hi selects the odd column): y = v * r, then 16
-// E2M1 codes, row i in nibble i (round-to-nearest-even, or stochastic rounding with
-// the four random words w of the column block's Philox call).
-template <bool SR>
-__device__ __forceinline__ uint2 encode_column(const uint64_t* y, bool hi, const uint4& w) {
-  float e[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) e[i] = hi ? f2_hi(y[i]) : f2_lo(y[i]);
-  if (SR)
-    return make_uint2(e2m1x4_rs(e[0], e[1], e[2], e[3], w.x) | (e2m1x4_rs(e[4], e[5], e[6], e[7], w.y) << 16),
-                      e2m1x4_rs(e[8], e[9], e[10], e[11], w.z) | (e2m1x4_rs(e[12], e[13], e[14], e[15], w.w) << 16));
-  return make_uint2(e2m1x8_rn(e), e2m1x8_rn(e + 8));
-}
-
 // AMAX: first pass (maxima only).  Otherwise ER / EC emit the row / col layout,
 // SR stochastic rounding, RR / RC the transform on the row / col layout, TD
 // 16x16 blocks.
-// Two CTAs of 288 threads per SM leave 113 registers per thread; the register cap is
-// set explicitly (launch bounds alone let the compiler stop at 96 and spill).
-constexpr int kQMaxRegs = 112;
-static_assert(kQMaxRegs * kQThreads * kQCtasPerSm <= 65536, "two CTAs per SM must fit the register file");
-
 template <bool AMAX, bool ER, bool EC, bool SR, bool RR, bool RC, bool TD>
-__global__ void __maxnreg__(kQMaxRegs)
+__global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     quant_tile_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t bar_base = smem_base + kQStages * kTileBytes;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kQStages * kTileBytes + 8 * 2 * kQStages);
-  float* tables = reinterpret_cast<float*>(smem + kQStages * kTileBytes + 256);   // rtab row, rtab col, thr row, thr col
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (kQStages + s); };
 
@@ -345,29 +225,21 @@ __global__ void __maxnreg__(kQMaxRegs)
   const int cw = warp - 1;                 // 0..7
   const int ct = threadIdx.x - 32;         // 0..255
   const int64_t rows = p.rows, cols = p.cols;
-  ScaleTables trow{tables, tables + 256, 0.0f, true, 1.0f};
-  ScaleTables tcol{tables + 128, tables + 384, 0.0f, true, 1.0f};
+  float S_row = 1.0f, S_col = 1.0f;
   if (!AMAX) {
     const float amax_raw = p.amax[0];
     const float amax_col = RC ? p.amax[1] : amax_raw;
     const float amax_row = RR ? p.amax[2] : amax_raw;
-    trow.S = tensor_scale_from_amax(amax_row);
-    tcol.S = tensor_scale_from_amax(amax_col);
-    trow.c = __fdiv_rn(1.0f, __fmul_rn(6.0f, trow.S));
-    tcol.c = __fdiv_rn(1.0f, __fmul_rn(6.0f, tcol.S));
-    trow.exact = !(isfinite(trow.c) && trow.c > 0.0f);
-    tcol.exact = !(isfinite(tcol.c) && tcol.c > 0.0f);
-    // encode multipliers and thresholds of all E4M3 scale bytes for both tensor scales
-    {
-      const uint32_t k = (uint32_t)(ct & 127);
-      const float S = ct < 128 ? trow.S : tcol.S;
-      tables[ct] = scale_multiplier(k, S);
-      tables[256 + ct] = k == 0u ? 0.0f : (k == 127u ? __uint_as_float(0x7F800000u) : scale_threshold(k, S));
-    }
+    S_row = tensor_scale_from_amax(amax_row);
+    S_col = tensor_scale_from_amax(amax_col);
+    // encode multipliers of all E4M3 scale bytes for both tensor scales
+    float* tab = reinterpret_cast<float*>(smem + kQStages * kTileBytes + 256);
+    if (ct < 128) tab[ct] = scale_multiplier((uint32_t)ct, S_row);
+    else tab[ct] = scale_multiplier((uint32_t)(ct - 128), S_col);
     asm volatile("bar.sync 1, %0;" ::"r"(32 * kQComputeWarps) : "memory");
     if (blockIdx.x == 0 && ct == 0) {
-      if (ER) *p.row.tensor_scale = trow.S;
-      if (EC) *p.col.tensor_scale = tcol.S;
+      if (ER) *p.row.tensor_scale = S_row;
+      if (EC) *p.col.tensor_scale = S_col;
       if (p.amax_out) {
         p.amax_out[0] = amax_raw;
         p.amax_out[1] = RC ? amax_col : 0.0f;
@@ -375,6 +247,8 @@ __global__ void __maxnreg__(kQMaxRegs)
       }
     }
   }
+  const float* rtab_row = reinterpret_cast<const float*>(smem + kQStages * kTileBytes + 256);
+  const float* rtab_col = rtab_row + 128;
   float m_raw = 0.0f, m_col = 0.0f, m_row = 0.0f;
   const int64_t nblk_row = cols / 16, nblk_col = rows / 16;
   const int64_t rows_padded = (rows + 127) & ~int64_t(127);
@@ -404,13 +278,13 @@ __global__ void __maxnreg__(kQMaxRegs)
           float v[16];
           unpack8(*reinterpret_cast<const uint4*>(src + 16 * swap), v);
           unpack8(*reinterpret_cast<const uint4*>(src + 16 * (1 - swap)), v + 8);
-          tile_max = fmaxf(tile_max, absmax16_3(v));
+          tile_max = fmaxf(tile_max, absmax16(v));
         }
         tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 8));
         tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 16));
       }
-      uint32_t tile_sbyte = 0u;
-      if (TD && !AMAX) tile_sbyte = scale_byte(tile_max, trow);
+      BlockScale tbs;
+      if (TD && !AMAX) tbs = block_scale_tab(tile_max, S_row, rtab_row);
 #pragma unroll 2
       for (int it = 0; it < 4; ++it) {
         const int rl = cw * 16 + it * 4 + rsub;
@@ -430,9 +304,9 @@ __global__ void __maxnreg__(kQMaxRegs)
             v[2 * k + 1] = bf16_hi(w[k] ^ m);
           }
           if (AMAX) {
-            m_raw = fmaxf(m_raw, absmax16_3(v));   // the sign flips leave |x| unchanged
+            m_raw = fmaxf(m_raw, absmax16(v));   // the sign flips leave |x| unchanged
             wht16_scaled(v);
-            m_row = fmaxf(m_row, absmax16_3(v));
+            m_row = fmaxf(m_row, absmax16(v));
             continue;
           }
           wht16_scaled(v);
@@ -440,127 +314,117 @@ __global__ void __maxnreg__(kQMaxRegs)
           unpack8(h0, v);
           unpack8(h1, v + 8);
           if (AMAX) {
-            m_raw = fmaxf(m_raw, absmax16_3(v));
+            m_raw = fmaxf(m_raw, absmax16(v));
             continue;
           }
         }
-        const uint32_t sbyte = TD ? tile_sbyte : scale_byte(absmax16_3(v), trow);
-        const float rr = trow.rtab[sbyte];
+        const BlockScale bs = TD ? tbs : block_scale_tab(absmax16(v), S_row, rtab_row);
         uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (SR) w = philox4x32_10_rk(make_uint4((uint32_t)((uint64_t)(r * cols + c) >> 4),
-                                                (uint32_t)((uint64_t)(r * cols + c) >> 36), 0u, p.offset), p.rk);
+        if (SR) w = philox4x32_10_rk(make_uint4((uint32_t)((uint64_t)(r * cols + c) >> 4), (uint32_t)((uint64_t)(r * cols + c) >> 36), 0u, p.offset), p.rk);
         // v[0..7] holds the half read first; pick the matching random words
         const bool phys_swap = swap && !RR;
         const uint32_t wa0 = phys_swap ? w.z : w.x, wa1 = phys_swap ? w.w : w.y;
         const uint32_t wb0 = phys_swap ? w.x : w.z, wb1 = phys_swap ? w.y : w.w;
-        const uint32_t ca = encode8<SR>(v, rr, wa0, wa1);
-        const uint32_t cb = encode8<SR>(v + 8, rr, wb0, wb1);
+        const uint32_t ca = encode8<SR>(v, bs.r, wa0, wa1);
+        const uint32_t cb = encode8<SR>(v + 8, bs.r, wb0, wb1);
         uint32_t lo = phys_swap ? cb : ca, hi = phys_swap ? ca : cb;
-        if (rr == 0.0f) lo = hi = 0u;                       // dead block: all-zero codes
+        if (bs.r == 0.0f) lo = hi = 0u;                     // dead block: all-zero codes
         if (r < rows && c < cols) *reinterpret_cast<uint2*>(p.row.codes + r * (cols / 2) + c / 2) = make_uint2(lo, hi);
         if (p.row.mma_layout) {
           // blocks 4g .. 4g+3 of a row are 4 consecutive bytes: gather them on lanes b = 0 and 4
-          const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sbyte, 1);
-          const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sbyte, 2);
-          const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sbyte, 3);
+          const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 1);
+          const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 2);
+          const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 3);
           if ((b & 3) == 0) {
             const int64_t j = c / 16;
             if ((j >> 2) < p.row.kgroups && r < rows_padded)
               *reinterpret_cast<uint32_t*>(p.row.scales + mma_scale_offset(r, j, p.row.kgroups)) =
-                  sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24);
+                  bs.sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24);
           }
         } else if (r < rows && c < cols) {
-          p.row.scales[r * nblk_row + c / 16] = (uint8_t)sbyte;
+          p.row.scales[r * nblk_row + c / 16] = (uint8_t)bs.sbyte;
         }
       }
     }
 
     // ---------------------------------------------------------------- col pass
-    // thread ct: columns 2cp, 2cp + 1 (cp = ct % 64) and tile rows 32qr .. 32qr + 31
-    // (qr = ct / 64), two blocks per column; element i of both columns in one register
-    // pair v[i], so the transform and the encode multiply run on both columns at once.
     if ((AMAX && RC) || (!AMAX && EC)) {
-      const int cp = ct & 63, qr = ct >> 6;
-      uint64_t v[32];
+      const int cp = ct & 63, q = ct >> 6;
+      uint32_t codes[2][2][2];
+      uint32_t sb[2][2];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        uint32_t w = *reinterpret_cast<const uint32_t*>(in + (qr * 32 + i) * kTileRowBytes + cp * 4);
-        if (RC) w ^= pair_sign_mask(p.signs, i & 15);         // element i % 16 of its block
-        v[i] = f2_pack(bf16_lo(w), bf16_hi(w));
-      }
-      if (AMAX) {
-        float m0, m1, m2, m3;
-        absmax_pairs(v, m0, m1);                              // the sign flips leave |x| unchanged
-        absmax_pairs(v + 16, m2, m3);
-        m_raw = fmaxf(m_raw, fmax3(m0, m1, fmax3(m2, m3, 0.0f)));
-        wht16_pairs(v);
-        wht16_pairs(v + 16);
-        absmax_pairs(v, m0, m1);
-        absmax_pairs(v + 16, m2, m3);
-        m_col = fmaxf(m_col, fmax3(m0, m1, fmax3(m2, m3, 0.0f)));
-      } else {
+      for (int b = 0; b < 2; ++b) {
+        const int rl0 = q * 32 + b * 16;
+        float va[16], vb[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          uint32_t w = *reinterpret_cast<const uint32_t*>(in + (rl0 + i) * kTileRowBytes + cp * 4);
+          if (RC) w ^= pair_sign_mask(p.signs, i);        // element i of both column groups
+          va[i] = bf16_lo(w);
+          vb[i] = bf16_hi(w);
+        }
+        if (AMAX) m_raw = fmaxf(m_raw, fmaxf(absmax16(va), absmax16(vb)));   // signs leave |x| unchanged
         if (RC) {
-          wht16_pairs(v);
-          wht16_pairs(v + 16);
+          wht16_scaled(va);
+          wht16_scaled(vb);
         }
-        float mb[2][2];                                       // [block][column]
-        absmax_pairs(v, mb[0][0], mb[0][1]);
-        absmax_pairs(v + 16, mb[1][0], mb[1][1]);
+        if (AMAX) {
+          m_col = fmaxf(m_col, fmaxf(absmax16(va), absmax16(vb)));
+          continue;
+        }
+        float ma, mb;
         if (TD) {
-          // the 16x16 tile spans the 8 lanes holding columns 16 * (cp / 8) .. + 15
+          // the 16x16 tile spans the 8 lanes holding columns 16*(cp/8) .. +15
+          float m = fmaxf(absmax16(va), absmax16(vb));
+          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+          ma = mb = m;
+        } else {
+          ma = absmax16(va);
+          mb = absmax16(vb);
+        }
 #pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            float m = fmaxf(mb[b][0], mb[b][1]);
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
-            mb[b][0] = mb[b][1] = m;
+        for (int k = 0; k < 2; ++k) {
+          const float* v = k ? vb : va;
+          const BlockScale bs = block_scale_tab(k ? mb : ma, S_col, rtab_col);
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (SR) {
+            const int64_t c = c_base + 2 * cp + k;
+            const uint64_t ctr = (uint64_t)(c * rows + r_base + rl0) >> 4;
+            w = philox4x32_10_rk(make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), 1u, p.offset), p.rk);
           }
+          uint32_t lo = encode8<SR>(v, bs.r, w.x, w.y);
+          uint32_t hi = encode8<SR>(v + 8, bs.r, w.z, w.w);
+          if (bs.r == 0.0f) lo = hi = 0u;
+          codes[k][b][0] = lo;
+          codes[k][b][1] = hi;
+          sb[k][b] = bs.sbyte;
         }
-        uint32_t sb[2][2];
-        scale_byte2(mb[0][0], mb[0][1], tcol, sb[0][0], sb[0][1]);
-        scale_byte2(mb[1][0], mb[1][1], tcol, sb[1][0], sb[1][1]);
-        float rr[2][2];
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          rr[b][0] = tcol.rtab[sb[b][0]];
-          rr[b][1] = tcol.rtab[sb[b][1]];
-          const uint64_t rp = f2_pack(rr[b][0], rr[b][1]);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[16 * b + i] = f2_mul(v[16 * b + i], rp);
-        }
-        const int64_t rg = r_base + qr * 32;                  // first of this thread's 32 rows
+      }
+      if (!AMAX) {
+        const int64_t rg = r_base + q * 32;                  // first of this thread's 32 rows
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const int64_t c = c_base + 2 * cp + k;
-          uint2 code[2];
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            uint4 w = make_uint4(0u, 0u, 0u, 0u);
-            if (SR) {
-              const uint64_t ctr = (uint64_t)(c * rows + rg + 16 * b) >> 4;
-              w = philox4x32_10_rk(make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), 1u, p.offset), p.rk);
-            }
-            code[b] = encode_column<SR>(v + 16 * b, k != 0, w);
-            if (rr[b][k] == 0.0f) code[b] = make_uint2(0u, 0u);   // dead block: all-zero codes
-          }
           if (c >= cols || rg >= rows) continue;
           uint8_t* dst = p.col.codes + c * (rows / 2) + rg / 2;
           const bool both = rg + 16 < rows;
-          if (both && ((rows / 2) % 16) == 0) {
-            *reinterpret_cast<uint4*>(dst) = make_uint4(code[0].x, code[0].y, code[1].x, code[1].y);
+          if (((rows / 2) % 16) == 0 && both) {
+            *reinterpret_cast<uint4*>(dst) =
+                make_uint4(codes[k][0][0], codes[k][0][1], codes[k][1][0], codes[k][1][1]);
           } else {
-            *reinterpret_cast<uint2*>(dst) = code[0];
-            if (both) *reinterpret_cast<uint2*>(dst + 8) = code[1];
+            *reinterpret_cast<uint2*>(dst) = make_uint2(codes[k][0][0], codes[k][0][1]);
+            if (both) *reinterpret_cast<uint2*>(dst + 8) = make_uint2(codes[k][1][0], codes[k][1][1]);
           }
-          const int64_t j0 = rg / 16;                          // even: blocks j0, j0+1 are adjacent bytes
+          const int64_t j0 = rg / 16;                        // even: blocks j0, j0+1 are adjacent bytes
           if (p.col.mma_layout) {
             if ((j0 >> 2) < p.col.kgroups)
               *reinterpret_cast<uint16_t*>(p.col.scales + mma_scale_offset(c, j0, p.col.kgroups)) =
-                  (uint16_t)(sb[0][k] | (sb[1][k] << 8));
+                  (uint16_t)(sb[k][0] | (sb[k][1] << 8));
           } else {
-            p.col.scales[c * nblk_col + j0] = (uint8_t)sb[0][k];
-            if (both) p.col.scales[c * nblk_col + j0 + 1] = (uint8_t)sb[1][k];
+            p.col.scales[c * nblk_col + j0] = (uint8_t)sb[k][0];
+            if (both) p.col.scales[c * nblk_col + j0 + 1] = (uint8_t)sb[k][1];
           }
         }
       }
