@@ -662,12 +662,15 @@ __device__ __forceinline__ TileRef locate(const PairGroup<MAXP>& g, int32_t t) {
   return TileRef{pi, t - (pi ? g.tile_end[pi - 1] : 0)};
 }
 
-template <int MAXP>
+// Stages of a tile: the NVFP4 K-stages, then (LR) the low-rank stage.
+template <bool LR>
 __device__ __forceinline__ int stages_of(const Params& p) {
-  return p.num_k_stages + (p.lr_ksteps ? 1 : 0);
+  return LR ? p.num_k_stages + 1 : p.num_k_stages;
 }
 
-template <int EPI, int MAXP>
+// EPI: output mode; MAXP: problems per launch; LR: a low-rank stage ends every tile (a
+// separate instantiation, so that the plain GEMM carries none of its branches).
+template <int EPI, int MAXP, bool LR>
 __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     gemm_kernel_pair(const __grid_constant__ PairGroup<MAXP> grp) {
   extern __shared__ uint8_t smem_raw[];
@@ -729,8 +732,6 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
 
   const int32_t num_tiles = grp.tile_end[grp.count - 1];
   const int32_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
-  // Each tile's problem p (tensor maps M, parameters p); its stages: the NVFP4 K-stages,
-  // then the low-rank stage when there is one.
   const uint32_t leader_full0 = map_to_cta(full_bar(0), 0);
   const uint32_t leader_acc_empty = map_to_cta(acc_empty, 0);
 
@@ -748,7 +749,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
         const TileRef tr = locate(grp, t);
         const Params& p = grp.p[tr.pi];
         const PairMaps& M = grp.maps[tr.pi];
-        const int tile_stages = stages_of<MAXP>(p);
+        const int tile_stages = stages_of<LR>(p);
         const int pf_n = min(P_PREFETCH, p.num_k_stages);
         const TileCoord tc = pair_tile_coord(p, tr.lt);
         const bool has_next = t + num_pairs < num_tiles;
@@ -773,7 +774,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           }
           const uint32_t fb = leader_full0 + 8u * stage;
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * P_AB_BYTES);
-          if (ks == p.num_k_stages) {
+          if (LR && ks == p.num_k_stages) {
             // low-rank stage: 128 rows x 64 BF16 of U (this CTA's A rows) and of V (its half
             // of the B rows), zero-filled past the rank
             tma_load_2d_pair(a_smem(stage), &grp.u, 0, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
@@ -784,7 +785,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             tma_load_2d_pair(b_smem(stage), &M.b, kx, tc.n_blk * BN + (int32_t)rank * 128, fb);
           }
           const int pf = ks - (p.num_k_stages - pf_n);
-          if (has_next && pf >= 0 && pf < pf_n && pf < pn.num_k_stages) {
+          if (has_next && pf >= 0 && (!LR || pf < pf_n) && (MAXP == 1 || pf < pn.num_k_stages)) {
             tma_prefetch_2d(&Mn.a, pf * BK_BYTES, nc.m_blk * P_BM + (int32_t)rank * 128);
             tma_prefetch_2d(&Mn.b, pf * BK_BYTES, nc.n_blk * BN + (int32_t)rank * 128);
           }
@@ -814,10 +815,14 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
       int stage = 0, slot = 0;                          // operand stage, scale slot (q % P_SF_SLOTS)
       uint32_t phase = 0, acc_phase = 0;
       int64_t total = 0;                                // stages over all tiles of this pair
-      for (int32_t t = pair; t < num_tiles; t += num_pairs) total += stages_of<MAXP>(grp.p[locate(grp, t).pi]);
+      if constexpr (MAXP == 1) {
+        total = (int64_t)((num_tiles - pair + num_pairs - 1) / num_pairs) * stages_of<LR>(grp.p[0]);
+      } else {
+        for (int32_t t = pair; t < num_tiles; t += num_pairs) total += stages_of<LR>(grp.p[locate(grp, t).pi]);
+      }
       for (int32_t t = pair; t < num_tiles; t += num_pairs) {
         const Params& p = grp.p[locate(grp, t).pi];
-        const int tile_stages = stages_of<MAXP>(p);
+        const int tile_stages = stages_of<LR>(p);
         for (int ks = 0; ks < tile_stages; ++ks, ++q) {
           if ((q & 1) == me) {
             if (ok && ks == 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag));
@@ -826,7 +831,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             if (q > 0) asm volatile("bar.sync %0, 64;" ::"r"(me == 0 ? 2 : 1) : "memory");
             tc_fence_after();
             if (ok && lane == 0) {
-              if (ks == p.num_k_stages) {
+              if (LR && ks == p.num_k_stages) {
                 // low-rank stage: U V^T (BF16, K = 16 per MMA) into the same accumulator
                 for (int kk = 0; kk < p.lr_ksteps; ++kk)
                   tc_mma_pair_bf16(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * 32),
@@ -875,7 +880,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
         const TileRef tr = locate(grp, t);
         const Params& p = grp.p[tr.pi];
         const PairMaps& M = grp.maps[tr.pi];
-        const int tile_stages = stages_of<MAXP>(p);
+        const int tile_stages = stages_of<LR>(p);
         const int pf_n = min(P_PREFETCH, p.num_k_stages);
         const TileCoord tc = pair_tile_coord(p, tr.lt);
         const bool has_next = t + num_pairs < num_tiles;
@@ -885,7 +890,8 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
         const TileCoord nc = pair_tile_coord(pn, nr.lt);
         for (int ks = 0; ks < tile_stages; ++ks) {
           const int pf = ks - (p.num_k_stages - pf_n);
-          if (has_next && pf >= 0 && pf < pf_n && pf < pn.num_k_stages) {   // the next tile's scales
+          if (has_next && pf >= 0 && (!LR || pf < pf_n) && (MAXP == 1 || pf < pn.num_k_stages)) {
+            // the next tile's scales
             const int32_t pk = pf * (BK / MMA_K);
             tma_prefetch_2d(&Mn.sfa, 0, (int32_t)((nc.m_blk * 2 + (int32_t)rank) * pn.sf_kgroups_a) + pk);
             tma_prefetch_2d(&Mn.sfb, 0, (int32_t)((nc.n_blk * 2) * pn.sf_kgroups) + pk);
@@ -896,7 +902,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             break;
           }
           const uint32_t sb = sf_full_bar(j);
-          if (ks == p.num_k_stages) {
+          if (LR && ks == p.num_k_stages) {
             // the low-rank stage has no block scales: complete the slot's phase without
             // loading, so the writers' and issuers' stage counts stay in step
             mbar_arrive(sb);
@@ -941,7 +947,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     int64_t q = 0;
     bool ok = true;
     for (int32_t t = pair; t < num_tiles && ok; t += num_pairs) {
-      const int tile_stages = stages_of<MAXP>(grp.p[locate(grp, t).pi]);
+      const int tile_stages = stages_of<LR>(grp.p[locate(grp, t).pi]);
       for (int ks = 0; ks < tile_stages; ++ks, ++q) {
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(sf_full_bar(j), sf_phase, abort_flag));
         if (!ok) break;
@@ -1018,11 +1024,13 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
     constexpr bool accumulate = EPI == EPI_BF16_ACC || EPI == EPI_F32_ACC;
     uint8_t* stg = smem + P_EPI_OFFSET + ew * P_EPI_BOX_BYTES;
     uint32_t acc_phase = 0;
+    auto scale_of = [](const Params& q) { return __fmul_rn(__fmul_rn(*q.scale_a, *q.scale_b), q.alpha); };
+    const float g1 = MAXP == 1 ? scale_of(grp.p[0]) : 0.0f;   // one problem: read once
     for (int32_t t = pair; t < num_tiles; t += num_pairs) {
       const TileRef tr = locate(grp, t);
       const Params& p = grp.p[tr.pi];
       const CUtensorMap* tma_c = &grp.maps[tr.pi].c;
-      const float g = __fmul_rn(__fmul_rn(*p.scale_a, *p.scale_b), p.alpha);
+      const float g = MAXP == 1 ? g1 : scale_of(p);
       const TileCoord tc = pair_tile_coord(p, tr.lt);
       const int n_cols = min(BN, p.N - tc.n_blk * BN);
       const int64_t m = (int64_t)tc.m_blk * P_BM + row_in_tile;
@@ -1066,13 +1074,12 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             }
           } else {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              uint32_t r[64];
-              tc_load_32cols(taddr + 64 * hh, r);
-              tc_load_32cols(taddr + 64 * hh + 32, r + 32);
+            for (int k = 0; k < 4; ++k) {
+              uint32_t r[32];
+              tc_load_32cols(taddr + 32 * k, r);
               tc_wait_loads();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) pk[32 * hh + j] = scale_pack_bf16x2(r[2 * j], r[2 * j + 1], g);
+              for (int j = 0; j < 16; ++j) pk[16 * k + j] = scale_pack_bf16x2(r[2 * j], r[2 * j + 1], g);
             }
           }
         }

@@ -69,12 +69,13 @@ nvfp4_status device_info(DeviceInfo** out) {
                              nvfp4::gemm::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
     using namespace nvfp4::gemm;
-    for (auto kernel : {gemm_kernel_pair<EPI_BF16, 1>, gemm_kernel_pair<EPI_BF16_ACC, 1>, gemm_kernel_pair<EPI_F32, 1>,
-                        gemm_kernel_pair<EPI_F32_ACC, 1>}) {
+    for (auto kernel : {gemm_kernel_pair<EPI_BF16, 1, false>, gemm_kernel_pair<EPI_BF16_ACC, 1, false>,
+                        gemm_kernel_pair<EPI_F32, 1, false>, gemm_kernel_pair<EPI_F32_ACC, 1, false>,
+                        gemm_kernel_pair<EPI_BF16, 1, true>}) {
       e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
     }
-    for (auto kernel : {gemm_kernel_pair<EPI_BF16, kMaxGroup>, gemm_kernel_pair<EPI_F32, kMaxGroup>}) {
+    for (auto kernel : {gemm_kernel_pair<EPI_BF16, kMaxGroup, false>, gemm_kernel_pair<EPI_F32, kMaxGroup, false>}) {
       e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(grouped gemm pair)");
     }
@@ -90,7 +91,7 @@ nvfp4_status device_info(DeviceInfo** out) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel_pair<EPI_BF16, 1>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel_pair<EPI_BF16, 1, false>, &cfg);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
     d.pair_clusters = clusters;
     d.gemm_attr = true;
@@ -604,8 +605,10 @@ nvfp4_status gemm_impl(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, in
     grp.count = 1;
     using namespace nvfp4::gemm;
     const bool f32 = out_dtype == NVFP4_OUT_F32;
-    auto kernel = f32 ? (accumulate ? gemm_kernel_pair<EPI_F32_ACC, 1> : gemm_kernel_pair<EPI_F32, 1>)
-                      : (accumulate ? gemm_kernel_pair<EPI_BF16_ACC, 1> : gemm_kernel_pair<EPI_BF16, 1>);
+    // the low-rank stage is only taken with a plain BF16 output (nvfp4_gemm_lowrank)
+    auto kernel = lr ? gemm_kernel_pair<EPI_BF16, 1, true>
+                  : f32 ? (accumulate ? gemm_kernel_pair<EPI_F32_ACC, 1, false> : gemm_kernel_pair<EPI_F32, 1, false>)
+                        : (accumulate ? gemm_kernel_pair<EPI_BF16_ACC, 1, false> : gemm_kernel_pair<EPI_BF16, 1, false>);
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[1];
     pair_launch_config(&cfg, attr, grp.tile_end[0], dev->pair_clusters, s);
@@ -717,7 +720,8 @@ nvfp4_status nvfp4_gemm_grouped(const nvfp4_tensor* const* A, const nvfp4_tensor
   }
   grp.count = count;
   using namespace nvfp4::gemm;
-  auto kernel = out_dtype == NVFP4_OUT_F32 ? gemm_kernel_pair<EPI_F32, kMaxGroup> : gemm_kernel_pair<EPI_BF16, kMaxGroup>;
+  auto kernel = out_dtype == NVFP4_OUT_F32 ? gemm_kernel_pair<EPI_F32, kMaxGroup, false>
+                                                 : gemm_kernel_pair<EPI_BF16, kMaxGroup, false>;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   pair_launch_config(&cfg, attr, tiles, dev->pair_clusters, static_cast<cudaStream_t>(stream));
