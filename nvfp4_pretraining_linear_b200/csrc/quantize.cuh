@@ -70,25 +70,6 @@ __device__ __forceinline__ void unpack8(const uint4& w, float* v) {
   v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
 }
 
-// Row-block transform: this lane holds elements e = 8*(lane&1) + j of a 16-group
-// spread over a lane pair.  Stages h = 1, 2, 4 are local, stage 8 crosses the
-// pair, then the 1/4 normalisation -- the same operation order as rht16().
-__device__ __forceinline__ void rht16_pair(float* v, uint32_t signs, int lane) {
-  const uint32_t half = (uint32_t)(lane & 1) * 8u;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] = flip_sign(v[j], (signs >> (half + j)) & 1u);
-  wht_stage<8>(v, 1);
-  wht_stage<8>(v, 2);
-  wht_stage<8>(v, 4);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float other = __shfl_xor_sync(0xFFFFFFFFu, v[j], 1);
-    v[j] = (lane & 1) ? __fsub_rn(other, v[j]) : __fadd_rn(v[j], other);
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(v[j], 0.25f);
-}
-
 // Butterfly stages h = 1, 2, 4, 8 and the 1/4 normalisation over 16 values whose
 // signs were already applied (the transform of rht16 after its sign flips).
 // Stage 1 pairs neighbours, so it runs on scalars; after it, elements 2p and 2p+1
