@@ -788,12 +788,14 @@ def run_lora(args, dims, flush):
         "project_ms": timed(lambda: api.lowrank_project(x, r, out=u)),
         "project_scaled_ms": timed(lambda: api.lowrank_project_scaled(x, r, xr.tensor_scale, wq_row.tensor_scale,
                                                                       out=u)),
+        "project_dgrad_ms": timed(lambda: api.lowrank_project(dy, l, b_trans=True, out=u)),
         "gemm_plain_ms": timed(lambda: api.gemm(xr, wq_row, out=y)),
         "gemm_lowrank_ms": timed(lambda: api.gemm_lowrank(xr, wq_row, u, l, out=y)),
         "expand_ms": timed(lambda: api.lowrank_expand_add(y, u, l)),
     }
     api.get_status()
     res["project_gbs"] = (2.0 * M * K + 2.0 * M * rank) / res["project_ms"] / 1e6
+    res["project_dgrad_gbs"] = (2.0 * M * N + 2.0 * M * rank) / res["project_dgrad_ms"] / 1e6
     res["expand_gbs"] = 4.0 * M * N / res["expand_ms"] / 1e6
     res["residual_gbs"] = 4.0 * N * K / res["residual_ms"] / 1e6
     res["fwd_overhead"] = res["fwd_lora_ms"] / res["fwd_plain_ms"] - 1.0

@@ -296,7 +296,8 @@ nvfp4_status nvfp4_lora_residual(const void* W, int64_t N, int64_t K, int64_t ld
 /* U = BF16(A B^T): A [M x K] BF16 (row stride lda); B [r x K] (b_trans == 0, row
  * stride ldb) or given as its transpose [K x r] (b_trans != 0, row stride ldb);
  * U [M x r] BF16 (row stride ldu).  FP32 accumulation, one rounding to BF16.
- * Requires M % 64 == 0, K a positive multiple of 64, 16-byte aligned rows. */
+ * Requires M % 16 == 0, K a positive multiple of 64, 16-byte aligned rows.
+ * Enqueues one persistent kernel (one CTA per SM at most) on `stream`. */
 nvfp4_status nvfp4_lowrank_project(const void* A, int64_t M, int64_t K, int64_t lda, const void* B, int64_t ldb,
                                    int32_t b_trans, int32_t rank, void* U, int64_t ldu, void* stream);
 

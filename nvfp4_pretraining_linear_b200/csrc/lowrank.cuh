@@ -9,15 +9,17 @@
 //                          BF16 values is exact in FP32, so a fused multiply-add
 //                          rounds exactly as the separate product and sum would).
 //   lowrank_project_kernel U = BF16(A B^T), A [M x K] BF16, B [r x K] (or given as
-//                          [K x r]); HBM-bound on A.
+//                          [K x r]); HBM-bound on A: persistent, one CTA per SM,
+//                          each CTA a balanced run of 16-row units, A and B
+//                          streamed by TMA through a deep ring.
 //   lowrank_expand_kernel  Y = BF16(fl32(Y + U C^T)), U [M x r], C [N x r] (or given
 //                          as [r x N]); HBM-bound on the read-modify-write of Y,
 //                          persistent, with a ring of Y tiles in flight.
 //
 // The two products are dense contractions with a short side (r <= 64), so they run
 // on the warp-level BF16 tensor-core MMA (m16n8k16, FP32 accumulation) from shared
-// memory; the tiles are small and the work is bound by streaming A or Y, not by the
-// MMA rate.
+// memory; the work is bound by streaming A or Y, not by the MMA rate, and the 16-row
+// granularity of the warp-level MMA lets the projection split M evenly over the SMs.
 #pragma once
 
 #include <cstdint>
@@ -30,12 +32,22 @@ namespace lowrank {
 constexpr int kMaxRank = 64;
 constexpr int kResidualThreads = 256;
 constexpr int kResRows = 4;            // rows of W per residual thread
-constexpr int kProjRows = 64;          // rows of A per CTA (4 warps x 16)
-constexpr int kProjThreads = 128;
-constexpr int kProjKc = 64;            // K per pipeline stage
-constexpr int kProjStages = 4;
-constexpr int kPad = 72;               // shared row stride in BF16 elements (144 B, conflict-free)
-constexpr int kProjSmemBytes = kProjStages * (kProjRows + kMaxRank) * kPad * 2;
+constexpr int kProjUnit = 16;          // rows of A per work unit (one m16 MMA row block)
+constexpr int kProjUnits = 8;          // units a CTA holds at once, one consumer warp each
+constexpr int kProjThreads = 32 * (1 + kProjUnits);   // TMA producer warp + consumer warps
+constexpr int kProjKc = 64;            // K per TMA box (128 bytes of BF16: one swizzle row)
+constexpr int kProjBoxBytes = kProjUnit * 128;                        // 2 KB: one A box
+constexpr int kProjBBytes = 64 * 128;                                 // B box, at most 64 rows x 128 B
+constexpr int kProjBoxSets = 8;        // ring capacity in sets of (kProjUnits A boxes + one B box)
+constexpr int kProjSetBytes = kProjUnits * kProjBoxBytes + kProjBBytes;   // 24 KB
+constexpr int kProjBarOffset = kProjBoxSets * kProjSetBytes;          // 192 KB of ring
+constexpr int kProjSmemBytes = kProjBarOffset + 256 + 1024;           // ring, barriers, alignment slack
+// Boxes along K per unit and stage (H; each row is then read 128 * H contiguous bytes
+// per stage) and ring depth kProjBoxSets / H.  Measured at the 12B shapes: H = 4 (two
+// stages) for B given as [K x r] (the dgrad projection dY L, 671 MB of A), H = 2 (four
+// stages) for B as [r x K] (X R^T, 168 MB).
+template <bool BT>
+__host__ __device__ constexpr int proj_halves() { return BT ? 4 : 2; }
 constexpr int kExpTile = 128;          // Y tile 128 x 128
 constexpr int kExpThreads = 256;
 
@@ -116,107 +128,201 @@ __device__ __forceinline__ uint32_t pack_bf16_pair(const uint16_t* lo, const uin
   return (uint32_t)*lo | ((uint32_t)*hi << 16);
 }
 
-// RT = rank / 8 (n8 tiles).  CTA: 64 rows of A; warp w owns rows 16w..16w+15 and all
-// rank columns.  K streams through a kProjStages-deep cp.async ring of 64-column
-// chunks (dynamic shared memory, kProjSmemBytes), so about 24 KB of A is in flight per
-// CTA.  B is staged as given: [r x K] rows (BT false) give each MMA operand register
-// as one 32-bit load; [K x r] rows (BT true, e.g. L in dgrad) are staged unchanged and
-// each register is packed from two 16-bit loads.
+// Four 8x8 BF16 matrices from shared memory (lane l gives the address of row l % 8 of
+// matrix l / 8); .trans delivers each transposed.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// Shared address of 16-byte chunk `chunk` of row `row` in a box written by TMA with the
+// 128-byte swizzle (rows of 128 bytes, 1024-byte aligned box): the chunk index is
+// XORed with row % 8.
+__device__ __forceinline__ uint32_t sw128_addr(uint32_t box, int row, int chunk) {
+  return box + (uint32_t)(row * 128) + (uint32_t)(((chunk ^ row) & 7) << 4);
+}
+
+__device__ __forceinline__ void proj_tma_load(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                              uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// RT = rank / 8 (n8 tiles).  A persistent CTA owns the 16-row units [u0, u1) of A, an
+// even split of the M / 16 units over the grid, and takes them kProjUnits at a time:
+// warp 1 + j computes unit j of the group for all r columns while warp 0 streams the
+// group's K range through a ring of 64H-column chunks (H = proj_halves: per chunk H
+// 16 x 64 TMA boxes per unit, adjacent along K so that each row is read 128H bytes at
+// a time, and H boxes of B; 128-byte swizzle).  K need not be a multiple of 64H: the
+// boxes of a last partial chunk lie past K and TMA fills them with zeros.  Operand registers come
+// from ldmatrix: A and B given as [r x K] row-major, B given as [K x r] (BT, e.g. L in
+// dgrad) transposed on the way.  B boxes are 64 columns wide; with BT the columns past
+// r are zero-filled by TMA and never read.
 //
 // With scale_a and scale_b given, the sums are divided by g = fl32(*scale_a * *scale_b)
 // before the rounding: U' = BF16(fl32(fl32(sum) * fl32(1 / g))) -- the projection that
 // joins an NVFP4 GEMM's accumulator, which that GEMM multiplies by g.
 template <int RT, bool BT>
-__global__ void __launch_bounds__(kProjThreads) lowrank_project_kernel(const uint16_t* __restrict__ a, int64_t lda,
-                                                                       const uint16_t* __restrict__ b, int64_t ldb,
-                                                                       int64_t K, uint16_t* __restrict__ u,
-                                                                       int64_t ldu, const float* scale_a,
-                                                                       const float* scale_b) {
-  constexpr int R = RT * 8, RSn = R + 8;          // RSn: row stride of a staged [K x r] chunk
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  uint16_t (*As)[kProjRows][kPad] = reinterpret_cast<uint16_t (*)[kProjRows][kPad]>(smem_raw);
-  uint16_t (*Bs)[kMaxRank][kPad] =
-      reinterpret_cast<uint16_t (*)[kMaxRank][kPad]>(smem_raw + kProjStages * kProjRows * kPad * 2);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int64_t m0 = (int64_t)blockIdx.x * kProjRows;
-  const int chunks = (int)(K / kProjKc);
-
-  auto load = [&](int c, int buf) {
-    const int64_t k0 = (int64_t)c * kProjKc;
-#pragma unroll
-    for (int i = 0; i < (kProjRows * 8) / kProjThreads; ++i) {
-      const int idx = tid + i * kProjThreads, row = idx >> 3, ch = idx & 7;
-      cp_async16(&As[buf][row][ch * 8], a + (m0 + row) * lda + k0 + ch * 8);
-    }
-    if constexpr (!BT) {
-      for (int idx = tid; idx < R * 8; idx += kProjThreads) {
-        const int j = idx >> 3, ch = idx & 7;
-        cp_async16(&Bs[buf][j][ch * 8], b + (int64_t)j * ldb + k0 + ch * 8);
-      }
-    } else {
-      uint16_t* bn = &Bs[buf][0][0];                 // [kProjKc][RSn] within the same stage buffer
-      for (int idx = tid; idx < kProjKc * RT; idx += kProjThreads) {
-        const int kr = idx / RT, jc = idx - kr * RT;
-        cp_async16(bn + kr * RSn + jc * 8, b + (k0 + kr) * ldb + jc * 8);
-      }
-    }
+__global__ void __launch_bounds__(kProjThreads, 1)
+    lowrank_project_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                           int64_t units, int32_t chunks, uint16_t* __restrict__ u, int64_t ldu,
+                           const float* scale_a, const float* scale_b) {
+  constexpr int R = RT * 8;
+  constexpr uint32_t kBBoxBytes = BT ? (uint32_t)kProjBBytes : (uint32_t)(R * 128);
+  constexpr int kProjHalves = proj_halves<BT>();
+  constexpr int kProjStages = kProjBoxSets / kProjHalves;
+  constexpr int kProjStageBytes = kProjHalves * kProjSetBytes;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t base = smem_u32(smem);
+  const uint32_t bar_base = base + kProjBarOffset;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kProjBarOffset + 16 * kProjStages);
+  auto full_bar = [&](int st) { return bar_base + 8u * st; };
+  auto empty_bar = [&](int st) { return bar_base + 8u * (kProjStages + st); };
+  auto a_box = [&](int st, int h, int j) {
+    return base + (uint32_t)(st * kProjStageBytes + (h * kProjUnits + j) * kProjBoxBytes);
+  };
+  auto b_box = [&](int st, int h) {
+    return base + (uint32_t)(st * kProjStageBytes + kProjHalves * kProjUnits * kProjBoxBytes + h * kProjBBytes);
   };
 
-  float acc[RT][4];
-#pragma unroll
-  for (int nt = 0; nt < RT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-
-  // prologue: chunks 0 .. S-2, one commit group each (empty past the end)
-#pragma unroll
-  for (int c = 0; c < kProjStages - 1; ++c) {
-    if (c < chunks) load(c, c);
-    cp_async_commit();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kProjStages; ++st) {
+      mbar_init(full_bar(st), 1);
+      mbar_init(empty_bar(st), kProjUnits);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  for (int c = 0; c < chunks; ++c) {
-    cp_async_wait_pending<kProjStages - 2>();         // chunk c has landed (this thread's copies)
-    __syncthreads();                                  // ... everyone's; chunk c-1's buffer is free
-    const int nc = c + kProjStages - 1;
-    if (nc < chunks) load(nc, nc % kProjStages);
-    cp_async_commit();
-    const int buf = c % kProjStages;
-    const int r0 = warp * 16 + g;
-#pragma unroll
-    for (int kk = 0; kk < kProjKc / 16; ++kk) {
-      const int kc = kk * 16 + 2 * t;
-      uint32_t af[4];
-      af[0] = *reinterpret_cast<const uint32_t*>(&As[buf][r0][kc]);
-      af[1] = *reinterpret_cast<const uint32_t*>(&As[buf][r0 + 8][kc]);
-      af[2] = *reinterpret_cast<const uint32_t*>(&As[buf][r0][kc + 8]);
-      af[3] = *reinterpret_cast<const uint32_t*>(&As[buf][r0 + 8][kc + 8]);
-#pragma unroll
-      for (int nt = 0; nt < RT; ++nt) {
-        uint32_t bfr[2];
-        if constexpr (!BT) {
-          bfr[0] = *reinterpret_cast<const uint32_t*>(&Bs[buf][nt * 8 + g][kc]);
-          bfr[1] = *reinterpret_cast<const uint32_t*>(&Bs[buf][nt * 8 + g][kc + 8]);
-        } else {
-          const uint16_t* bn = &Bs[buf][0][0] + nt * 8 + g;
-          bfr[0] = pack_bf16_pair(bn + kc * RSn, bn + (kc + 1) * RSn);
-          bfr[1] = pack_bf16_pair(bn + (kc + 8) * RSn, bn + (kc + 9) * RSn);
+  __syncthreads();
+
+  const int64_t u0 = (int64_t)blockIdx.x * units / gridDim.x;
+  const int64_t u1 = (int64_t)(blockIdx.x + 1) * units / gridDim.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int st = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      bool issued[kProjStages] = {};
+      uint32_t issued_phase[kProjStages] = {};
+      for (int64_t g0 = u0; g0 < u1 && ok; g0 += kProjUnits) {
+        const int nu = (int)(u1 - g0 < kProjUnits ? u1 - g0 : kProjUnits);
+        for (int c = 0; c < chunks; ++c) {
+          if (!mbar_wait(empty_bar(st), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(st), (uint32_t)kProjHalves * ((uint32_t)(nu * kProjBoxBytes) + kBBoxBytes));
+          for (int j = 0; j < nu; ++j)
+            for (int h = 0; h < kProjHalves; ++h)
+              proj_tma_load(a_box(st, h, j), &amap, (c * kProjHalves + h) * kProjKc, (int32_t)((g0 + j) * kProjUnit),
+                            full_bar(st));
+          for (int h = 0; h < kProjHalves; ++h) {
+            if (BT)
+              proj_tma_load(b_box(st, h), &bmap, 0, (c * kProjHalves + h) * kProjKc, full_bar(st));
+            else
+              proj_tma_load(b_box(st, h), &bmap, (c * kProjHalves + h) * kProjKc, 0, full_bar(st));
+          }
+          issued[st] = true;
+          issued_phase[st] = phase;
+          if (++st == kProjStages) {
+            st = 0;
+            phase ^= 1u;
+          }
         }
-        mma_bf16_16816(acc[nt], af, bfr);
+      }
+      if (!ok) {
+        // wind down: let every load already issued land before the CTA exits
+        for (int k = 0; k < kProjStages; ++k) {
+          if (!issued[k]) continue;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(full_bar(k), issued_phase[k]) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
       }
     }
+    return;
   }
-  cp_async_wait_pending<0>();
-  const int64_t row = m0 + warp * 16 + g;
-  if (scale_a) {
-    const float inv = __fdiv_rn(1.0f, __fmul_rn(*scale_a, *scale_b));
+
+  // ------------------------------------------------------------ consumer warps
+  const int j = warp - 1;                        // unit of the group
+  const int g = lane >> 2, t = lane & 3;
+  float inv = 1.0f;
+  if (scale_a) inv = __fdiv_rn(1.0f, __fmul_rn(*scale_a, *scale_b));
+  // ldmatrix lane roles: A (16 x 16 per k-step): row lane % 16, k half lane / 16;
+  // B [r x K]: row 8 * (lane / 16) + lane % 8 of an n8 pair, k half (lane / 8) % 2;
+  // B [K x r] (transposed): k row lane % 16, n tile of the pair lane / 16.
+  const int a_row = lane & 15, a_half = lane >> 4;
+  const int b_row = (lane & 7) + ((lane >> 4) << 3), b_half = (lane >> 3) & 1;
+  int st = 0;
+  uint32_t phase = 0;
+  bool ok = true;
+  for (int64_t g0 = u0; g0 < u1 && ok; g0 += kProjUnits) {
+    const int nu = (int)(u1 - g0 < kProjUnits ? u1 - g0 : kProjUnits);
+    const bool active = j < nu;
+    float acc[RT][4];
 #pragma unroll
-    for (int nt = 0; nt < RT; ++nt)
+    for (int nt = 0; nt < RT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    for (int c = 0; c < chunks; ++c) {
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(full_bar(st), phase, abort_flag));
+      if (!ok) break;
+      if (active) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[nt][e] = __fmul_rn(acc[nt][e], inv);
-  }
+        for (int k16 = 0; k16 < kProjHalves * kProjKc / 16; ++k16) {
+          const int kk = k16 % (kProjKc / 16);
+          const uint32_t abox = a_box(st, k16 / (kProjKc / 16), j), bbox = b_box(st, k16 / (kProjKc / 16));
+          uint32_t af[4];
+          ldsm_x4(sw128_addr(abox, a_row, 2 * kk + a_half), af);
 #pragma unroll
-  for (int nt = 0; nt < RT; ++nt) {
-    const int col = nt * 8 + 2 * t;
-    *reinterpret_cast<uint32_t*>(u + row * ldu + col) = pack_bf16x2_rn(acc[nt][0], acc[nt][1]);
-    *reinterpret_cast<uint32_t*>(u + (row + 8) * ldu + col) = pack_bf16x2_rn(acc[nt][2], acc[nt][3]);
+          for (int np = 0; np < RT / 2; ++np) {
+            uint32_t bf[4];                      // b0, b1 of n tile 2np, then of 2np + 1
+            if constexpr (!BT) {
+              ldsm_x4(sw128_addr(bbox, 16 * np + b_row, 2 * kk + b_half), bf);
+            } else {
+              const int krow = 16 * kk + (lane & 15);
+              uint32_t tr[4];
+              ldsm_x4_trans(sw128_addr(bbox, krow, 2 * np + (lane >> 4)), tr);
+              bf[0] = tr[0], bf[1] = tr[1], bf[2] = tr[2], bf[3] = tr[3];
+            }
+            mma_bf16_16816(acc[2 * np], af, bf);
+            mma_bf16_16816(acc[2 * np + 1], af, bf + 2);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(st));
+      if (++st == kProjStages) {
+        st = 0;
+        phase ^= 1u;
+      }
+    }
+    if (!ok || !active) continue;
+    const int64_t row = (g0 + j) * kProjUnit + g;
+    if (scale_a) {
+#pragma unroll
+      for (int nt = 0; nt < RT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = __fmul_rn(acc[nt][e], inv);
+    }
+#pragma unroll
+    for (int nt = 0; nt < RT; ++nt) {
+      const int col = nt * 8 + 2 * t;
+      *reinterpret_cast<uint32_t*>(u + row * ldu + col) = pack_bf16x2_rn(acc[nt][0], acc[nt][1]);
+      *reinterpret_cast<uint32_t*>(u + (row + 8) * ldu + col) = pack_bf16x2_rn(acc[nt][2], acc[nt][3]);
+    }
   }
 }
 

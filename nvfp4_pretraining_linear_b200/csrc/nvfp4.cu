@@ -878,24 +878,43 @@ namespace {
 
 bool rank_ok(int32_t rank) { return rank >= 16 && rank <= nvfp4::lowrank::kMaxRank && rank % 16 == 0; }
 
+// Tensor map of a row-major BF16 matrix [outer x inner] (row stride ld elements) for
+// the projection: boxes of box_outer rows x 64 elements (128 bytes), 128-byte swizzle;
+// a box reaching past `inner` is zero-filled.
+nvfp4_status make_bf16_box_map(CUtensorMap* map, const void* X, int64_t inner, int64_t outer, int64_t ld,
+                               uint32_t box_outer) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  nvfp4_status st = get_encoder(&encode);
+  if (st != NVFP4_OK) return st;
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2u};
+  const cuuint32_t box[2] = {64u, box_outer};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled(projection operand) failed (%d)", (int)r);
+  return NVFP4_OK;
+}
+
 template <int RT, bool BT>
-cudaError_t launch_project(const uint16_t* a, int64_t lda, const uint16_t* b, int64_t ldb, int64_t M, int64_t K,
+cudaError_t launch_project(const CUtensorMap& am, const CUtensorMap& bm, int64_t units, int32_t chunks, int grid,
                            uint16_t* u, int64_t ldu, const float* sa, const float* sb, cudaStream_t s) {
   static bool done[kMaxDevices] = {};
   static std::mutex m;
   auto kernel = nvfp4::lowrank::lowrank_project_kernel<RT, BT>;
   cudaError_t e = ensure_smem(kernel, nvfp4::lowrank::kProjSmemBytes, done, m);
   if (e != cudaSuccess) return e;
-  kernel<<<(unsigned)(M / nvfp4::lowrank::kProjRows), nvfp4::lowrank::kProjThreads, nvfp4::lowrank::kProjSmemBytes,
-           s>>>(a, lda, b, ldb, K, u, ldu, sa, sb);
+  kernel<<<grid, nvfp4::lowrank::kProjThreads, nvfp4::lowrank::kProjSmemBytes, s>>>(am, bm, units, chunks, u, ldu, sa,
+                                                                                    sb);
   return cudaGetLastError();
 }
 
 template <int RT>
-cudaError_t dispatch_project(bool bt, const uint16_t* a, int64_t lda, const uint16_t* b, int64_t ldb, int64_t M,
-                             int64_t K, uint16_t* u, int64_t ldu, const float* sa, const float* sb, cudaStream_t s) {
-  return bt ? launch_project<RT, true>(a, lda, b, ldb, M, K, u, ldu, sa, sb, s)
-            : launch_project<RT, false>(a, lda, b, ldb, M, K, u, ldu, sa, sb, s);
+cudaError_t dispatch_project(bool bt, const CUtensorMap& am, const CUtensorMap& bm, int64_t units, int32_t chunks,
+                             int grid, uint16_t* u, int64_t ldu, const float* sa, const float* sb, cudaStream_t s) {
+  return bt ? launch_project<RT, true>(am, bm, units, chunks, grid, u, ldu, sa, sb, s)
+            : launch_project<RT, false>(am, bm, units, chunks, grid, u, ldu, sa, sb, s);
 }
 
 template <int KS, bool CT>
@@ -954,8 +973,9 @@ nvfp4_status lowrank_project_impl(const void* A, int64_t M, int64_t K, int64_t l
                                   int64_t ldu, void* stream) {
   if (!rank_ok(rank)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rank %d is not 16, 32, 48 or 64", rank);
   if (M < 0 || K < 0) return fail(NVFP4_ERR_INVALID_ARG, "negative extent");
-  if (M % nvfp4::lowrank::kProjRows || K % nvfp4::lowrank::kProjKc || K == 0)
-    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "projection needs M %% 64 == 0 and K a positive multiple of 64");
+  if (M % nvfp4::lowrank::kProjUnit || K % nvfp4::lowrank::kProjKc || K == 0)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "projection needs M %% 16 == 0 and K a positive multiple of 64");
+  if (K / nvfp4::lowrank::kProjKc > INT32_MAX) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K above 2^37");
   if (M == 0) return NVFP4_OK;
   if (!A || !B || !U) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
   if ((sa == nullptr) != (sb == nullptr)) return fail(NVFP4_ERR_INVALID_ARG, "give both tensor scales or neither");
@@ -963,17 +983,29 @@ nvfp4_status lowrank_project_impl(const void* A, int64_t M, int64_t K, int64_t l
     return fail(NVFP4_ERR_INVALID_ARG, "leading dimension too small");
   if (!aligned16(A) || !aligned16(B) || !aligned16(U) || lda % 8 || ldb % 8 || ldu % 8)
     return fail(NVFP4_ERR_MISALIGNED, "A, B and U rows must be 16-byte aligned");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const uint16_t* a = static_cast<const uint16_t*>(A);
-  const uint16_t* b = static_cast<const uint16_t*>(B);
-  uint16_t* u = static_cast<uint16_t*>(U);
+  DeviceInfo* dev;
+  nvfp4_status st = device_info(&dev);
+  if (st != NVFP4_OK) return st;
   const bool bt = b_trans != 0;
+  CUtensorMap am, bm;
+  if ((st = make_bf16_box_map(&am, A, K, M, lda, nvfp4::lowrank::kProjUnit)) != NVFP4_OK) return st;
+  // B as [r x K]: boxes of r rows x 64 K; B as [K x r]: boxes of 64 K-rows x 64 columns
+  if ((st = bt ? make_bf16_box_map(&bm, B, rank, K, ldb, (uint32_t)nvfp4::lowrank::kProjKc)
+               : make_bf16_box_map(&bm, B, K, rank, ldb, (uint32_t)rank)) != NVFP4_OK)
+    return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* u = static_cast<uint16_t*>(U);
+  const int64_t units = M / nvfp4::lowrank::kProjUnit;
+  const int64_t chunk_cols = (int64_t)nvfp4::lowrank::kProjKc *
+                             (bt ? nvfp4::lowrank::proj_halves<true>() : nvfp4::lowrank::proj_halves<false>());
+  const int32_t chunks = (int32_t)((K + chunk_cols - 1) / chunk_cols);   // a last half-chunk reads zeros past K
+  const int grid = (int)std::min<int64_t>(units, dev->sm_count);
   cudaError_t e;
   switch (rank / 8) {
-    case 2: e = dispatch_project<2>(bt, a, lda, b, ldb, M, K, u, ldu, sa, sb, s); break;
-    case 4: e = dispatch_project<4>(bt, a, lda, b, ldb, M, K, u, ldu, sa, sb, s); break;
-    case 6: e = dispatch_project<6>(bt, a, lda, b, ldb, M, K, u, ldu, sa, sb, s); break;
-    default: e = dispatch_project<8>(bt, a, lda, b, ldb, M, K, u, ldu, sa, sb, s); break;
+    case 2: e = dispatch_project<2>(bt, am, bm, units, chunks, grid, u, ldu, sa, sb, s); break;
+    case 4: e = dispatch_project<4>(bt, am, bm, units, chunks, grid, u, ldu, sa, sb, s); break;
+    case 6: e = dispatch_project<6>(bt, am, bm, units, chunks, grid, u, ldu, sa, sb, s); break;
+    default: e = dispatch_project<8>(bt, am, bm, units, chunks, grid, u, ldu, sa, sb, s); break;
   }
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "low-rank projection launch");
 }

@@ -136,7 +136,7 @@ def test_lowrank_argument_errors(lib):
     a, b, u, y = 0x100000, 0x200000, 0x300000, 0x400000
     assert lib.nvfp4_lowrank_project(a, 128, 256, 256, b, 256, 0, 24, u, 24, None) == 2       # rank not 16k
     assert lib.nvfp4_lowrank_project(a, 128, 256, 256, b, 256, 0, 80, u, 80, None) == 2       # rank above 64
-    assert lib.nvfp4_lowrank_project(a, 96, 256, 256, b, 256, 0, 32, u, 32, None) == 2        # M % 64
+    assert lib.nvfp4_lowrank_project(a, 104, 256, 256, b, 256, 0, 32, u, 32, None) == 2       # M % 16
     assert lib.nvfp4_lowrank_project(a, 128, 200, 200, b, 200, 0, 32, u, 32, None) == 2       # K % 64
     assert lib.nvfp4_lowrank_project(a, 128, 256, 256, b, 16, 1, 32, u, 32, None) == 1        # ldb < rank (transposed)
     assert lib.nvfp4_lowrank_project(a + 8, 128, 256, 256, b, 256, 0, 32, u, 32, None) == 3

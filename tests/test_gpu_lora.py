@@ -76,6 +76,20 @@ def test_project_within_bound(rank, b_trans):
     within(bf16_to_np(u), O.gemm_ref(av, bv), O.gemm_abs_ref(av, bv), "U")
 
 
+@pytest.mark.parametrize("m,k,rank", [(208, 320, 16), (208, 320, 48), (19200, 128, 32), (19200, 192, 64)])
+@pytest.mark.parametrize("b_trans", [False, True])
+def test_project_unit_split(m, k, rank, b_trans):
+    """The projection splits M into 16-row units over a persistent grid: 13 units (fewer
+    than the SMs, one or none per CTA) and 1200 units (more than eight per CTA on a
+    148-SM part, so CTAs take two groups in turn)."""
+    a = synthetic.normal((m, k), 1.0, seed=m + rank, device="cuda")
+    b = synthetic.normal((rank, k), 0.05, seed=k + rank, device="cuda")
+    av, bv = bf16_to_np(a), bf16_to_np(b)
+    arg = b.t().contiguous() if b_trans else b
+    u = api.lowrank_project(a, arg, b_trans=b_trans)
+    within(bf16_to_np(u), O.gemm_ref(av, bv), O.gemm_abs_ref(av, bv), "U")
+
+
 @pytest.mark.parametrize("rank", [16, 32, 48, 64])
 @pytest.mark.parametrize("c_trans", [False, True])
 def test_expand_add_within_bound(rank, c_trans):
