@@ -286,6 +286,16 @@ def cpu_cores():
         return os.cpu_count()
 
 
+def blas_threads():
+    """Threads of the BLAS library NumPy uses for the oracle's FP64 products (None if unknown)."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else None
+    except Exception:
+        return None
+
+
 def time_oracle(min_seconds=10.0, min_steps=3):
     state, flops, desc = oracle_sample_inputs()
     times = []
@@ -297,8 +307,8 @@ def time_oracle(min_seconds=10.0, min_steps=3):
         if len(times) >= 50:
             break
     t = statistics.median(times)
-    return {"value": flops / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-            "sample": desc + "; median of %d steps, %.2f s each" % (len(times), t)}
+    return {"value": flops / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "blas_threads": blas_threads(),
+            "kind": "oracle", "sample": desc + "; median of %d steps, %.2f s each" % (len(times), t)}
 
 
 def step_config(world):
@@ -326,7 +336,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantise / f64 GEMM",
             "data": "synthetic", "config": step_config(world),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "blas_threads": blas_threads(),
+                             "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
