@@ -20,8 +20,19 @@ SHAPES = [
     (384, 640, 320),      # N tail of 128 (half tile), K tail of 64
     (512, 384, 1024),
     (256, 1280, 768),     # several N tiles, K tail of 0
-    (1152, 512, 2112),    # more tiles than one wave per CTA? K tail 64
+    (1152, 512, 2112),    # 10 pair tiles (one wave), half-empty last row block, K tail of 64
 ]
+
+
+def random_shapes(n, seed):
+    """Seeded shapes over the GEMM's constraints (M, N multiples of 128, K of 64): one
+    or several pair tiles, half-empty row blocks (M % 256 == 128), N tails of 128 and
+    every K tail (K % 256 in {0, 64, 128, 192})."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        out.append((128 * int(rng.integers(1, 9)), 128 * int(rng.integers(1, 7)), 64 * int(rng.integers(1, 21))))
+    return out
 
 
 def operands(M, N, K, seed, kind="outliers"):
@@ -52,6 +63,17 @@ def test_gemm_f32_within_bound(M, N, K):
     torch.cuda.synchronize()
     ratio = gemm_check(c.cpu().numpy(), ah, bh)
     assert ratio <= 1.0, ratio
+
+
+@pytest.mark.parametrize("M,N,K", random_shapes(12, 2026))
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_random_shapes_within_bound(M, N, K, out_dtype):
+    a, b = operands(M, N, K, seed=3 * M + 5 * N + K, kind="t" if out_dtype == torch.bfloat16 else "outliers")
+    qa, qb, ah, bh = quantised_pair(a, b)
+    c = api.gemm(qa, qb, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    ratio = gemm_check(c.float().cpu().numpy(), ah, bh, bf16=out_dtype == torch.bfloat16)
+    assert ratio <= 1.0, (M, N, K, ratio)
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES[:4])
@@ -131,3 +153,27 @@ def test_gemm_accumulate_multiwave(out_dtype):
                        bf16=out_dtype == torch.bfloat16)
     assert ratio <= 1.0, ratio
     api.get_status()
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_grouped_mixed_shapes(out_dtype):
+    """One grouped launch over problems of different M, N and K (K tails, an N tail, a
+    half-empty row block, a single-row-block problem): every output within the bound of
+    the oracle, and equal bit for bit to a single launch of the same pair kernel where
+    that launch exists (M >= 256; a 128-row single GEMM takes the single-CTA kernel)."""
+    shapes = [(512, 384, 576), (384, 256, 1088), (256, 640, 64), (128, 256, 320), (768, 128, 832)]
+    problems, refs = [], []
+    for i, (M, N, K) in enumerate(shapes):
+        a, b = operands(M, N, K, seed=100 + i, kind="t" if i % 2 else "outliers")
+        qa, qb, ah, bh = quantised_pair(a, b)
+        problems.append((qa, qb))
+        refs.append((ah, bh))
+    outs = api.gemm_grouped(problems, out_dtype=out_dtype)
+    api.get_status()
+    bf16 = out_dtype == torch.bfloat16
+    for (M, N, K), (qa, qb), (ah, bh), c in zip(shapes, problems, refs, outs):
+        ratio = gemm_check(c.float().cpu().numpy(), ah, bh, bf16=bf16)
+        assert ratio <= 1.0, ((M, N, K), ratio)
+        if M >= 256:
+            single = api.gemm(qa, qb, out_dtype=out_dtype)
+            assert torch.equal(c, single), (M, N, K)
