@@ -698,7 +698,8 @@ def run_ns(args, dims, flush):
     """nvfp4_newton_schulz on a Gaussian [m x n] matrix: the whole call (normalisation and
     --iters steps, L2 flushed before each call) and, from the final iterate, each stage of
     one step timed alone: quantise X (row + col), the GEMM adding -X X^T into R, quantise
-    R (row), the GEMM adding R X / 2 into X."""
+    R (row), the GEMM adding R X / 2 into X; the two GEMMs also 20 launches back to back
+    without a flush, as they run inside the loop (their operands fit in L2)."""
     from nvfp4_pretraining_linear_b200 import api, synthetic as syn
     m, n = dims[:2]
     iters = args.iters
@@ -736,6 +737,21 @@ def run_ns(args, dims, flush):
     api.quantize(r, out_row=rr)
     t_qr = timed(lambda: api.quantize(r, out_row=rr))
     t_g2 = timed(lambda: api.gemm(rr, xc, alpha=0.5, accumulate=True, out=xs))
+
+    def back_to_back(fn, reps=20):
+        # as inside the iteration loop: launches queued back to back, operands warm in L2
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b) / reps
+
+    b_g1 = back_to_back(lambda: api.gemm(xr, xr, alpha=-1.0, accumulate=True, out=r))
+    b_g2 = back_to_back(lambda: api.gemm(rr, xc, alpha=0.5, accumulate=True, out=xs))
     api.get_status()
     step_flops = 4.0 * m * m * n
     print(json.dumps({
@@ -744,6 +760,8 @@ def run_ns(args, dims, flush):
         "stages_ms": {"quantize_x_row_col": t_qx, "gemm_x_xt": t_g1,
                       "quantize_r_row": t_qr, "gemm_r_x": t_g2},
         "gemm_tflops": {"x_xt": 2.0 * m * m * n / t_g1 / 1e9, "r_x": 2.0 * m * m * n / t_g2 / 1e9},
+        "gemm_back_to_back_ms": {"x_xt": b_g1, "r_x": b_g2},
+        "gemm_back_to_back_tflops": {"x_xt": 2.0 * m * m * n / b_g1 / 1e9, "r_x": 2.0 * m * m * n / b_g2 / 1e9},
         "quantize_gbs": {"x": m * n * 5.125 / t_qx / 1e6, "r": m * m * 4.5625 / t_qr / 1e6},
         "steps": args.steps, "l2": "flushed (256 MB write) before each timed call", "clocks": clock_info}),
         flush=True)
