@@ -152,6 +152,15 @@ __device__ __forceinline__ void tc_load_32cols(uint32_t taddr, uint32_t* r) {
 
 __device__ __forceinline__ void tc_wait_loads() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// One lane of the (fully active) warp, chosen by elect.sync.  Single-thread tcgen05
+// operations are issued under it with operands the whole warp computed, so that they
+// stay warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(e));
+  return e != 0;
+}
+
 // Scale 32 accumulator columns by g and store them (BF16 or FP32, optionally
 // adding the existing values) at crow (row-major C, 16-byte aligned).
 __device__ __forceinline__ void store_32cols(const Params& p, const uint32_t* r, float g, void* crow_v) {
@@ -314,7 +323,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop and computes the operands (warp-uniform); one
+    // elected lane issues the scale copies, the MMAs and the commits.
+    {
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -322,39 +333,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const TileCoord tc = tile_coord(p, t);
         const int nb_valid = min(2, (p.N - tc.n_blk * BN) / 128);
         const uint32_t idesc = make_idesc(nb_valid * 128);
-        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag))) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int ks = 0; ks < p.num_k_stages; ++ks) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag)) {
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(full_bar(stage), phase, abort_flag))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
-          for (int kk = 0; kk < atoms; ++kk) {
-            tc_copy_scales(tmem + SFA_COL + 4 * kk, sf_desc(sfa_smem(stage) + kk * SF_ATOM));
-            for (int nb = 0; nb < nb_valid; ++nb)
-              tc_copy_scales(tmem + SFB_COL + 8 * kk + 4 * nb,
-                             sf_desc(sfb_smem(stage) + (nb * (BK / MMA_K) + kk) * SF_ATOM));
-            tc_mma(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * (MMA_K / 2)),
-                   sw128_desc(b_smem(stage) + kk * (MMA_K / 2)), idesc, (ks | kk) != 0 ? 1u : 0u,
-                   tmem + SFA_COL + 4 * kk, tmem + SFB_COL + 8 * kk);
+          const uint64_t a_desc0 = sw128_desc(a_smem(stage)), b_desc0 = sw128_desc(b_smem(stage));
+          if (elect_one()) {
+            for (int kk = 0; kk < atoms; ++kk) {
+              tc_copy_scales(tmem + SFA_COL + 4 * kk, sf_desc(sfa_smem(stage) + kk * SF_ATOM));
+              for (int nb = 0; nb < nb_valid; ++nb)
+                tc_copy_scales(tmem + SFB_COL + 8 * kk + 4 * nb,
+                               sf_desc(sfb_smem(stage) + (nb * (BK / MMA_K) + kk) * SF_ATOM));
+              tc_mma(tmem + ACC_COL, a_desc0 + (uint64_t)(kk * (MMA_K / 2 / 16)),
+                     b_desc0 + (uint64_t)(kk * (MMA_K / 2 / 16)), idesc, (ks | kk) != 0 ? 1u : 0u,
+                     tmem + SFA_COL + 4 * kk, tmem + SFB_COL + 8 * kk);
+            }
+            tc_commit(empty_bar(stage));
           }
-          tc_commit(empty_bar(stage));
+          __syncwarp();
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        if (elect_one()) tc_commit(acc_full);
+        __syncwarp();
         acc_phase ^= 1u;
       }
-      // every MMA issued by this thread has finished once mma_done flips
-      tc_commit(mma_done);
+      // every MMA issued by the elected lanes has finished once mma_done flips
+      if (elect_one()) tc_commit(mma_done);
+      __syncwarp();
       mbar_wait_drain(mma_done, 0);
     }
   } else {
@@ -830,19 +847,23 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(sf_ready_bar(stage), phase, abort_flag));
             if (q > 0) asm volatile("bar.sync %0, 64;" ::"r"(me == 0 ? 2 : 1) : "memory");
             tc_fence_after();
-            if (ok && lane == 0) {
+            // Operands of this stage's MMAs, computed by every lane so that they stay
+            // warp-uniform; one lane chosen by elect.sync issues.  (Computing them under a
+            // lane == 0 branch instead cost 5 % of the GEMM's throughput.)
+            const uint64_t a_desc0 = sw128_desc(a_smem(stage)), b_desc0 = sw128_desc(b_smem(stage));
+            const uint32_t sfa0 = tmem + P_SF_COL0 + P_SF_SLOT_COLS * slot;
+            const int atoms_u = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
+            if (ok && elect_one()) {
               if (LR && ks == p.num_k_stages) {
                 // low-rank stage: U V^T (BF16, K = 16 per MMA) into the same accumulator
                 for (int kk = 0; kk < p.lr_ksteps; ++kk)
                   tc_mma_pair_bf16(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * 32),
                                    sw128_desc(b_smem(stage) + kk * 32), make_idesc_pair_bf16());
               } else {
-                const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
-                const uint32_t sfa = tmem + P_SF_COL0 + P_SF_SLOT_COLS * slot, sfb = sfa + 16;
-                for (int kk = 0; kk < atoms; ++kk)
-                  tc_mma_pair(tmem + ACC_COL, sw128_desc(a_smem(stage) + kk * (MMA_K / 2)),
-                              sw128_desc(b_smem(stage) + kk * (MMA_K / 2)), idesc, (ks | kk) != 0 ? 1u : 0u,
-                              sfa + 4 * kk, sfb + 8 * kk);
+                for (int kk = 0; kk < atoms_u; ++kk)
+                  tc_mma_pair(tmem + ACC_COL, a_desc0 + (uint64_t)(kk * (MMA_K / 2 / 16)),
+                              b_desc0 + (uint64_t)(kk * (MMA_K / 2 / 16)), idesc, (ks | kk) != 0 ? 1u : 0u,
+                              sfa0 + 4 * kk, sfa0 + 16 + 8 * kk);
               }
               tc_commit_pair(empty_bar(stage));
               if (ks == tile_stages - 1) tc_commit_pair(acc_full);
