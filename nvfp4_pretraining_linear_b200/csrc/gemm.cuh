@@ -280,7 +280,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane arms the barrier and issues the copies.
+    {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_phase[STAGES];
@@ -291,22 +292,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const TileCoord tc = tile_coord(p, t);
         const int nb_valid = min(2, (p.N - tc.n_blk * BN) / 128);
         for (int ks = 0; ks < p.num_k_stages; ++ks) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag))) {
             ok = false;
             break;
           }
           const int atoms = (ks == p.num_k_stages - 1) ? p.tail_atoms : BK / MMA_K;
           const uint32_t sf_bytes = (uint32_t)atoms * SF_ATOM;
-          mbar_arrive_expect_tx(full_bar(stage), (uint32_t)(A_BYTES + B_BYTES) + sf_bytes * (1u + nb_valid));
-          tma_load_2d(a_smem(stage), &tma_a, ks * BK_BYTES, tc.m_blk * BM, full_bar(stage));
-          tma_load_2d(b_smem(stage), &tma_b, ks * BK_BYTES, tc.n_blk * BN, full_bar(stage));
           const int64_t kg = (int64_t)ks * (BK / MMA_K);
-          bulk_load(sfa_smem(stage), p.sfa + ((int64_t)tc.m_blk * p.sf_kgroups + kg) * SF_ATOM, sf_bytes,
-                    full_bar(stage));
-          for (int nb = 0; nb < nb_valid; ++nb)
-            bulk_load(sfb_smem(stage) + nb * (BK / MMA_K) * SF_ATOM,
-                      p.sfb + ((int64_t)(tc.n_blk * 2 + nb) * p.sf_kgroups + kg) * SF_ATOM, sf_bytes,
+          if (elect_one()) {
+            mbar_arrive_expect_tx(full_bar(stage), (uint32_t)(A_BYTES + B_BYTES) + sf_bytes * (1u + nb_valid));
+            tma_load_2d(a_smem(stage), &tma_a, ks * BK_BYTES, tc.m_blk * BM, full_bar(stage));
+            tma_load_2d(b_smem(stage), &tma_b, ks * BK_BYTES, tc.n_blk * BN, full_bar(stage));
+            bulk_load(sfa_smem(stage), p.sfa + ((int64_t)tc.m_blk * p.sf_kgroups + kg) * SF_ATOM, sf_bytes,
                       full_bar(stage));
+            for (int nb = 0; nb < nb_valid; ++nb)
+              bulk_load(sfb_smem(stage) + nb * (BK / MMA_K) * SF_ATOM,
+                        p.sfb + ((int64_t)(tc.n_blk * 2 + nb) * p.sf_kgroups + kg) * SF_ATOM, sf_bytes,
+                        full_bar(stage));
+          }
+          __syncwarp();
           issued[stage] = true;
           issued_phase[stage] = phase;
           if (++stage == STAGES) {
@@ -754,7 +758,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ operand producer (both CTAs)
-    if (lane == 0) {
+    {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -775,7 +779,7 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
         const PairMaps& Mn = grp.maps[nr.pi];
         const TileCoord nc = pair_tile_coord(pn, nr.lt);
         for (int ks = 0; ks < tile_stages; ++ks, ++q) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag))) {
             ok = false;
             break;
           }
@@ -790,22 +794,25 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
             continue;
           }
           const uint32_t fb = leader_full0 + 8u * stage;
-          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * P_AB_BYTES);
-          if (LR && ks == p.num_k_stages) {
-            // low-rank stage: 128 rows x 64 BF16 of U (this CTA's A rows) and of V (its half
-            // of the B rows), zero-filled past the rank
-            tma_load_2d_pair(a_smem(stage), &grp.u, 0, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
-            tma_load_2d_pair(b_smem(stage), &grp.v, 0, tc.n_blk * BN + (int32_t)rank * 128, fb);
-          } else {
-            const int32_t kx = ks * BK_BYTES;
-            tma_load_2d_pair(a_smem(stage), &M.a, kx, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
-            tma_load_2d_pair(b_smem(stage), &M.b, kx, tc.n_blk * BN + (int32_t)rank * 128, fb);
-          }
+          const int32_t kx = ks * BK_BYTES;
           const int pf = ks - (p.num_k_stages - pf_n);
-          if (has_next && pf >= 0 && (!LR || pf < pf_n) && (MAXP == 1 || pf < pn.num_k_stages)) {
-            tma_prefetch_2d(&Mn.a, pf * BK_BYTES, nc.m_blk * P_BM + (int32_t)rank * 128);
-            tma_prefetch_2d(&Mn.b, pf * BK_BYTES, nc.n_blk * BN + (int32_t)rank * 128);
+          if (elect_one()) {
+            if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * P_AB_BYTES);
+            if (LR && ks == p.num_k_stages) {
+              // low-rank stage: 128 rows x 64 BF16 of U (this CTA's A rows) and of V (its half
+              // of the B rows), zero-filled past the rank
+              tma_load_2d_pair(a_smem(stage), &grp.u, 0, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
+              tma_load_2d_pair(b_smem(stage), &grp.v, 0, tc.n_blk * BN + (int32_t)rank * 128, fb);
+            } else {
+              tma_load_2d_pair(a_smem(stage), &M.a, kx, tc.m_blk * P_BM + (int32_t)rank * 128, fb);
+              tma_load_2d_pair(b_smem(stage), &M.b, kx, tc.n_blk * BN + (int32_t)rank * 128, fb);
+            }
+            if (has_next && pf >= 0 && (!LR || pf < pf_n) && (MAXP == 1 || pf < pn.num_k_stages)) {
+              tma_prefetch_2d(&Mn.a, pf * BK_BYTES, nc.m_blk * P_BM + (int32_t)rank * 128);
+              tma_prefetch_2d(&Mn.b, pf * BK_BYTES, nc.n_blk * BN + (int32_t)rank * 128);
+            }
           }
+          __syncwarp();
           if (++stage == P_STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -880,20 +887,21 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
         }
         acc_phase ^= 1u;
       }
-      // every MMA this warp issued has finished once mma_done flips (one barrier per issuer)
-      if (lane == 0) {
-        const uint32_t done = me == 0 ? mma_done : mma_done2;
+      // every MMA this warp issued has finished once mma_done flips (one barrier per
+      // issuer; the commit comes from the lane that issued them)
+      const uint32_t done = me == 0 ? mma_done : mma_done2;
+      if (elect_one())
         asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(done)
                      : "memory");
-        mbar_wait_drain(done, 0);
-      }
+      __syncwarp();
+      mbar_wait_drain(done, 0);
     }
   } else if (warp == P_SF_PRODUCER) {
     // ------------------------------------------------------------ scale producer (both CTAs)
     // Each CTA loads the scales of its own A rows and of all 256 B rows of the tile,
     // up to P_SF_STAGES stages ahead; a slot is reused once the four writers of this
     // CTA have stored it to tensor memory.
-    if (lane == 0) {
+    {
       int j = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -911,14 +919,15 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
         const TileCoord nc = pair_tile_coord(pn, nr.lt);
         for (int ks = 0; ks < tile_stages; ++ks) {
           const int pf = ks - (p.num_k_stages - pf_n);
-          if (has_next && pf >= 0 && (!LR || pf < pf_n) && (MAXP == 1 || pf < pn.num_k_stages)) {
+          if (has_next && pf >= 0 && (!LR || pf < pf_n) && (MAXP == 1 || pf < pn.num_k_stages) && elect_one()) {
             // the next tile's scales
             const int32_t pk = pf * (BK / MMA_K);
             tma_prefetch_2d(&Mn.sfa, 0, (int32_t)((nc.m_blk * 2 + (int32_t)rank) * pn.sf_kgroups_a) + pk);
             tma_prefetch_2d(&Mn.sfb, 0, (int32_t)((nc.n_blk * 2) * pn.sf_kgroups) + pk);
             tma_prefetch_2d(&Mn.sfb, 0, (int32_t)((nc.n_blk * 2 + 1) * pn.sf_kgroups) + pk);
           }
-          if (!mbar_wait(sf_empty_bar(j), phase ^ 1u, abort_flag)) {
+          __syncwarp();
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(sf_empty_bar(j), phase ^ 1u, abort_flag))) {
             ok = false;
             break;
           }
@@ -926,20 +935,24 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
           if (LR && ks == p.num_k_stages) {
             // the low-rank stage has no block scales: complete the slot's phase without
             // loading, so the writers' and issuers' stage counts stay in step
-            mbar_arrive(sb);
+            if (elect_one()) mbar_arrive(sb);
+            __syncwarp();
             if (++j == P_SF_STAGES) {
               j = 0;
               phase ^= 1u;
             }
             continue;
           }
-          mbar_arrive_expect_tx(sb, (uint32_t)P_SF_BYTES);
           const int32_t katom = ks * (BK / MMA_K);
-          tma_load_2d(sfa_smem(j), &M.sfa, 0, (int32_t)((tc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + katom,
-                      sb);
-          tma_load_2d(sfb_smem(j), &M.sfb, 0, (int32_t)((tc.n_blk * 2) * p.sf_kgroups) + katom, sb);
-          tma_load_2d(sfb_smem(j) + (BK / MMA_K) * SF_ATOM, &M.sfb, 0,
-                      (int32_t)((tc.n_blk * 2 + 1) * p.sf_kgroups) + katom, sb);
+          if (elect_one()) {
+            mbar_arrive_expect_tx(sb, (uint32_t)P_SF_BYTES);
+            tma_load_2d(sfa_smem(j), &M.sfa, 0, (int32_t)((tc.m_blk * 2 + (int32_t)rank) * p.sf_kgroups_a) + katom,
+                        sb);
+            tma_load_2d(sfb_smem(j), &M.sfb, 0, (int32_t)((tc.n_blk * 2) * p.sf_kgroups) + katom, sb);
+            tma_load_2d(sfb_smem(j) + (BK / MMA_K) * SF_ATOM, &M.sfb, 0,
+                        (int32_t)((tc.n_blk * 2 + 1) * p.sf_kgroups) + katom, sb);
+          }
+          __syncwarp();
           if (++j == P_SF_STAGES) {
             j = 0;
             phase ^= 1u;
