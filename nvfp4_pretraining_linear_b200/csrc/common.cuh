@@ -318,6 +318,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One lane of the (fully active) warp, chosen by elect.sync (the same lane every time
+// the whole warp calls it).  Single-thread operations -- tcgen05 MMAs, copies and
+// commits, TMA copies, barrier arming -- are issued under it with operands the whole
+// warp computed, so that they stay warp-uniform; issuing them under lane == 0 with
+// operands computed inside the branch measured 5-8 % slower in the GEMM.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(e));
+  return e != 0;
+}
+
 // Wait until the phase with the given parity of mbarrier `bar` has completed.
 // Gives up after kWaitLimitNs, or as soon as *abort is set by another role of
 // the CTA: records kErrTimeout, raises *abort and returns false.

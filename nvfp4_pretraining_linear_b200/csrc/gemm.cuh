@@ -152,14 +152,6 @@ __device__ __forceinline__ void tc_load_32cols(uint32_t taddr, uint32_t* r) {
 
 __device__ __forceinline__ void tc_wait_loads() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// One lane of the (fully active) warp, chosen by elect.sync.  Single-thread tcgen05
-// operations are issued under it with operands the whole warp computed, so that they
-// stay warp-uniform.
-__device__ __forceinline__ bool elect_one() {
-  uint32_t e;
-  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(e));
-  return e != 0;
-}
 
 // Scale 32 accumulator columns by g and store them (BF16 or FP32, optionally
 // adding the existing values) at crow (row-major C, 16-byte aligned).

@@ -212,7 +212,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane arms the barrier and issues the copies.
+    {
       int st = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -221,21 +222,25 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       for (int64_t g0 = u0; g0 < u1 && ok; g0 += kProjUnits) {
         const int nu = (int)(u1 - g0 < kProjUnits ? u1 - g0 : kProjUnits);
         for (int c = 0; c < chunks; ++c) {
-          if (!mbar_wait(empty_bar(st), phase ^ 1u, abort_flag)) {
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(st), phase ^ 1u, abort_flag))) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(st), (uint32_t)kProjHalves * ((uint32_t)(nu * kProjBoxBytes) + kBBoxBytes));
-          for (int j = 0; j < nu; ++j)
-            for (int h = 0; h < kProjHalves; ++h)
-              proj_tma_load(a_box(st, h, j), &amap, (c * kProjHalves + h) * kProjKc, (int32_t)((g0 + j) * kProjUnit),
-                            full_bar(st));
-          for (int h = 0; h < kProjHalves; ++h) {
-            if (BT)
-              proj_tma_load(b_box(st, h), &bmap, 0, (c * kProjHalves + h) * kProjKc, full_bar(st));
-            else
-              proj_tma_load(b_box(st, h), &bmap, (c * kProjHalves + h) * kProjKc, 0, full_bar(st));
+          if (elect_one()) {
+            mbar_arrive_expect_tx(full_bar(st),
+                                  (uint32_t)kProjHalves * ((uint32_t)(nu * kProjBoxBytes) + kBBoxBytes));
+            for (int j = 0; j < nu; ++j)
+              for (int h = 0; h < kProjHalves; ++h)
+                proj_tma_load(a_box(st, h, j), &amap, (c * kProjHalves + h) * kProjKc,
+                              (int32_t)((g0 + j) * kProjUnit), full_bar(st));
+            for (int h = 0; h < kProjHalves; ++h) {
+              if (BT)
+                proj_tma_load(b_box(st, h), &bmap, 0, (c * kProjHalves + h) * kProjKc, full_bar(st));
+              else
+                proj_tma_load(b_box(st, h), &bmap, (c * kProjHalves + h) * kProjKc, 0, full_bar(st));
+            }
           }
+          __syncwarp();
           issued[st] = true;
           issued_phase[st] = phase;
           if (++st == kProjStages) {

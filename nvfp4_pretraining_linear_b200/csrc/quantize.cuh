@@ -157,14 +157,15 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane arms the barrier and issues the copy.
+    {
       int stage = 0;
       uint32_t phase = 0;
       bool issued[kQStages] = {};
       uint32_t issued_phase[kQStages] = {};
       bool ok = true;
       for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x) {
-        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag))) {
           ok = false;
           break;
         }
@@ -179,9 +180,12 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
           }
           continue;
         }
-        mbar_arrive_expect_tx(full_bar(stage), kTileBytes);
-        tma_load_tile(smem_base + stage * kTileBytes, &xmap, (int32_t)(tc * kTileCols), (int32_t)(tr * kTileRows),
-                      full_bar(stage));
+        if (elect_one()) {
+          mbar_arrive_expect_tx(full_bar(stage), kTileBytes);
+          tma_load_tile(smem_base + stage * kTileBytes, &xmap, (int32_t)(tc * kTileCols), (int32_t)(tr * kTileRows),
+                        full_bar(stage));
+        }
+        __syncwarp();
         issued[stage] = true;
         issued_phase[stage] = phase;
         if (++stage == kQStages) {
