@@ -591,7 +591,13 @@ nvfp4_status gemm_impl(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, in
   if (lr && (M < 256 || dev->pair_clusters == 0))
     return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the low-rank term needs M >= 256 and the CTA-pair GEMM");
   p.lr_ksteps = lr ? lr->rank / 16 : 0;
-  if (M >= 256 && dev->pair_clusters > 0) {
+  // CTA pairs unless M = 128 leaves more 256-column tiles than pairs: a 128-row problem
+  // runs on the pair kernel with half of each pair tile empty, which is faster only
+  // while every tile gets a pair of SMs (one wave); past that the single-CTA kernel's
+  // 128 x 256 tiles fill the SMs in fewer waves.
+  const bool use_pair = dev->pair_clusters > 0 &&
+                        (M >= 256 || amax_out || ceil_div(N, nvfp4::gemm::BN) <= (int64_t)dev->pair_clusters);
+  if (use_pair) {
     // CTA pairs, 256 x 256 tiles: a table of one problem
     nvfp4::gemm::PairGroup<1> grp;
     std::memset(&grp, 0, sizeof(grp));

@@ -21,6 +21,7 @@ SHAPES = [
     (512, 384, 1024),
     (256, 1280, 768),     # several N tiles, K tail of 0
     (1152, 512, 2112),    # 10 pair tiles (one wave), half-empty last row block, K tail of 64
+    (128, 20480, 320),    # 128 rows and more 256-column tiles than CTA pairs: the single-CTA kernel
 ]
 
 
