@@ -6,17 +6,20 @@
 // accumulator is FP32 in tensor memory and the global scales are applied once,
 // in the epilogue.
 //
-// Two kernels.  gemm_kernel_pair (further below) serves M >= 256: CTA pairs
-// (cta_group::2) on 256 x 256 output tiles, block scales stored into tensor memory
-// by writer warps, two MMA-issuing warps, BF16 output through TMA stores.
-// gemm_kernel serves M = 128 and devices that cannot co-schedule a pair:
+// Two kernels.  gemm_kernel_pair (further below) serves M >= 256, and M = 128 while
+// its tiles fit one wave of pairs: CTA pairs (cta_group::2) on 256 x 256 output
+// tiles, block scales stored into tensor memory by writer warps, two MMA-issuing
+// warps, output through TMA stores.  gemm_kernel serves the other 128-row problems
+// and devices that cannot co-schedule a pair.  In both, a role warp runs its loop as
+// a whole warp and issues single-thread operations (TMA copies, barrier arming,
+// MMAs, commits) from one elected lane with warp-uniform operands.
 //
 // Structure (one CTA per SM, persistent over output tiles of 128 x 256):
 //   warp 0      TMA producer: per K-stage of 256 elements, one tiled TMA load of
 //               A (128 rows x 128 bytes) and of B (256 x 128 bytes), 128-byte
 //               swizzled, plus bulk copies of the matching block-scale tiles
 //               (already in the tensor-core order, 512 bytes per 128 rows x 64 K).
-//   warp 1      MMA issuer (one thread): copies each stage's scales into tensor
+//   warp 1      MMA issuer (one elected lane): copies each stage's scales into tensor
 //               memory (tcgen05.cp) and issues four tcgen05.mma kind::mxf4nvf4
 //               block16 (M=128, N=256, K=64) into an FP32 accumulator in tensor
 //               memory; tcgen05.commit frees the stage and, after the last one,
@@ -437,9 +440,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 //
 // Block scales reach tensor memory through tcgen05.st from four scale-writer warps
 // per CTA (one per 32-lane quarter), not through tcgen05.cp from the MMA thread:
-// copies issued between the MMAs stretch each M256N256K64 MMA from 128 to about
-// 275 cycles on random operands, while stores from other warps leave the MMA
-// stream at 128.  Each operand stage has its own scale slot in tensor memory (48
+// measured with copies and MMAs issued from a lane == 0 branch, copies between the
+// MMAs stretched each M256N256K64 MMA from 128 to about 275 cycles on random
+// operands, while stores from other warps left the MMA stream at 128.  Each operand stage has its own scale slot in tensor memory (48
 // columns: 16 of A scales, 32 of B scales), freed with the stage.  The layout
 // written is the one a 32x128b.warpx4 copy of the 512-byte scale tile gives:
 // every quarter holds the same 32 lanes x 4 columns per tile.  The scales stream
@@ -497,10 +500,6 @@ __device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
 
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // Arrival that only hands over tensor-memory accesses: the arriving warp has waited
