@@ -270,10 +270,20 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
       }
       BlockScale tbs;
       if (TD && !AMAX) tbs = block_scale_tab(tile_max, S_row, rtab_row);
+      // This lane's row advances by 4 per step: its Philox counter ((r * cols + c) / 16,
+      // exact since cols and c are multiples of 16), its code address and the tile part
+      // of its scale offset are set up once per tile and advanced by additions.
+      const int64_t r0 = r_base + cw * 16 + rsub;
+      const uint64_t ctr0 = (uint64_t)r0 * (uint64_t)(cols >> 4) + (uint64_t)(c >> 4);
+      const uint64_t ctr_step = (uint64_t)(cols >> 4) * 4u;
+      uint8_t* const code0 = p.row.codes + r0 * (cols / 2) + c / 2;
+      const int64_t code_step = 4 * (cols / 2);
+      const int64_t j = c / 16;
+      const int64_t sc_tile = (((r_base >> 7) * p.row.kgroups + (j >> 2)) << 9) + (j & 3);
 #pragma unroll 2
       for (int it = 0; it < 4; ++it) {
         const int rl = cw * 16 + it * 4 + rsub;
-        const int64_t r = r_base + rl;
+        const int64_t r = r0 + 4 * it;
         const uint8_t* src = in + rl * kTileRowBytes + b * 32;
         uint4 h0 = *reinterpret_cast<const uint4*>(src + 16 * swap);
         uint4 h1 = *reinterpret_cast<const uint4*>(src + 16 * (1 - swap));
@@ -305,7 +315,10 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
         }
         const BlockScale bs = TD ? tbs : block_scale_tab(absmax16(v), S_row, rtab_row);
         uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (SR) w = philox4x32_10_rk(make_uint4((uint32_t)((uint64_t)(r * cols + c) >> 4), (uint32_t)((uint64_t)(r * cols + c) >> 36), 0u, p.offset), p.rk);
+        if (SR) {
+          const uint64_t ctr = ctr0 + (uint64_t)it * ctr_step;
+          w = philox4x32_10_rk(make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), 0u, p.offset), p.rk);
+        }
         // v[0..7] holds the half read first; pick the matching random words
         const bool phys_swap = swap && !RR;
         const uint32_t wa0 = phys_swap ? w.z : w.x, wa1 = phys_swap ? w.w : w.y;
@@ -314,16 +327,16 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
         const uint32_t cb = encode8<SR>(v + 8, bs.r, wb0, wb1);
         uint32_t lo = phys_swap ? cb : ca, hi = phys_swap ? ca : cb;
         if (bs.r == 0.0f) lo = hi = 0u;                     // dead block: all-zero codes
-        if (r < rows && c < cols) *reinterpret_cast<uint2*>(p.row.codes + r * (cols / 2) + c / 2) = make_uint2(lo, hi);
+        if (r < rows && c < cols) *reinterpret_cast<uint2*>(code0 + it * code_step) = make_uint2(lo, hi);
         if (p.row.mma_layout) {
           // blocks 4g .. 4g+3 of a row are 4 consecutive bytes: gather them on lanes b = 0 and 4
           const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 1);
           const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 2);
           const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, bs.sbyte, 3);
           if ((b & 3) == 0) {
-            const int64_t j = c / 16;
+            // mma_scale_offset(r, j, kgroups): the tile part, then the row within the tile
             if ((j >> 2) < p.row.kgroups && r < rows_padded)
-              *reinterpret_cast<uint32_t*>(p.row.scales + mma_scale_offset(r, j, p.row.kgroups)) =
+              *reinterpret_cast<uint32_t*>(p.row.scales + sc_tile + ((rl & 31) << 4) + (((rl >> 5) & 3) << 2)) =
                   bs.sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24);
           }
         } else if (r < rows && c < cols) {
@@ -375,8 +388,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
           const BlockScale bs = block_scale_tab(k ? mb : ma, S_col, rtab_col);
           uint4 w = make_uint4(0u, 0u, 0u, 0u);
           if (SR) {
+            // (c * rows + r_base + rl0) / 16, exact: rows and r_base + rl0 are multiples of 16
             const int64_t c = c_base + 2 * cp + k;
-            const uint64_t ctr = (uint64_t)(c * rows + r_base + rl0) >> 4;
+            const uint64_t ctr = (uint64_t)c * (uint64_t)(rows >> 4) + (uint64_t)((r_base + rl0) >> 4);
             w = philox4x32_10_rk(make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), 1u, p.offset), p.rk);
           }
           uint32_t lo = encode8<SR>(v, bs.r, w.x, w.y);
