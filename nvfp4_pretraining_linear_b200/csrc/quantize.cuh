@@ -234,6 +234,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   }
   const float* rtab_row = reinterpret_cast<const float*>(smem + kQStages * kTileBytes + 256);
   const float* rtab_col = rtab_row + 128;
+  const float K_row = AMAX ? 0.0f : fast_scale_factor(S_row), K_col = AMAX ? 0.0f : fast_scale_factor(S_col);
   float m_raw = 0.0f, m_col = 0.0f, m_row = 0.0f;
   const int64_t nblk_row = cols / 16, nblk_col = rows / 16;
   const int64_t rows_padded = (rows + 127) & ~int64_t(127);
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
         tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 16));
       }
       BlockScale tbs;
-      if (TD && !AMAX) tbs = block_scale_tab(tile_max, S_row, rtab_row);
+      if (TD && !AMAX) tbs = block_scale_tab(tile_max, S_row, rtab_row);   // one per 16 x 16 tile
       // This lane's row advances by 4 per step: its Philox counter ((r * cols + c) / 16,
       // exact since cols and c are multiples of 16), its code address and the tile part
       // of its scale offset are set up once per tile and advanced by additions.
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
             continue;
           }
         }
-        const BlockScale bs = TD ? tbs : block_scale_tab(absmax16(v), S_row, rtab_row);
+        const BlockScale bs = TD ? tbs : block_scale_fast(absmax16(v), S_row, K_row, rtab_row);
         uint4 w = make_uint4(0u, 0u, 0u, 0u);
         if (SR) {
           const uint64_t ctr = ctr0 + (uint64_t)it * ctr_step;
@@ -385,7 +386,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const float* v = k ? vb : va;
-          const BlockScale bs = block_scale_tab(k ? mb : ma, S_col, rtab_col);
+          const BlockScale bs = TD ? block_scale_tab(k ? mb : ma, S_col, rtab_col)
+                                   : block_scale_fast(k ? mb : ma, S_col, K_col, rtab_col);
           uint4 w = make_uint4(0u, 0u, 0u, 0u);
           if (SR) {
             // (c * rows + r_base + rl0) / 16, exact: rows and r_base + rl0 are multiples of 16

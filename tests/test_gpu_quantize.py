@@ -167,3 +167,43 @@ def test_2d_weight_col_is_exact_transpose():
     assert rS == cS
     assert np.array_equal(O.unpack_codes(rc).T, O.unpack_codes(cc))
     assert np.array_equal(np.repeat(rs[::16, :].T, 16, axis=0), cs)
+
+
+def near_midpoint_blocks(rows, cols, amax, seed):
+    """BF16-valued FP32 [rows x cols] whose 16-element row blocks each have a maximum b
+    close to 6 * S * m for an E4M3 rounding midpoint m (S = fl(amax / 2688), set by one
+    element equal to amax): the BF16 value nearest 6 S m, or one up to 4 BF16 steps away,
+    so that the block scale fl(fl(b / 6) / S) lands on or within a few FP32 ulps of the
+    place where its E4M3 rounding changes."""
+    rng = np.random.default_rng(seed)
+    S = float(np.float32(np.float32(amax) / np.float32(2688.0)))
+    mids = [(1.0 + (2 * k + 1) / 16.0) * 2.0 ** e for e in range(-6, 9) for k in range(8)]
+    mids = [m for m in mids if m < 448.0] + [(k + 0.5) * 2.0 ** -9 for k in range(8)]   # + subnormal midpoints
+    nb = rows * cols // 16
+    x = np.empty((nb, 16), dtype=np.float32)
+    for i in range(nb):
+        b = O.bf16_round(np.array([6.0 * S * mids[i % len(mids)]], dtype=np.float32))
+        bits = b.view(np.uint32).astype(np.int64) + 0x10000 * int(rng.integers(-4, 5))
+        bb = np.array([bits[0]], dtype=np.uint32).view(np.float32)[0]
+        row = np.empty(16, dtype=np.float32)
+        row[0] = bb if rng.random() < 0.5 else -bb
+        row[1:] = O.bf16_round((rng.uniform(-0.9, 0.9, 15) * bb).astype(np.float32))
+        rng.shuffle(row)
+        x[i] = row
+    x = x.reshape(rows, cols)
+    x[0, 0] = np.float32(amax)
+    return x
+
+
+@pytest.mark.parametrize("amax", [2688.0, 3008.0, 2688.0 * 2.0 ** -20, 0.01171875])
+@pytest.mark.parametrize("mode", ["rne_row_col", "sr_row", "2d"])
+def test_block_scales_near_e4m3_midpoints(amax, mode):
+    """Block maxima whose scales sit on or next to E4M3 rounding midpoints, with tensor
+    scales that are powers of two (S = 1 and 2^-20: exact ties) and general ones: the
+    block scale bytes, codes and tensor scales equal the oracle's bit for bit."""
+    x = torch.from_numpy(near_midpoint_blocks(256, 512, amax, seed=int(amax * 7) % 1000)).to(torch.bfloat16).cuda()
+    rq, cq, ref = run_both(x, mode)
+    if rq is not None:
+        assert_layout_equal(rq, ref["row"], mode + " row")
+    if cq is not None:
+        assert_layout_equal(cq, ref["col"], mode + " col")
