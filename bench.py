@@ -396,7 +396,7 @@ def measure_targets(fp4_burst, hbm):
     for mode, kw in TARGET_QUANT_MODES.items():
         ms = flushed_median_ms(lambda: api.quantize(x, out_row=rq, out_col=cq, **kw), flush)
         gbs = n * n * 5.125 / (ms * 1e-3) / 1e9
-        quant[mode] = {"ms": ms, "gbs": gbs, "frac_hbm_measured": gbs / hbm, "frac_hbm_nominal_8000": gbs / 8000.0}
+        quant[mode] = {"ms": ms, "gbs": gbs, "frac_hbm": gbs / hbm, "frac_hbm_nominal_8000": gbs / 8000.0}
     api.get_status()
     return {"gemm_16384": gemm,
             "quantizer_16384": dict(quant, bytes_per_elem="5.125 (two passes, row + col)", target_frac=0.70)}
@@ -564,7 +564,7 @@ def run_ours(args):
         if world == 1 and not args.no_targets:
             del linears
             torch.cuda.empty_cache()
-            line["targets"] = measure_targets(fp4_burst, hbm)
+            line["targets"] = dict(measure_targets(fp4_burst, hbm), peak_source=peak_src)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = time_oracle(args.cpu_seconds)
         print(json.dumps(line), flush=True)
