@@ -70,12 +70,22 @@ __device__ __forceinline__ void unpack8(const uint4& w, float* v) {
   v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
 }
 
-// Butterfly stages h = 1, 2, 4, 8 and the 1/4 normalisation over 16 values whose
-// signs were already applied (the transform of rht16 after its sign flips).
-// Stage 1 pairs neighbours, so it runs on scalars; after it, elements 2p and 2p+1
-// share register pair p, and stages 2, 4, 8 combine pairs p and p + h/2 lane by
-// lane with packed FP32 instructions (same operations, same order per element).
-__device__ __forceinline__ void wht16_scaled(float* v) {
+// Butterfly stages h = 1, 2, 4, 8 over 16 values whose signs were already applied:
+// the transform of rht16 after its sign flips, without the final 1/4.  Stage 1 pairs
+// neighbours, so it runs on scalars; after it, elements 2p and 2p+1 share register
+// pair p, and stages 2, 4, 8 combine pairs p and p + h/2 lane by lane with packed FP32
+// instructions (same operations, same order per element).
+//
+// The 1/4 is left to the caller because it is exact here and can be folded: every
+// input is a BF16 value, a multiple of 2^-133, and so is every rounded sum of such
+// values (a sum below 2^-109 in magnitude is exact, a larger one rounds to a multiple of
+// its ulp, itself a multiple of 2^-133).  A multiple of 2^-133 divided by 4 is a
+// multiple of 2^-135, which FP32 represents exactly, subnormal or not.  So with u the
+// unscaled output, fl(u / 4) = u / 4, max|u / 4| = max|u| / 4, and fl(fl(u / 4) r) =
+// fl(u (r / 4)) whenever r / 4 is itself exact (r >= 2^-124).  QUARTER applies the 1/4
+// here, on the packed pairs.
+template <bool QUARTER>
+__device__ __forceinline__ void wht16(float* v) {
   wht_stage<16>(v, 1);
   uint64_t pr[8];
 #pragma unroll
@@ -91,9 +101,13 @@ __device__ __forceinline__ void wht16_scaled(float* v) {
       }
     }
   }
-  const uint64_t quarter = f2_pack(0.25f, 0.25f);
+  if (QUARTER) {
+    const uint64_t quarter = f2_pack(0.25f, 0.25f);
 #pragma unroll
-  for (int p = 0; p < 8; ++p) f2_unpack(f2_mul(pr[p], quarter), v[2 * p], v[2 * p + 1]);
+    for (int p = 0; p < 8; ++p) pr[p] = f2_mul(pr[p], quarter);
+  }
+#pragma unroll
+  for (int p = 0; p < 8; ++p) f2_unpack(pr[p], v[2 * p], v[2 * p + 1]);
 }
 
 // Sign-flip mask for a word holding two BF16 elements that both have group index i.
@@ -109,6 +123,36 @@ __device__ __forceinline__ float absmax8(const float* v) {
 }
 
 __device__ __forceinline__ float absmax16(const float* v) { return fmaxf(absmax8(v), absmax8(v + 8)); }
+
+// Maxima of |x| over BF16 values still packed two to a word.  max.xorsign.abs.bf16x2
+// selects, in each half, the operand of larger magnitude (its sign bit, the XOR of
+// the operands' signs, is not used); a NaN operand yields the other one.  Being a
+// selection, it equals absmax16 of the unpacked values: the magnitude comes out
+// exact, and a final maximum with 0 gives 0 where every value was NaN, as fmaxf from 0
+// does.
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Both halves' maxima of 8 words (e.g. two columns of a block, one per half).
+__device__ __forceinline__ uint32_t bf16x2_absmax8(const uint32_t* w) {
+  const uint32_t a = bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3]));
+  const uint32_t b = bf16x2_absmax(bf16x2_absmax(w[4], w[5]), bf16x2_absmax(w[6], w[7]));
+  return bf16x2_absmax(a, b);
+}
+
+__device__ __forceinline__ float bf16_lo_abs(uint32_t m) { return __uint_as_float((m << 16) & 0x7FFFFFFFu); }
+__device__ __forceinline__ float bf16_hi_abs(uint32_t m) { return __uint_as_float(m & 0x7FFF0000u); }
+
+// absmax16 of the 16 BF16 values in h0, h1 (any order of the halves).
+__device__ __forceinline__ float absmax16_bf16(const uint4& h0, const uint4& h1) {
+  const uint32_t w[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+  uint32_t m = bf16x2_absmax8(w);
+  m = bf16x2_absmax(bf16x2_absmax(m, __byte_perm(m, 0u, 0x1032)), 0u);
+  return bf16_hi_abs(m);
+}
 
 template <bool SR>
 __device__ __forceinline__ uint32_t encode8(const float* v, float r, uint32_t w0, uint32_t w1) {
@@ -132,9 +176,10 @@ __device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* m
 // AMAX: first pass (maxima only).  Otherwise ER / EC emit the row / col layout,
 // SR stochastic rounding, RR / RC the transform on the row / col layout, TD
 // 16x16 blocks.
-template <bool AMAX, bool ER, bool EC, bool SR, bool RR, bool RC, bool TD>
-__global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
-    quant_tile_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ QuantParams p) {
+// FOLD: the col transform's 1/4 goes into the block maxima and encode multipliers
+// (see wht16) instead of onto the values.
+template <bool AMAX, bool ER, bool EC, bool SR, bool RR, bool RC, bool TD, bool FOLD>
+__device__ __forceinline__ void quant_tile(const CUtensorMap& xmap, const QuantParams& p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const uint32_t smem_base = smem_u32(smem);
@@ -261,10 +306,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
           const uint8_t* src = in + (cw * 16 + it * 4 + rsub) * kTileRowBytes + b * 32;
-          float v[16];
-          unpack8(*reinterpret_cast<const uint4*>(src + 16 * swap), v);
-          unpack8(*reinterpret_cast<const uint4*>(src + 16 * (1 - swap)), v + 8);
-          tile_max = fmaxf(tile_max, absmax16(v));
+          tile_max = fmaxf(tile_max, absmax16_bf16(*reinterpret_cast<const uint4*>(src + 16 * swap),
+                                                   *reinterpret_cast<const uint4*>(src + 16 * (1 - swap))));
         }
         tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 8));
         tile_max = fmaxf(tile_max, __shfl_xor_sync(0xFFFFFFFFu, tile_max, 16));
@@ -301,20 +344,22 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
           }
           if (AMAX) {
             m_raw = fmaxf(m_raw, absmax16(v));   // the sign flips leave |x| unchanged
-            wht16_scaled(v);
-            m_row = fmaxf(m_row, absmax16(v));
+            wht16<false>(v);
+            m_row = fmaxf(m_row, absmax16(v));   // unscaled: the 1/4 is applied at the end
             continue;
           }
-          wht16_scaled(v);
+          wht16<true>(v);
         } else {
+          if (AMAX) {
+            m_raw = fmaxf(m_raw, absmax16_bf16(h0, h1));
+            continue;
+          }
           unpack8(h0, v);
           unpack8(h1, v + 8);
-          if (AMAX) {
-            m_raw = fmaxf(m_raw, absmax16(v));
-            continue;
-          }
         }
-        const BlockScale bs = TD ? tbs : block_scale_fast(absmax16(v), S_row, K_row, rtab_row);
+        // (with stochastic rounding the packed maximum measured slower here)
+        const float bmax = (RR || SR) ? absmax16(v) : absmax16_bf16(h0, h1);
+        const BlockScale bs = TD ? tbs : block_scale_fast(bmax, S_row, K_row, rtab_row);
         uint4 w = make_uint4(0u, 0u, 0u, 0u);
         if (SR) {
           const uint64_t ctr = ctr0 + (uint64_t)it * ctr_step;
@@ -354,34 +399,50 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         const int rl0 = q * 32 + b * 16;
+        // maxima of the raw words: column a in the low halves, column b in the high
+        // halves (with stochastic rounding, unpacked maxima measured faster)
+        constexpr bool kPacked = AMAX || (!RC && !SR);
         float va[16], vb[16];
+        uint32_t wr[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           uint32_t w = *reinterpret_cast<const uint32_t*>(in + (rl0 + i) * kTileRowBytes + cp * 4);
+          if (kPacked) wr[i] = w;
           if (RC) w ^= pair_sign_mask(p.signs, i);        // element i of both column groups
           va[i] = bf16_lo(w);
           vb[i] = bf16_hi(w);
         }
-        if (AMAX) m_raw = fmaxf(m_raw, fmaxf(absmax16(va), absmax16(vb)));   // signs leave |x| unchanged
+        const uint32_t mab =
+            kPacked ? bf16x2_absmax(bf16x2_absmax(bf16x2_absmax8(wr), bf16x2_absmax8(wr + 8)), 0u) : 0u;
+        if (AMAX) m_raw = fmaxf(m_raw, fmaxf(bf16_lo_abs(mab), bf16_hi_abs(mab)));   // signs leave |x| unchanged
         if (RC) {
-          wht16_scaled(va);
-          wht16_scaled(vb);
+          wht16<!AMAX && !FOLD>(va);
+          wht16<!AMAX && !FOLD>(vb);
         }
         if (AMAX) {
-          m_col = fmaxf(m_col, fmaxf(absmax16(va), absmax16(vb)));
+          m_col = fmaxf(m_col, fmaxf(absmax16(va), absmax16(vb)));   // unscaled, as m_row
           continue;
         }
         float ma, mb;
         if (TD) {
           // the 16x16 tile spans the 8 lanes holding columns 16*(cp/8) .. +15
-          float m = fmaxf(absmax16(va), absmax16(vb));
+          float m = fmaxf(bf16_lo_abs(mab), bf16_hi_abs(mab));
           m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
           m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
           m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
           ma = mb = m;
         } else {
-          ma = absmax16(va);
-          mb = absmax16(vb);
+          if (kPacked) {
+            ma = bf16_lo_abs(mab);
+            mb = bf16_hi_abs(mab);
+          } else {
+            ma = absmax16(va);
+            mb = absmax16(vb);
+            if (RC && FOLD) {
+              ma *= 0.25f;
+              mb *= 0.25f;
+            }
+          }
         }
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
@@ -395,8 +456,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
             const uint64_t ctr = (uint64_t)c * (uint64_t)(rows >> 4) + (uint64_t)((r_base + rl0) >> 4);
             w = philox4x32_10_rk(make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), 1u, p.offset), p.rk);
           }
-          uint32_t lo = encode8<SR>(v, bs.r, w.x, w.y);
-          uint32_t hi = encode8<SR>(v + 8, bs.r, w.z, w.w);
+          const float r_enc = (RC && FOLD) ? 0.25f * bs.r : bs.r;
+          uint32_t lo = encode8<SR>(v, r_enc, w.x, w.y);
+          uint32_t hi = encode8<SR>(v + 8, r_enc, w.z, w.w);
           if (bs.r == 0.0f) lo = hi = 0u;
           codes[k][b][0] = lo;
           codes[k][b][1] = hi;
@@ -440,6 +502,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   }
 
   if (AMAX) {
+    m_col *= 0.25f;   // maxima of the unscaled transforms (exact, see wht16)
+    m_row *= 0.25f;
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) {
       m_raw = fmaxf(m_raw, __shfl_xor_sync(0xFFFFFFFFu, m_raw, s));
@@ -452,6 +516,23 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
       if (RC) atomicMax(p.amax_acc + 1, __float_as_uint(m_col));
       if (RR) atomicMax(p.amax_acc + 2, __float_as_uint(m_row));
     }
+  }
+}
+
+template <bool AMAX, bool ER, bool EC, bool SR, bool RR, bool RC, bool TD>
+__global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
+    quant_tile_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ QuantParams p) {
+  if constexpr (RC && !AMAX && !SR) {
+    // The fold is exact when r / 4 is, for every encode multiplier r of the tensor: r
+    // >= 1 / (448 S) stays far above 2^-124 for S <= 2^100 (the same decision in every
+    // CTA).  With stochastic rounding the fold measured slower, so those modes keep the
+    // 1/4 on the values.
+    if (tensor_scale_from_amax(p.amax[1]) <= 0x1p100f)
+      quant_tile<AMAX, ER, EC, SR, RR, RC, TD, true>(xmap, p);
+    else
+      quant_tile<AMAX, ER, EC, SR, RR, RC, TD, false>(xmap, p);
+  } else {
+    quant_tile<AMAX, ER, EC, SR, RR, RC, TD, false>(xmap, p);
   }
 }
 

@@ -207,3 +207,24 @@ def test_block_scales_near_e4m3_midpoints(amax, mode):
         assert_layout_equal(rq, ref["row"], mode + " row")
     if cq is not None:
         assert_layout_equal(cq, ref["col"], mode + " col")
+
+
+@pytest.mark.parametrize("above", [False, True])
+@pytest.mark.parametrize("mode", ["rne_row_rhtcol", "sr_row_rhtcol", "sr_rht_both"])
+def test_rht_quarter_fold_boundary(above, mode):
+    """The transform's 1/4 is folded into the block maximum and the encode multiplier
+    while the tensor scale S is at most 2^100, and applied to the values above it.
+    Tensors with S = 2^100 exactly (maximum 2688 * 2^100) and with the next BF16
+    maximum up, their values spread over 160 binades, equal the oracle bit for bit on
+    both sides of the switch."""
+    rng = np.random.default_rng(31 + int(above))
+    x = rng.standard_normal((256, 384)) * np.exp2(rng.integers(-60, 100, (256, 384)).astype(np.float64))
+    x = O.bf16_round(x.astype(np.float32))
+    amax = np.array([2688.0 * 2.0 ** 100], dtype=np.float32)
+    if above:
+        amax = (amax.view(np.uint32) + np.uint32(0x10000)).view(np.float32)
+    x[7, 9] = amax[0]
+    assert np.abs(x).max() == amax[0]
+    rq, cq, ref = run_both(torch.from_numpy(x).to(torch.bfloat16).cuda(), mode)
+    assert_layout_equal(rq, ref["row"], mode + " row")
+    assert_layout_equal(cq, ref["col"], mode + " col")
