@@ -317,6 +317,16 @@ __device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t j, int64_
 
 // ----------------------------------------------------------------- PTX wrappers
 
+// Programmatic dependent launch: a kernel launched as a programmatic dependent of
+// the one before it in the stream may start once every CTA of that one has called
+// griddep_launch_dependents (or exited); griddep_wait then blocks until that kernel
+// has completed and its memory operations are visible.  In a normal launch the wait
+// returns at once.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }

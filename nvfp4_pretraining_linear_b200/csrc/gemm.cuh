@@ -741,6 +741,11 @@ __global__ void __launch_bounds__(P_NUM_THREADS, 1)
   cluster_sync();                                     // barriers of both CTAs initialised
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The launch may be a programmatic dependent of the kernel before it in the stream:
+  // nothing above touches global memory, and every role below starts after that
+  // kernel has completed.  A dependent of this kernel may start as its CTAs leave.
+  griddep_launch_dependents();
+  griddep_wait();
 
   const int32_t num_tiles = grp.tile_end[grp.count - 1];
   const int32_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;

@@ -233,50 +233,69 @@ int64_t injected_gemm_skip_stage() {
   return (end && *end == '\0' && n >= 0) ? (int64_t)n : -1;
 }
 
+// A quantise pass that directly follows its own amax pass in the stream is launched
+// as a programmatic dependent of it (after_amax): it loads its first tiles while the
+// amax pass finishes and waits for it before reading the maxima.
 template <bool AM, bool ER, bool EC, bool SR, bool RR, bool RC, bool TD>
-cudaError_t launch_tiles(const CUtensorMap& map, const nvfp4::QuantParams& p, int grid, cudaStream_t s) {
+cudaError_t launch_tiles(const CUtensorMap& map, const nvfp4::QuantParams& p, int grid, cudaStream_t s,
+                         bool after_amax = false) {
   static bool done[kMaxDevices] = {};
   static std::mutex m;
   auto kernel = nvfp4::quant_tile_kernel<AM, ER, EC, SR, RR, RC, TD>;
   cudaError_t e = ensure_smem(kernel, nvfp4::kQSmemBytes, done, m);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, nvfp4::kQThreads, nvfp4::kQSmemBytes, s>>>(map, p);
-  return cudaGetLastError();
+  if (!after_amax) {
+    kernel<<<grid, nvfp4::kQThreads, nvfp4::kQSmemBytes, s>>>(map, p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(nvfp4::kQThreads);
+  cfg.dynamicSmemBytes = nvfp4::kQSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, map, p);
 }
 
 template <bool ER, bool EC, bool SR, bool RR, bool RC>
-cudaError_t dispatch_td(bool td, const CUtensorMap& m, const nvfp4::QuantParams& p, int g, cudaStream_t s) {
+cudaError_t dispatch_td(bool td, const CUtensorMap& m, const nvfp4::QuantParams& p, int g, cudaStream_t s, bool dep) {
   if constexpr (!SR && !RR && !RC) {
-    if (td) return launch_tiles<false, ER, EC, false, false, false, true>(m, p, g, s);
+    if (td) return launch_tiles<false, ER, EC, false, false, false, true>(m, p, g, s, dep);
   }
-  return launch_tiles<false, ER, EC, SR, RR, RC, false>(m, p, g, s);
+  return launch_tiles<false, ER, EC, SR, RR, RC, false>(m, p, g, s, dep);
 }
 
 template <bool ER, bool EC, bool SR, bool RR>
-cudaError_t dispatch_rc(bool rc, bool td, const CUtensorMap& m, const nvfp4::QuantParams& p, int g, cudaStream_t s) {
-  if (rc) return dispatch_td<ER, EC, SR, RR, true>(td, m, p, g, s);
-  return dispatch_td<ER, EC, SR, RR, false>(td, m, p, g, s);
+cudaError_t dispatch_rc(bool rc, bool td, const CUtensorMap& m, const nvfp4::QuantParams& p, int g, cudaStream_t s,
+                        bool dep) {
+  if (rc) return dispatch_td<ER, EC, SR, RR, true>(td, m, p, g, s, dep);
+  return dispatch_td<ER, EC, SR, RR, false>(td, m, p, g, s, dep);
 }
 
 template <bool ER, bool EC, bool SR>
 cudaError_t dispatch_rr(bool rr, bool rc, bool td, const CUtensorMap& m, const nvfp4::QuantParams& p, int g,
-                        cudaStream_t s) {
-  if (rr) return dispatch_rc<ER, EC, SR, true>(rc, td, m, p, g, s);
-  return dispatch_rc<ER, EC, SR, false>(rc, td, m, p, g, s);
+                        cudaStream_t s, bool dep) {
+  if (rr) return dispatch_rc<ER, EC, SR, true>(rc, td, m, p, g, s, dep);
+  return dispatch_rc<ER, EC, SR, false>(rc, td, m, p, g, s, dep);
 }
 
 template <bool ER, bool EC>
 cudaError_t dispatch_sr(bool sr, bool rr, bool rc, bool td, const CUtensorMap& m, const nvfp4::QuantParams& p, int g,
-                        cudaStream_t s) {
-  if (sr) return dispatch_rr<ER, EC, true>(rr, rc, td, m, p, g, s);
-  return dispatch_rr<ER, EC, false>(rr, rc, td, m, p, g, s);
+                        cudaStream_t s, bool dep) {
+  if (sr) return dispatch_rr<ER, EC, true>(rr, rc, td, m, p, g, s, dep);
+  return dispatch_rr<ER, EC, false>(rr, rc, td, m, p, g, s, dep);
 }
 
+// dep: the quantise pass follows its own amax pass in the stream (see launch_tiles).
 cudaError_t dispatch_quant(bool er, bool ec, bool sr, bool rr, bool rc, bool td, const CUtensorMap& m,
-                           const nvfp4::QuantParams& p, int g, cudaStream_t s) {
-  if (er && ec) return dispatch_sr<true, true>(sr, rr, rc, td, m, p, g, s);
-  if (er) return dispatch_sr<true, false>(sr, rr, rc, td, m, p, g, s);
-  return dispatch_sr<false, true>(sr, rr, rc, td, m, p, g, s);
+                           const nvfp4::QuantParams& p, int g, cudaStream_t s, bool dep) {
+  if (er && ec) return dispatch_sr<true, true>(sr, rr, rc, td, m, p, g, s, dep);
+  if (er) return dispatch_sr<true, false>(sr, rr, rc, td, m, p, g, s, dep);
+  return dispatch_sr<false, true>(sr, rr, rc, td, m, p, g, s, dep);
 }
 
 cudaError_t dispatch_amax(bool rr, bool rc, const CUtensorMap& m, const nvfp4::QuantParams& p, int g, cudaStream_t s) {
@@ -431,7 +450,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
   p.amax_acc = nullptr;
   p.skip_tile = injected_skip_tile();
   e = dispatch_quant(out_row != nullptr, out_col != nullptr, opts->stochastic != 0, opts->rht_row != 0,
-                     opts->rht_col != 0, opts->block_2d != 0, map, p, grid, s);
+                     opts->rht_col != 0, opts->block_2d != 0, map, p, grid, s, opts->amax_in == nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return NVFP4_OK;
 }
@@ -505,21 +524,25 @@ nvfp4_status pair_problem(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C,
 }
 
 // Launch configuration of the pair kernel: clusters of 2 CTAs, one pair per two SMs up to
-// the co-resident maximum, never more pairs than tiles.
-void pair_launch_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, int64_t tiles, int pair_clusters,
+// the co-resident maximum, never more pairs than tiles.  It is a programmatic dependent
+// of the kernel before it in the stream (attr[1]): its set-up overlaps that kernel's
+// last CTAs, and it waits for that kernel before touching global memory.
+void pair_launch_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute (&attr)[2], int64_t tiles, int pair_clusters,
                         cudaStream_t s) {
   std::memset(cfg, 0, sizeof(*cfg));
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   const int pairs = (int)std::min<int64_t>(tiles, pair_clusters);
   cfg->gridDim = dim3(2 * pairs, 1, 1);
   cfg->blockDim = dim3(nvfp4::gemm::P_NUM_THREADS, 1, 1);
   cfg->dynamicSmemBytes = nvfp4::gemm::P_SMEM_BYTES;
   cfg->stream = s;
   cfg->attrs = attr;
-  cfg->numAttrs = 1;
+  cfg->numAttrs = 2;
 }
 
 // nvfp4_gemm; with amax_out (3 floats) the maxima of nvfp4_gemm_amax; with a low-rank
@@ -616,7 +639,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor* A, const nvfp4_tensor* B, void* C, in
                   : f32 ? (accumulate ? gemm_kernel_pair<EPI_F32_ACC, 1, false> : gemm_kernel_pair<EPI_F32, 1, false>)
                         : (accumulate ? gemm_kernel_pair<EPI_BF16_ACC, 1, false> : gemm_kernel_pair<EPI_BF16, 1, false>);
     cudaLaunchConfig_t cfg;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     pair_launch_config(&cfg, attr, grp.tile_end[0], dev->pair_clusters, s);
     e = cudaLaunchKernelEx(&cfg, kernel, grp);
   } else {
@@ -729,7 +752,7 @@ nvfp4_status nvfp4_gemm_grouped(const nvfp4_tensor* const* A, const nvfp4_tensor
   auto kernel = out_dtype == NVFP4_OUT_F32 ? gemm_kernel_pair<EPI_F32, kMaxGroup, false>
                                                  : gemm_kernel_pair<EPI_BF16, kMaxGroup, false>;
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   pair_launch_config(&cfg, attr, tiles, dev->pair_clusters, static_cast<cudaStream_t>(stream));
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, grp);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "grouped gemm launch");

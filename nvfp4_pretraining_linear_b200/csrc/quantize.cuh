@@ -173,85 +173,15 @@ __device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* m
       : "memory");
 }
 
-// AMAX: first pass (maxima only).  Otherwise ER / EC emit the row / col layout,
-// SR stochastic rounding, RR / RC the transform on the row / col layout, TD
-// 16x16 blocks.
-// FOLD: the col transform's 1/4 goes into the block maxima and encode multipliers
-// (see wht16) instead of onto the values.
+// The compute warps' part of quant_tile_kernel.  FOLD: the col transform's 1/4 goes
+// into the block maxima and encode multipliers (see wht16) instead of onto the values.
 template <bool AMAX, bool ER, bool EC, bool SR, bool RR, bool RC, bool TD, bool FOLD>
-__device__ __forceinline__ void quant_tile(const CUtensorMap& xmap, const QuantParams& p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  const uint32_t smem_base = smem_u32(smem);
-  const uint32_t bar_base = smem_base + kQStages * kTileBytes;
+__device__ __forceinline__ void quant_compute(const QuantParams& p, uint8_t* smem) {
+  const uint32_t bar_base = smem_u32(smem) + kQStages * kTileBytes;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kQStages * kTileBytes + 8 * 2 * kQStages);
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (kQStages + s); };
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kQStages; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), kQComputeWarps);
-    }
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  }
-  __syncthreads();
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    // The whole warp runs the loop; one elected lane arms the barrier and issues the copy.
-    {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool issued[kQStages] = {};
-      uint32_t issued_phase[kQStages] = {};
-      bool ok = true;
-      for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x) {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag))) {
-          ok = false;
-          break;
-        }
-        const int64_t tr = t / p.tiles_c, tc = t - tr * p.tiles_c;
-        if (t == p.skip_tile) {
-          // fault injection: this stage's data never arrives, so the compute warps'
-          // bounded wait on it expires and records kErrTimeout; nothing is in flight
-          issued[stage] = false;
-          if (++stage == kQStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-          continue;
-        }
-        if (elect_one()) {
-          mbar_arrive_expect_tx(full_bar(stage), kTileBytes);
-          tma_load_tile(smem_base + stage * kTileBytes, &xmap, (int32_t)(tc * kTileCols), (int32_t)(tr * kTileRows),
-                        full_bar(stage));
-        }
-        __syncwarp();
-        issued[stage] = true;
-        issued_phase[stage] = phase;
-        if (++stage == kQStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      if (!ok) {
-        // wind down: let every load already issued land before the CTA exits
-        for (int s = 0; s < kQStages; ++s) {
-          if (!issued[s]) continue;
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(full_bar(s), issued_phase[s]) && globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
-        }
-      }
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------ compute warps
   const int cw = warp - 1;                 // 0..7
   const int ct = threadIdx.x - 32;         // 0..255
   const int64_t rows = p.rows, cols = p.cols;
@@ -519,20 +449,106 @@ __device__ __forceinline__ void quant_tile(const CUtensorMap& xmap, const QuantP
   }
 }
 
+
+// AMAX: first pass (maxima only).  Otherwise ER / EC emit the row / col layout,
+// SR stochastic rounding, RR / RC the transform on the row / col layout, TD
+// 16x16 blocks.
+//
+// Launch order.  Both passes let the kernel that follows them in the stream start
+// early (griddepcontrol.launch_dependents).  The quantise pass is launched as a
+// programmatic dependent of its own amax pass, which itself starts only after all
+// earlier work: its producer streams the first tiles of x (which the amax pass does
+// not write) while the amax pass finishes, and its compute warps wait for the amax
+// pass (griddepcontrol.wait, a no-op in a normal launch) before they read the maxima
+// or write anything.  A GEMM that follows waits likewise before touching memory.
 template <bool AMAX, bool ER, bool EC, bool SR, bool RR, bool RC, bool TD>
 __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     quant_tile_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ QuantParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_base = smem_base + kQStages * kTileBytes;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kQStages * kTileBytes + 8 * 2 * kQStages);
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (kQStages + s); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), kQComputeWarps);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    // The whole warp runs the loop; one elected lane arms the barrier and issues the copy.
+    {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued[kQStages] = {};
+      uint32_t issued_phase[kQStages] = {};
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag))) {
+          ok = false;
+          break;
+        }
+        const int64_t tr = t / p.tiles_c, tc = t - tr * p.tiles_c;
+        if (t == p.skip_tile) {
+          // fault injection: this stage's data never arrives, so the compute warps'
+          // bounded wait on it expires and records kErrTimeout; nothing is in flight
+          issued[stage] = false;
+          if (++stage == kQStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          continue;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(full_bar(stage), kTileBytes);
+          tma_load_tile(smem_base + stage * kTileBytes, &xmap, (int32_t)(tc * kTileCols), (int32_t)(tr * kTileRows),
+                        full_bar(stage));
+        }
+        __syncwarp();
+        issued[stage] = true;
+        issued_phase[stage] = phase;
+        if (++stage == kQStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        // wind down: let every load already issued land before the CTA exits
+        for (int s = 0; s < kQStages; ++s) {
+          if (!issued[s]) continue;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(full_bar(s), issued_phase[s]) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  if (!AMAX) griddep_wait();
   if constexpr (RC && !AMAX && !SR) {
     // The fold is exact when r / 4 is, for every encode multiplier r of the tensor: r
     // >= 1 / (448 S) stays far above 2^-124 for S <= 2^100 (the same decision in every
     // CTA).  With stochastic rounding the fold measured slower, so those modes keep the
     // 1/4 on the values.
     if (tensor_scale_from_amax(p.amax[1]) <= 0x1p100f)
-      quant_tile<AMAX, ER, EC, SR, RR, RC, TD, true>(xmap, p);
+      quant_compute<AMAX, ER, EC, SR, RR, RC, TD, true>(p, smem);
     else
-      quant_tile<AMAX, ER, EC, SR, RR, RC, TD, false>(xmap, p);
+      quant_compute<AMAX, ER, EC, SR, RR, RC, TD, false>(p, smem);
   } else {
-    quant_tile<AMAX, ER, EC, SR, RR, RC, TD, false>(xmap, p);
+    quant_compute<AMAX, ER, EC, SR, RR, RC, TD, false>(p, smem);
   }
 }
 
