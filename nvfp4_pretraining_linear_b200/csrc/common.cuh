@@ -174,12 +174,6 @@ __device__ __forceinline__ uint4 philox4x32_10_rk(uint4 c, const uint32_t* rk) {
 }
 
 
-// ----------------------------------------------------------------- Hadamard
-
-__device__ __forceinline__ float flip_sign(float v, uint32_t bit) {
-  return __uint_as_float(__float_as_uint(v) ^ (bit << 31));
-}
-
 // ----------------------------------------------------------------- packed FP32 pairs
 //
 // sm_100 executes two FP32 additions or multiplications as one instruction on a
@@ -214,6 +208,8 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return r;
 }
 
+// ----------------------------------------------------------------- Hadamard
+
 // Butterfly stage h over N values held in registers: (v[i], v[i+h]) <- (v[i]+v[i+h], v[i]-v[i+h]).
 template <int N>
 __device__ __forceinline__ void wht_stage(float* v, int h) {
@@ -225,18 +221,6 @@ __device__ __forceinline__ void wht_stage(float* v, int h) {
       v[i + h] = __fsub_rn(a, b);
     }
   }
-}
-
-// Signed, normalised 16-point Walsh-Hadamard transform of v[0..15] (natural order).
-__device__ __forceinline__ void rht16(float* v, uint32_t signs) {
-#pragma unroll
-  for (int j = 0; j < 16; ++j) v[j] = flip_sign(v[j], (signs >> j) & 1u);
-  wht_stage<16>(v, 1);
-  wht_stage<16>(v, 2);
-  wht_stage<16>(v, 4);
-  wht_stage<16>(v, 8);
-#pragma unroll
-  for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], 0.25f);
 }
 
 // ----------------------------------------------------------------- scales

@@ -70,8 +70,9 @@ __device__ __forceinline__ void unpack8(const uint4& w, float* v) {
   v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
 }
 
-// Butterfly stages h = 1, 2, 4, 8 over 16 values whose signs were already applied:
-// the transform of rht16 after its sign flips, without the final 1/4.  Stage 1 pairs
+// Butterfly stages h = 1, 2, 4, 8 (natural order: v[i], v[i+h] <- v[i]+v[i+h],
+// v[i]-v[i+h]) over 16 values whose random signs were already applied: the signed
+// 16-point Walsh-Hadamard transform, without its final 1/4.  Stage 1 pairs
 // neighbours, so it runs on scalars; after it, elements 2p and 2p+1 share register
 // pair p, and stages 2, 4, 8 combine pairs p and p + h/2 lane by lane with packed FP32
 // instructions (same operations, same order per element).
