@@ -76,3 +76,60 @@ def test_quantise_reads_input_written_just_before():
     for i, q in enumerate(outs):
         assert same_bytes(q, refs[i % 4]), i
     api.get_status()
+
+
+def test_step_captured_in_cuda_graph_matches_eager():
+    """The linear step's calls captured into a CUDA graph (the memsets become graph
+    nodes, the programmatic-dependent launches programmatic edges) and replayed give
+    the bytes of the eager calls, and a replay after the input is rewritten in place
+    follows the new values."""
+    M, K, N = 1024, 768, 1280
+    x = synthetic.normal((M, K), 1.0, seed=81, device="cuda", outlier_frac=0.001, outlier_mult=100.0)
+    x2 = synthetic.normal((M, K), 1.0, seed=82, device="cuda", outlier_frac=0.001, outlier_mult=100.0)
+    w = synthetic.normal((N, K), 0.02, seed=83, device="cuda")
+    dy = synthetic.normal((M, N), 1e-3, seed=84, device="cuda")
+    E = api.QTensor.empty
+    q = [E(N, K), E(K, N), E(M, K), E(K, M), E(M, N), E(N, M)]     # Wq, Xq, dYq: row, col
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+
+    def step():
+        api.quantize(w, emit_row=True, emit_col=True, block_2d=True, out_row=q[0], out_col=q[1])
+        api.quantize(x, emit_row=True, emit_col=True, rht_col=True, rht_signs=SIGNS, out_row=q[2], out_col=q[3])
+        api.gemm(q[2], q[0], out=y)
+        api.quantize(dy, emit_row=True, emit_col=True, stochastic=True, rht_col=True, seed=5, offset=2,
+                     rht_signs=SIGNS, out_row=q[4], out_col=q[5])
+        api.gemm(q[4], q[1], out=dx)
+        api.gemm(q[5], q[3], out=dw)
+
+    def snapshot():
+        torch.cuda.synchronize()
+        return ([(t.codes.clone(), t.scales.clone(), t.tensor_scale.clone()) for t in q],
+                [y.clone(), dx.clone(), dw.clone()])
+
+    def same(a, b):
+        return all(all(torch.equal(u, v) for u, v in zip(ta, tb)) for ta, tb in zip(a[0], b[0])) and \
+            all(torch.equal(u, v) for u, v in zip(a[1], b[1]))
+
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        step()                                   # eager; also creates stream s's workspace
+    ref = snapshot()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    for t in q:
+        t.codes.fill_(0x5A)
+        t.scales.fill_(0x33)
+    y.fill_(7.0)
+    g.replay()
+    assert same(snapshot(), ref)
+    x.copy_(x2)
+    g.replay()
+    replayed = snapshot()
+    with torch.cuda.stream(s):
+        step()
+    assert same(replayed, snapshot())
+    assert not torch.equal(replayed[1][0], ref[1][0])      # the new input did reach the output
+    api.get_status()
