@@ -275,17 +275,19 @@ __device__ __forceinline__ float fast_scale_factor(float S) {
 
 // block_scale_tab with one multiply where that provably gives the same byte.
 // s_a = fl(b K) carries three roundings of at most 2^-24 relative each, s = fl(fl(b / 6)
-// / S) two (b >= 2^-120 keeps b / 6 normal), so they are within 5 ulps of s_a of each
-// other.  E4M3 rounding changes only at the midpoints between its values; for s_a in
-// E4M3's normal range (>= 2^-6), a midpoint is where the 20 FP32 mantissa bits below
-// E4M3's 3 are exactly 0x80000.  If those bits of s_a are more than 16 away from it, s
-// rounds to the byte s_a rounds to (values above 448 saturate either way).  Otherwise
-// -- and for K = 0, tiny b or s_a below 2^-6 -- the two divisions are done.
+// / S) two (b / 6 normal, below), so they are within 5 ulps of s_a of each other.  E4M3
+// rounding changes only at the midpoints between its values; for s_a in E4M3's normal
+// range (>= 2^-6), a midpoint is where the 20 FP32 mantissa bits below E4M3's 3 are
+// exactly 0x80000.  If those bits of s_a are more than 16 away from it, s rounds to the
+// byte s_a rounds to (values above 448 saturate either way).  Otherwise -- and for s_a
+// below 2^-6 or not a number -- the two divisions are done.  s_a >= 2^-6 also implies
+// K != 0 (K = 0 gives s_a = 0 or NaN) and, as K = 0 unless S >= 2^-100,
+// b >= 2^-6 * 6 S * (1 - 2^-22) > 2^-104, which keeps b / 6 normal.
 __device__ __forceinline__ BlockScale block_scale_fast(float bmax, float S, float K, const float* rtab) {
   const float sa = __fmul_rn(bmax, K);
   const int dm = (int)(__float_as_uint(sa) & 0xFFFFFu) - 0x80000;
   float s = sa;
-  if (!(K != 0.0f && bmax >= 0x1p-120f && sa >= 0x1p-6f && (dm > 16 || dm < -16)))
+  if (!(sa >= 0x1p-6f && (uint32_t)(dm + 16) > 32u))   // |dm| > 16
     s = __fdiv_rn(__fdiv_rn(bmax, 6.0f), S);
   BlockScale out;
   out.sbyte = e4m3_encode_hw(s);
