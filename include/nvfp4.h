@@ -23,8 +23,9 @@
  *     as usual: the GEMMs and the quantiser's second pass are launched as
  *     programmatic dependents of the kernel before them, so their set-up overlaps
  *     that kernel's last thread blocks, but each waits for it to complete before
- *     touching memory (the second pass reads only the input of its own first pass
- *     earlier).  Every call may be captured into a CUDA graph.
+ *     touching memory; the one exception, the second pass streaming its input
+ *     early, reads a tensor that its own first pass only reads.  Every call may be
+ *     captured into a CUDA graph.
  *   - Argument errors are reported synchronously by the return value, before
  *     anything is launched.  Device-side errors (a bounded wait that gave up)
  *     are reported by nvfp4_get_status().  No exception crosses the ABI.
