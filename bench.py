@@ -50,13 +50,40 @@ SR_SEED = 1234
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def load_peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
+def _peak_number(v):
+    """A peak figure from MEASURED_PEAKS.json: a number, or a record holding one."""
+    if isinstance(v, bool):
+        return None
+    if isinstance(v, (int, float)):
+        return float(v) if v > 0 else None
+    if isinstance(v, dict):
+        for k in ("value", "median", "mean", "gbs", "tflops"):
+            if k in v:
+                return _peak_number(v[k])
+    return None
+
+
+def load_peaks(path=None):
+    """The roofline denominators: MEASURED_PEAKS.json where it holds them (per key),
+    else the fallback figures; the source says which."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
         with open(path) as f:
             d = json.load(f)
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+    peaks, missing = {}, []
+    for key, fb in FALLBACK_PEAKS.items():
+        v = _peak_number(d.get(key)) if isinstance(d, dict) else None
+        if v is None:
+            missing.append(key)
+            v = fb
+        peaks[key] = v
+    if not missing:
+        return peaks, "measured"
+    if len(missing) == len(FALLBACK_PEAKS):
+        return peaks, "fallback"
+    return peaks, "measured (fallback for %s)" % ", ".join(missing)
 
 
 def dist_env():

@@ -63,3 +63,21 @@ def test_gpus_flag_must_match_the_launched_world():
                          env=dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0"))
     assert res.returncode != 0
     assert "WORLD_SIZE is 1" in res.stderr
+
+
+def test_peaks_file_forms(tmp_path):
+    """MEASURED_PEAKS.json may hold plain numbers or records; anything unusable falls
+    back per key, and the source names it."""
+    import json
+    import bench
+    p = tmp_path / "peaks.json"
+    assert bench.load_peaks(str(tmp_path / "absent.json")) == (bench.FALLBACK_PEAKS, "fallback")
+    p.write_text(json.dumps({"hbm_gbs": 6538.0, "bf16_tflops": 1638, "bf16_tflops_sustained": 1372.5}))
+    peaks, src = bench.load_peaks(str(p))
+    assert src == "measured" and peaks == {"hbm_gbs": 6538.0, "bf16_tflops": 1638.0, "bf16_tflops_sustained": 1372.5}
+    p.write_text(json.dumps({"hbm_gbs": {"value": 6500}, "bf16_tflops": "n/a", "clocks": {"sm": 1965}}))
+    peaks, src = bench.load_peaks(str(p))
+    assert peaks["hbm_gbs"] == 6500.0 and peaks["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    assert src == "measured (fallback for bf16_tflops, bf16_tflops_sustained)"
+    p.write_text("not json")
+    assert bench.load_peaks(str(p))[1] == "fallback"
